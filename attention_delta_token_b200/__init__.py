@@ -1,0 +1,224 @@
+"""FOCUS importance-delta token eviction on B200 (sm_100a).
+
+A thin Python binding over the C ABI of ``libfocus.so`` (declared in
+``include/focus.h``).  Every function here only checks and marshals its
+arguments (torch CUDA tensors -> raw device pointers, the current CUDA stream)
+and calls the C entry point of the same name; all arithmetic of the eviction
+step runs in the library's CUDA kernels.  There is no CPU fallback: if the
+library is missing, importing this package raises.
+
+Method: "FOCUS: DLLMs Know How to Tame Their Compute Bound" (pith.science review
+page), "What carries the argument" and the Figure 5 caption.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "FocusError", "FocusDims", "make_dims", "focus_workspace_size", "Workspace",
+    "focus_clear_device_status", "focus_read_device_status", "focus_attn_stats",
+    "focus_importance_delta", "focus_topk_select", "focus_compact", "focus_evict",
+    "focus_status_string", "focus_abi_version", "focus_set_trace_events", "plan_capacity",
+    "LIB_PATH", "STATUS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfocus.so")
+
+STATUS = {
+    0: "FOCUS_OK", 1: "FOCUS_ERR_INVALID_ARGUMENT", 2: "FOCUS_ERR_UNSUPPORTED_SHAPE",
+    3: "FOCUS_ERR_CAPACITY", 4: "FOCUS_ERR_WORKSPACE", 5: "FOCUS_ERR_CUDA",
+    6: "FOCUS_ERR_DEVICE_CHECK", 7: "FOCUS_ERR_TIMEOUT",
+}
+
+
+class FocusError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {STATUS.get(self.status, self.status)}")
+
+
+class FocusDims(ctypes.Structure):
+    _fields_ = [("R", ctypes.c_int32), ("B", ctypes.c_int32), ("Hq", ctypes.c_int32),
+                ("Hkv", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("hidden", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float), ("pool_window", ctypes.c_int32)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing; build it with `python attention_delta_token_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+    D = ctypes.POINTER(FocusDims)
+    sig = {
+        "focus_workspace_size": (sz, [D]),
+        "focus_clear_device_status": (ctypes.c_int, [P, sz, P]),
+        "focus_read_device_status": (ctypes.c_int, [P, P, ctypes.c_int]),
+        "focus_attn_stats": (ctypes.c_int, [D, P, P, P, i64, P, P, P, sz, P]),
+        "focus_importance_delta": (ctypes.c_int, [D, P, P, P, P, P, P]),
+        "focus_topk_select": (ctypes.c_int, [D, P, P, P, P, P, i64, P, sz, P]),
+        "focus_compact": (ctypes.c_int, [D, P, P, P, P, i64, P, sz, P]),
+        "focus_evict": (ctypes.c_int, [D, P, P, P, P, P, P, P, i64, P, P, P, P, P, P, i64,
+                                       P, P, P, P, sz, P]),
+        "focus_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "focus_abi_version": (ctypes.c_int, []),
+        "focus_set_trace_events": (None, [P, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def make_dims(R, B, Hq, Hkv, head_dim, hidden, softmax_scale=None, pool_window=3) -> FocusDims:
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(head_dim)
+    return FocusDims(int(R), int(B), int(Hq), int(Hkv), int(head_dim), int(hidden),
+                     float(softmax_scale), int(pool_window))
+
+
+def _ptr(t: torch.Tensor | None, dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    return ctypes.c_void_p(t.data_ptr()) if t.numel() else None
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ok(st: int, where: str):
+    if st != 0:
+        raise FocusError(st, where)
+
+
+def focus_status_string(status: int) -> str:
+    return _lib.focus_status_string(int(status)).decode()
+
+
+def focus_abi_version() -> int:
+    return int(_lib.focus_abi_version())
+
+
+def focus_set_trace_events(start=None, stop=None):
+    """Record the torch.cuda.Event pair `start`/`stop` around the attention-statistics
+    kernel of every later focus_evict / focus_attn_stats call (None, None: off)."""
+    if start is None or stop is None:
+        _lib.focus_set_trace_events(None, None)
+        return
+    for e in (start, stop):
+        if e.cuda_event == 0:  # torch creates the CUDA event lazily
+            e.record()
+    _lib.focus_set_trace_events(ctypes.c_void_p(start.cuda_event), ctypes.c_void_p(stop.cuda_event))
+
+
+def focus_workspace_size(dims: FocusDims) -> int:
+    n = int(_lib.focus_workspace_size(ctypes.byref(dims)))
+    if n == 0:
+        raise FocusError(2, "focus_workspace_size")
+    return n
+
+
+class Workspace:
+    """Device scratch for one stream of calls (status word, request order, column sums)."""
+
+    def __init__(self, dims: FocusDims, device="cuda", stream=None):
+        self.nbytes = focus_workspace_size(dims)
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
+        focus_clear_device_status(self, stream)
+
+    @property
+    def ptr(self):
+        return ctypes.c_void_p(self.buf.data_ptr())
+
+
+def focus_clear_device_status(ws: Workspace, stream=None):
+    _ok(_lib.focus_clear_device_status(ws.ptr, ws.nbytes, _stream(stream)),
+        "focus_clear_device_status")
+
+
+def focus_read_device_status(ws: Workspace, stream=None, timeout_ms: int = 10000) -> int:
+    """Synchronises with `stream` and returns the device status code (0 = FOCUS_OK)."""
+    return int(_lib.focus_read_device_status(ws.ptr, _stream(stream), int(timeout_ms)))
+
+
+def focus_attn_stats(dims, q, k_prefix, cu_prefix, k_block, importance, ws: Workspace,
+                     stream=None):
+    bf = torch.bfloat16
+    _ok(_lib.focus_attn_stats(
+        ctypes.byref(dims), _ptr(q, bf, "q"), _ptr(k_prefix, bf, "k_prefix"),
+        _ptr(cu_prefix, torch.int32, "cu_prefix"), int(k_prefix.shape[0]),
+        _ptr(k_block, bf, "k_block"), _ptr(importance, torch.float32, "importance"),
+        ws.ptr, ws.nbytes, _stream(stream)), "focus_attn_stats")
+
+
+def focus_importance_delta(dims, i0, i1, decoded, delta, raw_delta=None, stream=None):
+    f32 = torch.float32
+    _ok(_lib.focus_importance_delta(
+        ctypes.byref(dims), _ptr(i0, f32, "i0"), _ptr(i1, f32, "i1"),
+        _ptr(decoded, torch.uint8, "decoded"), _ptr(delta, f32, "delta"),
+        _ptr(raw_delta, f32, "raw_delta"), _stream(stream)), "focus_importance_delta")
+
+
+def focus_topk_select(dims, delta, decoded, budget, kept_idx, cu_seqlens, ws: Workspace,
+                      stream=None):
+    _ok(_lib.focus_topk_select(
+        ctypes.byref(dims), _ptr(delta, torch.float32, "delta"),
+        _ptr(decoded, torch.uint8, "decoded"), _ptr(budget, torch.int32, "budget"),
+        _ptr(kept_idx, torch.int32, "kept_idx"), _ptr(cu_seqlens, torch.int32, "cu_seqlens"),
+        int(kept_idx.numel()), ws.ptr, ws.nbytes, _stream(stream)), "focus_topk_select")
+
+
+def focus_compact(dims, hidden, kept_idx, cu_seqlens, packed, ws: Workspace, stream=None):
+    bf = torch.bfloat16
+    _ok(_lib.focus_compact(
+        ctypes.byref(dims), _ptr(hidden, bf, "hidden"), _ptr(kept_idx, torch.int32, "kept_idx"),
+        _ptr(cu_seqlens, torch.int32, "cu_seqlens"), _ptr(packed, bf, "packed"),
+        int(packed.shape[0]), ws.ptr, ws.nbytes, _stream(stream)), "focus_compact")
+
+
+def focus_evict(dims, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block, cu_prefix, hidden,
+                decoded, budget, kept_idx, cu_seqlens, packed, ws: Workspace, delta_out=None,
+                i0_out=None, i1_out=None, stream=None):
+    bf, f32 = torch.bfloat16, torch.float32
+    if k0_prefix.shape[0] != k1_prefix.shape[0]:
+        raise ValueError("k0_prefix and k1_prefix must have the same number of rows")
+    _ok(_lib.focus_evict(
+        ctypes.byref(dims), _ptr(q0, bf, "q0"), _ptr(k0_prefix, bf, "k0_prefix"),
+        _ptr(k0_block, bf, "k0_block"), _ptr(q1, bf, "q1"), _ptr(k1_prefix, bf, "k1_prefix"),
+        _ptr(k1_block, bf, "k1_block"), _ptr(cu_prefix, torch.int32, "cu_prefix"),
+        int(k0_prefix.shape[0]), _ptr(hidden, bf, "hidden"),
+        _ptr(decoded, torch.uint8, "decoded"), _ptr(budget, torch.int32, "budget"),
+        _ptr(kept_idx, torch.int32, "kept_idx"), _ptr(cu_seqlens, torch.int32, "cu_seqlens"),
+        _ptr(packed, bf, "packed"), int(packed.shape[0]),
+        _ptr(delta_out, f32, "delta_out"), _ptr(i0_out, f32, "i0_out"),
+        _ptr(i1_out, f32, "i1_out"), ws.ptr, ws.nbytes, _stream(stream)), "focus_evict")
+
+
+def plan_capacity(decoded, budget) -> int:
+    """Rows the packed batch needs: sum_r min(max(budget_r, 0), masked_r).
+
+    Host-side planning helper for the scheduler that owns `decoded` and
+    `budget`: the kept-row counts never depend on the attention data."""
+    dec = decoded.detach().cpu()
+    bud = budget.detach().cpu().to(torch.int64)
+    masked = (dec == 0).sum(dim=1).to(torch.int64)
+    return int(torch.minimum(bud.clamp(min=0), masked).sum())

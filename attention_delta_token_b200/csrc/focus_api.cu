@@ -1,0 +1,441 @@
+// focus_api.cu -- the extern "C" entry points declared in include/focus.h:
+// host-side validation, workspace layout, TMA tensor-map encoding, and the
+// kernel sequence of each call.  No allocation, no synchronisation (except in
+// focus_read_device_status), no state kept between calls.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+#include <chrono>
+#include <mutex>
+#include <thread>
+
+#include "focus.h"
+#include "focus_device.cuh"
+#include "focus_kernels.cuh"
+
+namespace {
+
+using focus::AttnParams;
+
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int row_tiles(const focus_dims_t &d) {
+    const int G = d.Hq / d.Hkv;
+    return (G * d.B + focus::kTileRows - 1) / focus::kTileRows;
+}
+
+// Workspace: [status 256 B][order: R int32][partial: 2 x R x Hkv x MT x B fp32]
+struct WsLayout {
+    size_t status, order, partial, total;
+};
+
+WsLayout ws_layout(const focus_dims_t &d) {
+    WsLayout w;
+    w.status = 0;
+    w.order = kAlign;
+    w.partial = w.order + round_up(sizeof(int32_t) * static_cast<size_t>(d.R), kAlign);
+    const size_t np = 2ull * d.R * d.Hkv * row_tiles(d) * d.B;
+    w.total = w.partial + round_up(sizeof(float) * np, kAlign);
+    return w;
+}
+
+focus_status_t check_dims(const focus_dims_t *d) {
+    if (!d) return FOCUS_ERR_INVALID_ARGUMENT;
+    if (d->R < 1 || d->B < 1 || d->Hq < 1 || d->Hkv < 1 || d->head_dim < 1 || d->hidden < 1 ||
+        d->pool_window < 1)
+        return FOCUS_ERR_INVALID_ARGUMENT;
+    if (!isfinite(d->softmax_scale) || d->softmax_scale < 0.f) return FOCUS_ERR_INVALID_ARGUMENT;
+    if (d->B > 128 || (d->head_dim != 64 && d->head_dim != 128) || d->Hq % d->Hkv != 0 ||
+        d->hidden % 8 != 0 || d->pool_window % 2 == 0)
+        return FOCUS_ERR_UNSUPPORTED_SHAPE;
+    const int G = d->Hq / d->Hkv;
+    if (G > focus::kTileRows || focus::kTileRows % G != 0) return FOCUS_ERR_UNSUPPORTED_SHAPE;
+    const long long rb = static_cast<long long>(d->R) * d->B;
+    if (rb > (1ll << 30)) return FOCUS_ERR_UNSUPPORTED_SHAPE;
+    const long long ctas = static_cast<long long>(d->R) * 2 * d->Hkv * row_tiles(*d);
+    if (ctas > 0x7fffffffll) return FOCUS_ERR_UNSUPPORTED_SHAPE;
+    return FOCUS_OK;
+}
+
+focus_status_t check_ptr(const void *p, size_t align) {
+    if (!p || !aligned(p, align)) return FOCUS_ERR_INVALID_ARGUMENT;
+    return FOCUS_OK;
+}
+
+focus_status_t check_ws(const focus_dims_t &d, const void *ws, size_t bytes) {
+    if (!ws || !aligned(ws, kAlign) || bytes < ws_layout(d).total) return FOCUS_ERR_WORKSPACE;
+    return FOCUS_OK;
+}
+
+#define FOCUS_TRY(x)                          \
+    do {                                      \
+        focus_status_t _st = (x);             \
+        if (_st != FOCUS_OK) return _st;      \
+    } while (0)
+
+#define FOCUS_CUDA(x)                                   \
+    do {                                                \
+        if ((x) != cudaSuccess) return FOCUS_ERR_CUDA;  \
+    } while (0)
+
+// ---------------------------------------------------------------- tracing hook
+
+std::atomic<cudaEvent_t> g_trace_start{nullptr};
+std::atomic<cudaEvent_t> g_trace_stop{nullptr};
+
+cudaError_t launch_attn_traced(const AttnParams &p, int head_dim, cudaStream_t s) {
+    cudaEvent_t a = g_trace_start.load(), b = g_trace_stop.load();
+    if (a && b && cudaEventRecord(a, s) != cudaSuccess) return cudaErrorInvalidResourceHandle;
+    cudaError_t e = focus::launch_attn_stats(p, head_dim, s);
+    if (e != cudaSuccess) return e;
+    if (a && b) return cudaEventRecord(b, s);
+    return cudaSuccess;
+}
+
+// ---------------------------------------------------------------- tensor maps
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+focus_status_t get_encoder() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode ? FOCUS_OK : FOCUS_ERR_CUDA;
+}
+
+// bf16 tensor [rows, heads, d] viewed as (d, heads, rows); box (64, box_heads, box_rows),
+// 128-byte swizzle (the layout tcgen05 reads as a K-major operand).
+focus_status_t encode_rows_heads_d(CUtensorMap *tm, const void *base, long long rows, int heads,
+                                   int d, int box_heads, int box_rows) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                          static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                             static_cast<cuuint64_t>(heads) * d * 2};
+    cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_heads), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FOCUS_OK : FOCUS_ERR_CUDA;
+}
+
+// Fills the tensor maps of one layer.
+focus_status_t encode_layer(AttnParams &p, int layer, const focus_dims_t &d, const void *q,
+                            const void *k_prefix, long long total_prefix, const void *k_block) {
+    const int G = d.Hq / d.Hkv;
+    const long long rb = static_cast<long long>(d.R) * d.B;
+    FOCUS_TRY(encode_rows_heads_d(&p.tm_q[layer], q, rb, d.Hq, d.head_dim, G, focus::kTileRows / G));
+    // With no prefix rows anywhere the prefix map is never read; point it at the block keys.
+    if (total_prefix > 0)
+        FOCUS_TRY(encode_rows_heads_d(&p.tm_kp[layer], k_prefix, total_prefix, d.Hkv, d.head_dim, 1,
+                                      focus::kTileKeys));
+    else
+        FOCUS_TRY(encode_rows_heads_d(&p.tm_kp[layer], k_block, rb, d.Hkv, d.head_dim, 1,
+                                      focus::kTileKeys));
+    FOCUS_TRY(encode_rows_heads_d(&p.tm_kb[layer], k_block, rb, d.Hkv, d.head_dim, 1, p.n_blk));
+    return FOCUS_OK;
+}
+
+void fill_common(AttnParams &p, const focus_dims_t &d, const int32_t *cu_prefix,
+                 long long total_prefix, uint8_t *ws, int n_layers) {
+    const WsLayout w = ws_layout(d);
+    p.cu_prefix = cu_prefix;
+    p.order = reinterpret_cast<const int32_t *>(ws + w.order);
+    p.partial = reinterpret_cast<float *>(ws + w.partial);
+    p.status = reinterpret_cast<uint32_t *>(ws + w.status);
+    p.total_prefix = total_prefix;
+    p.R = d.R;
+    p.B = d.B;
+    p.Hq = d.Hq;
+    p.Hkv = d.Hkv;
+    p.G = d.Hq / d.Hkv;
+    p.MT = row_tiles(d);
+    p.n_layers = n_layers;
+    p.tok_per_tile = focus::kTileRows / p.G;
+    p.n_blk = (d.B + 15) / 16 * 16;
+    p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
+}
+
+focus_status_t check_attn_inputs(const focus_dims_t &d, const void *q, const void *k_prefix,
+                                 const int32_t *cu_prefix, long long total_prefix,
+                                 const void *k_block) {
+    FOCUS_TRY(check_ptr(q, 16));
+    FOCUS_TRY(check_ptr(k_block, 16));
+    FOCUS_TRY(check_ptr(cu_prefix, 4));
+    if (total_prefix < 0 || total_prefix > 0x7fffffffll) return FOCUS_ERR_INVALID_ARGUMENT;
+    if (total_prefix > 0) FOCUS_TRY(check_ptr(k_prefix, 16));
+    return FOCUS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t focus_workspace_size(const focus_dims_t *dims) {
+    if (check_dims(dims) != FOCUS_OK) return 0;
+    return ws_layout(*dims).total;
+}
+
+focus_status_t focus_clear_device_status(void *workspace, size_t workspace_bytes, void *stream) {
+    if (!workspace || !aligned(workspace, kAlign) || workspace_bytes < kAlign)
+        return FOCUS_ERR_WORKSPACE;
+    FOCUS_CUDA(cudaMemsetAsync(workspace, 0, sizeof(uint32_t), static_cast<cudaStream_t>(stream)));
+    return FOCUS_OK;
+}
+
+focus_status_t focus_read_device_status(const void *workspace, void *stream, int timeout_ms) {
+    if (!workspace || !aligned(workspace, kAlign)) return FOCUS_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaEvent_t ev;
+    FOCUS_CUDA(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+    if (cudaEventRecord(ev, s) != cudaSuccess) {
+        cudaEventDestroy(ev);
+        return FOCUS_ERR_CUDA;
+    }
+    const auto t0 = std::chrono::steady_clock::now();
+    for (;;) {
+        const cudaError_t q = cudaEventQuery(ev);
+        if (q == cudaSuccess) break;
+        if (q != cudaErrorNotReady) {
+            cudaEventDestroy(ev);
+            return FOCUS_ERR_CUDA;
+        }
+        if (timeout_ms >= 0 &&
+            std::chrono::steady_clock::now() - t0 > std::chrono::milliseconds(timeout_ms)) {
+            cudaEventDestroy(ev);
+            return FOCUS_ERR_TIMEOUT;
+        }
+        std::this_thread::sleep_for(std::chrono::microseconds(50));
+    }
+    cudaEventDestroy(ev);
+    uint32_t word = 0;
+    FOCUS_CUDA(cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost));
+    if (word & focus::FOCUS_DEV_TIMEOUT) return FOCUS_ERR_TIMEOUT;
+    if (word & focus::FOCUS_DEV_BAD_INPUT) return FOCUS_ERR_DEVICE_CHECK;
+    if (word & focus::FOCUS_DEV_CAPACITY) return FOCUS_ERR_CAPACITY;
+    return FOCUS_OK;
+}
+
+focus_status_t focus_attn_stats(const focus_dims_t *dims, const void *q, const void *k_prefix,
+                                const int32_t *cu_prefix, int64_t total_prefix,
+                                const void *k_block, float *importance, void *workspace,
+                                size_t workspace_bytes, void *stream) {
+    FOCUS_TRY(check_dims(dims));
+    const focus_dims_t &d = *dims;
+    FOCUS_TRY(check_attn_inputs(d, q, k_prefix, cu_prefix, total_prefix, k_block));
+    FOCUS_TRY(check_ptr(importance, 4));
+    FOCUS_TRY(check_ws(d, workspace, workspace_bytes));
+    FOCUS_TRY(get_encoder());
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+
+    AttnParams p;
+    memset(&p, 0, sizeof p);
+    fill_common(p, d, cu_prefix, total_prefix, ws, 1);
+    FOCUS_TRY(encode_layer(p, 0, d, q, k_prefix, total_prefix, k_block));
+    p.tm_q[1] = p.tm_q[0];
+    p.tm_kp[1] = p.tm_kp[0];
+    p.tm_kb[1] = p.tm_kb[0];
+
+    focus::PlanParams pp;
+    memset(&pp, 0, sizeof pp);
+    pp.cu_prefix = cu_prefix;
+    pp.order = const_cast<int32_t *>(p.order);
+    pp.status = p.status;
+    pp.R = d.R;
+    pp.B = d.B;
+    FOCUS_CUDA(focus::launch_plan(pp, s));
+    FOCUS_CUDA(launch_attn_traced(p, d.head_dim, s));
+    focus::ReduceParams rp{p.partial, importance, d.R, d.B, d.Hkv, p.MT};
+    FOCUS_CUDA(focus::launch_reduce(rp, s));
+    return FOCUS_OK;
+}
+
+focus_status_t focus_importance_delta(const focus_dims_t *dims, const float *i0, const float *i1,
+                                      const uint8_t *decoded, float *delta, float *raw_delta,
+                                      void *stream) {
+    FOCUS_TRY(check_dims(dims));
+    FOCUS_TRY(check_ptr(i0, 4));
+    FOCUS_TRY(check_ptr(i1, 4));
+    FOCUS_TRY(check_ptr(decoded, 1));
+    FOCUS_TRY(check_ptr(delta, 4));
+    if (raw_delta) FOCUS_TRY(check_ptr(raw_delta, 4));
+    focus::DeltaParams p{i0, i1, decoded, delta, raw_delta, dims->R, dims->B, dims->pool_window};
+    FOCUS_CUDA(focus::launch_delta(p, static_cast<cudaStream_t>(stream)));
+    return FOCUS_OK;
+}
+
+focus_status_t focus_topk_select(const focus_dims_t *dims, const float *delta,
+                                 const uint8_t *decoded, const int32_t *budget, int32_t *kept_idx,
+                                 int32_t *cu_seqlens, int64_t capacity, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
+    FOCUS_TRY(check_dims(dims));
+    const focus_dims_t &d = *dims;
+    FOCUS_TRY(check_ptr(delta, 4));
+    FOCUS_TRY(check_ptr(decoded, 1));
+    FOCUS_TRY(check_ptr(budget, 4));
+    FOCUS_TRY(check_ptr(cu_seqlens, 4));
+    if (capacity < 0) return FOCUS_ERR_INVALID_ARGUMENT;
+    if (capacity > 0) FOCUS_TRY(check_ptr(kept_idx, 4));
+    FOCUS_TRY(check_ws(d, workspace, workspace_bytes));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws + ws_layout(d).status);
+
+    focus::PlanParams pp;
+    memset(&pp, 0, sizeof pp);
+    pp.decoded = decoded;
+    pp.budget = budget;
+    pp.cu_seqlens = cu_seqlens;
+    pp.status = status;
+    pp.capacity = capacity;
+    pp.R = d.R;
+    pp.B = d.B;
+    FOCUS_CUDA(focus::launch_plan(pp, s));
+
+    focus::SelectParams sp;
+    memset(&sp, 0, sizeof sp);
+    sp.delta_in = delta;
+    sp.decoded = decoded;
+    sp.cu_seqlens = cu_seqlens;
+    sp.kept_idx = kept_idx;
+    sp.status = status;
+    sp.capacity = capacity;
+    sp.R = d.R;
+    sp.B = d.B;
+    sp.pool_window = d.pool_window;
+    FOCUS_CUDA(focus::launch_select_compact(sp, s));
+    return FOCUS_OK;
+}
+
+focus_status_t focus_compact(const focus_dims_t *dims, const void *hidden, const int32_t *kept_idx,
+                             const int32_t *cu_seqlens, void *packed, int64_t capacity,
+                             void *workspace, size_t workspace_bytes, void *stream) {
+    FOCUS_TRY(check_dims(dims));
+    const focus_dims_t &d = *dims;
+    FOCUS_TRY(check_ptr(hidden, 16));
+    FOCUS_TRY(check_ptr(cu_seqlens, 4));
+    if (capacity < 0) return FOCUS_ERR_INVALID_ARGUMENT;
+    if (capacity > 0) {
+        FOCUS_TRY(check_ptr(kept_idx, 4));
+        FOCUS_TRY(check_ptr(packed, 16));
+    }
+    FOCUS_TRY(check_ws(d, workspace, workspace_bytes));
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    focus::CompactParams p{static_cast<const uint16_t *>(hidden), kept_idx, cu_seqlens,
+                           static_cast<uint16_t *>(packed),
+                           reinterpret_cast<uint32_t *>(ws + ws_layout(d).status), capacity,
+                           d.R, d.B, d.hidden};
+    FOCUS_CUDA(focus::launch_compact(p, static_cast<cudaStream_t>(stream)));
+    return FOCUS_OK;
+}
+
+focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void *k0_prefix,
+                           const void *k0_block, const void *q1, const void *k1_prefix,
+                           const void *k1_block, const int32_t *cu_prefix, int64_t total_prefix,
+                           const void *hidden, const uint8_t *decoded, const int32_t *budget,
+                           int32_t *kept_idx, int32_t *cu_seqlens, void *packed, int64_t capacity,
+                           float *delta_out, float *i0_out, float *i1_out, void *workspace,
+                           size_t workspace_bytes, void *stream) {
+    FOCUS_TRY(check_dims(dims));
+    const focus_dims_t &d = *dims;
+    FOCUS_TRY(check_attn_inputs(d, q0, k0_prefix, cu_prefix, total_prefix, k0_block));
+    FOCUS_TRY(check_attn_inputs(d, q1, k1_prefix, cu_prefix, total_prefix, k1_block));
+    FOCUS_TRY(check_ptr(hidden, 16));
+    FOCUS_TRY(check_ptr(decoded, 1));
+    FOCUS_TRY(check_ptr(budget, 4));
+    FOCUS_TRY(check_ptr(cu_seqlens, 4));
+    if (capacity < 0) return FOCUS_ERR_INVALID_ARGUMENT;
+    if (capacity > 0) {
+        FOCUS_TRY(check_ptr(kept_idx, 4));
+        FOCUS_TRY(check_ptr(packed, 16));
+    }
+    if (delta_out) FOCUS_TRY(check_ptr(delta_out, 4));
+    if (i0_out) FOCUS_TRY(check_ptr(i0_out, 4));
+    if (i1_out) FOCUS_TRY(check_ptr(i1_out, 4));
+    FOCUS_TRY(check_ws(d, workspace, workspace_bytes));
+    FOCUS_TRY(get_encoder());
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+
+    AttnParams p;
+    memset(&p, 0, sizeof p);
+    fill_common(p, d, cu_prefix, total_prefix, ws, 2);
+    FOCUS_TRY(encode_layer(p, 0, d, q0, k0_prefix, total_prefix, k0_block));
+    FOCUS_TRY(encode_layer(p, 1, d, q1, k1_prefix, total_prefix, k1_block));
+
+    focus::PlanParams pp;
+    memset(&pp, 0, sizeof pp);
+    pp.cu_prefix = cu_prefix;
+    pp.decoded = decoded;
+    pp.budget = budget;
+    pp.order = const_cast<int32_t *>(p.order);
+    pp.cu_seqlens = cu_seqlens;
+    pp.status = p.status;
+    pp.capacity = capacity;
+    pp.R = d.R;
+    pp.B = d.B;
+    FOCUS_CUDA(focus::launch_plan(pp, s));
+    FOCUS_CUDA(launch_attn_traced(p, d.head_dim, s));
+
+    focus::SelectParams sp;
+    memset(&sp, 0, sizeof sp);
+    sp.partial = p.partial;
+    sp.decoded = decoded;
+    sp.cu_seqlens = cu_seqlens;
+    sp.kept_idx = kept_idx;
+    sp.hidden = static_cast<const uint16_t *>(hidden);
+    sp.packed = static_cast<uint16_t *>(packed);
+    sp.delta_out = delta_out;
+    sp.i0_out = i0_out;
+    sp.i1_out = i1_out;
+    sp.status = p.status;
+    sp.capacity = capacity;
+    sp.R = d.R;
+    sp.B = d.B;
+    sp.Hkv = d.Hkv;
+    sp.MT = p.MT;
+    sp.H = d.hidden;
+    sp.pool_window = d.pool_window;
+    FOCUS_CUDA(focus::launch_select_compact(sp, s));
+    return FOCUS_OK;
+}
+
+const char *focus_status_string(focus_status_t st) {
+    switch (st) {
+        case FOCUS_OK: return "FOCUS_OK";
+        case FOCUS_ERR_INVALID_ARGUMENT: return "FOCUS_ERR_INVALID_ARGUMENT";
+        case FOCUS_ERR_UNSUPPORTED_SHAPE: return "FOCUS_ERR_UNSUPPORTED_SHAPE";
+        case FOCUS_ERR_CAPACITY: return "FOCUS_ERR_CAPACITY";
+        case FOCUS_ERR_WORKSPACE: return "FOCUS_ERR_WORKSPACE";
+        case FOCUS_ERR_CUDA: return "FOCUS_ERR_CUDA";
+        case FOCUS_ERR_DEVICE_CHECK: return "FOCUS_ERR_DEVICE_CHECK";
+        case FOCUS_ERR_TIMEOUT: return "FOCUS_ERR_TIMEOUT";
+    }
+    return "FOCUS_ERR_UNKNOWN";
+}
+
+int focus_abi_version(void) { return FOCUS_ABI_VERSION; }
+
+void focus_set_trace_events(void *start_event, void *stop_event) {
+    g_trace_start.store(static_cast<cudaEvent_t>(start_event));
+    g_trace_stop.store(static_cast<cudaEvent_t>(stop_event));
+}
+
+}  // extern "C"

@@ -1,0 +1,93 @@
+// focus_kernels.cuh -- launch parameters and launchers of the FOCUS eviction kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace focus {
+
+// ---------------------------------------------------------------- attention statistics
+// One CTA = one (layer, request, kv head, 128-row query tile).  Its 128 query
+// rows are the G = Hq/Hkv query heads of that kv head for 128/G consecutive
+// block tokens (row = token * G + head-in-group), so every key tile that TMA
+// brings in is used by all query heads that read it.
+constexpr int kTileRows = 128;   // UMMA M: query rows per CTA
+constexpr int kTileKeys = 128;   // UMMA N: keys per prefix tile
+constexpr int kStages = 2;       // key-tile ring depth (two CTAs share an SM)
+constexpr int kAttnThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 softmax
+constexpr int kTmemCols = 256;   // two 128-column fp32 S buffers
+
+struct AttnParams {
+    CUtensorMap tm_q[2];    // per layer: Q  [R*B, Hq, d], box (64, G, 128/G)
+    CUtensorMap tm_kp[2];   // per layer: prefix K [total_prefix, Hkv, d], box (64, 1, 128)
+    CUtensorMap tm_kb[2];   // per layer: block K  [R*B, Hkv, d], box (64, 1, n_blk)
+    const int32_t *cu_prefix;  // [R+1]
+    const int32_t *order;      // [R] request processing order (longest prefix first)
+    float *partial;            // [n_layers][R][Hkv][MT][B] column sums per kv head / row tile
+    uint32_t *status;          // device status word
+    long long total_prefix;
+    int R, B, Hq, Hkv, G, MT, n_layers;
+    int tok_per_tile;          // 128 / G block tokens per row tile
+    int n_blk;                 // keys in the block tile: B rounded up to 16
+    float scale_log2;          // softmax_scale * log2(e)
+};
+
+size_t attn_smem_bytes(int head_dim);
+cudaError_t launch_attn_stats(const AttnParams &p, int head_dim, cudaStream_t stream);
+
+// ---------------------------------------------------------------- planning
+struct PlanParams {
+    const int32_t *cu_prefix;  // [R+1]
+    const uint8_t *decoded;    // [R,B] or null (no counts)
+    const int32_t *budget;     // [R]   or null
+    int32_t *order;            // [R]   or null (no ordering)
+    int32_t *cu_seqlens;       // [R+1] or null
+    uint32_t *status;
+    long long capacity;
+    int R, B;
+};
+cudaError_t launch_plan(const PlanParams &p, cudaStream_t stream);
+
+// ---------------------------------------------------------------- select / compact
+struct SelectParams {
+    const float *partial;      // [2][R][Hkv][MT][B] (fused path) or null
+    const float *delta_in;     // [R,B] pooled+masked delta (stand-alone select) or null
+    const uint8_t *decoded;    // [R,B]
+    const int32_t *cu_seqlens; // [R+1] (written by the planner)
+    int32_t *kept_idx;         // [capacity]
+    const uint16_t *hidden;    // [R,B,H] bf16 bits, null = no compaction
+    uint16_t *packed;          // [capacity,H]
+    float *delta_out, *i0_out, *i1_out, *raw_out;  // optional [R,B]
+    uint32_t *status;
+    long long capacity;
+    int R, B, Hkv, MT, H, pool_window;
+};
+cudaError_t launch_select_compact(const SelectParams &p, cudaStream_t stream);
+
+struct DeltaParams {
+    const float *i0, *i1;
+    const uint8_t *decoded;
+    float *delta, *raw;
+    int R, B, pool_window;
+};
+cudaError_t launch_delta(const DeltaParams &p, cudaStream_t stream);
+
+struct ReduceParams {
+    const float *partial;  // [R][Hkv][MT][B]
+    float *importance;     // [R,B]
+    int R, B, Hkv, MT;
+};
+cudaError_t launch_reduce(const ReduceParams &p, cudaStream_t stream);
+
+struct CompactParams {
+    const uint16_t *hidden;
+    const int32_t *kept_idx, *cu_seqlens;
+    uint16_t *packed;
+    uint32_t *status;
+    long long capacity;
+    int R, B, H;
+};
+cudaError_t launch_compact(const CompactParams &p, cudaStream_t stream);
+
+}  // namespace focus

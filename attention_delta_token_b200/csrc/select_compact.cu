@@ -1,0 +1,316 @@
+// select_compact.cu -- planning, importance delta, MaxPool1D, mask, top-K and
+// compaction kernels of the FOCUS eviction step (sm_100a, CUDA cores / LSU).
+//
+// Method: "FOCUS: DLLMs Know How to Tame Their Compute Bound" (pith.science
+// review page), "What carries the argument": dI = I(layer 1) - I(layer 0)
+// (Eq. 3), smoothed by MaxPool1D (Free-Parameter Ledger: k = 3, Eq. 15), top-K
+// candidates kept under a budget; "The pith": the remaining layers then run
+// only on the retained tokens, here packed into a varlen batch with cu_seqlens.
+//
+// Selection is exact and deterministic: a position's rank is the number of
+// positions that beat it under (value desc, position asc), so every tie goes to
+// the lower position and the kept set never depends on thread timing.
+#include <math.h>
+
+#include "focus_device.cuh"
+#include "focus_kernels.cuh"
+
+namespace focus {
+
+namespace {
+
+constexpr int kPlanThreads = 1024;
+constexpr int kMaxSortR = 4096;  // requests ordered on the device; larger batches keep input order
+
+// k_r = min(max(budget_r, 0), masked_r)
+__device__ __forceinline__ int kept_count(const uint8_t *decoded, const int32_t *budget, int r,
+                                          int B) {
+    int masked = 0;
+    const uint8_t *d = decoded + static_cast<size_t>(r) * B;
+    for (int j = 0; j < B; ++j) masked += d[j] == 0;
+    const int K = budget[r];
+    return min(max(K, 0), masked);
+}
+
+// Exclusive block-wide scan of one int per thread (kPlanThreads threads).
+__device__ __forceinline__ int block_exclusive_scan(int x, int *warp_tot, int &total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = x;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = warp_tot[lane];
+        int wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, wi, off);
+            if (lane >= off) wi += y;
+        }
+        warp_tot[lane] = wi - w;  // exclusive prefix of the warp totals
+        if (lane == 31) warp_tot[32] = wi;
+    }
+    __syncthreads();
+    const int ex = warp_tot[warp] + incl - x;
+    total = warp_tot[32];
+    __syncthreads();
+    return ex;
+}
+
+// One CTA: (a) the processing order of the requests, longest prefix first (a
+// bitonic sort of (L desc, r asc) keys), so the attention CTAs of the longest
+// requests start in the first wave; (b) k_r and cu_seqlens (depend only on
+// decoded and budget) and the capacity check.
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) {
+    __shared__ unsigned long long keys[kMaxSortR];
+    __shared__ int warp_tot[33];
+    const int R = p.R;
+
+    if (p.order) {
+        if (R <= kMaxSortR) {
+            int n = 1;
+            while (n < R) n <<= 1;
+            for (int i = threadIdx.x; i < n; i += blockDim.x) {
+                unsigned long long key = ~0ull;
+                if (i < R) {
+                    int L = p.cu_prefix[i + 1] - p.cu_prefix[i];
+                    L = max(L, 0);
+                    key = (static_cast<unsigned long long>(0x7fffffffu - static_cast<uint32_t>(L)) << 32) |
+                          static_cast<uint32_t>(i);
+                }
+                keys[i] = key;
+            }
+            __syncthreads();
+            for (int k = 2; k <= n; k <<= 1) {
+                for (int j = k >> 1; j > 0; j >>= 1) {
+                    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+                        const int ixj = i ^ j;
+                        if (ixj > i) {
+                            const unsigned long long a = keys[i], b = keys[ixj];
+                            const bool up = (i & k) == 0;
+                            if ((a > b) == up) {
+                                keys[i] = b;
+                                keys[ixj] = a;
+                            }
+                        }
+                    }
+                    __syncthreads();
+                }
+            }
+            for (int i = threadIdx.x; i < R; i += blockDim.x)
+                p.order[i] = static_cast<int32_t>(keys[i] & 0xffffffffu);
+        } else {
+            for (int i = threadIdx.x; i < R; i += blockDim.x) p.order[i] = i;
+        }
+    }
+
+    if (p.cu_seqlens) {
+        int running = 0;
+        if (threadIdx.x == 0) p.cu_seqlens[0] = 0;
+        for (int base = 0; base < R; base += kPlanThreads) {
+            const int r = base + threadIdx.x;
+            const int k = r < R ? kept_count(p.decoded, p.budget, r, p.B) : 0;
+            int total;
+            const int ex = block_exclusive_scan(k, warp_tot, total);
+            if (r < R) p.cu_seqlens[r + 1] = running + ex + k;
+            running += total;
+        }
+        if (threadIdx.x == 0 && static_cast<long long>(running) > p.capacity)
+            atomicOr(p.status, FOCUS_DEV_CAPACITY);
+    }
+}
+
+// Rank-based top-k over sv[0..B) (value desc, position asc); thread j < B
+// decides position j.  Writes the kept positions, ascending, into kept_s and
+// kept_idx[base ..].  Returns nothing; the caller syncs.
+__device__ __forceinline__ void select_block(const float *sv, const uint8_t *dec, int B, int k,
+                                             long long base, long long capacity, int *sel_s,
+                                             int *kept_s, int32_t *kept_idx, uint32_t *status) {
+    const int j = threadIdx.x;
+    if (j < 128) kept_s[j] = -1;
+    if (j < B) {
+        const float v = sv[j];
+        int rank = 0;
+        for (int t = 0; t < B; ++t) {  // only still-masked positions compete
+            const float u = sv[t];
+            rank += dec[t] == 0 && ((u > v) || (u == v && t < j));
+        }
+        sel_s[j] = (dec[j] == 0 && rank < k) ? 1 : 0;
+    }
+    __syncthreads();
+    if (j < B && sel_s[j]) {
+        int slot = 0;
+        for (int t = 0; t < j; ++t) slot += sel_s[t];
+        if (slot >= k) return;  // only reachable with non-finite values (out of contract)
+        kept_s[slot] = j;
+        const long long out = base + slot;
+        if (out < capacity)
+            kept_idx[out] = j;
+        else
+            atomicOr(status, FOCUS_DEV_CAPACITY);
+    }
+}
+
+// MaxPool1D (odd window, stride 1, same padding, padded cells ignored) of
+// raw[0..B) at position j, then the decoded mask.
+__device__ __forceinline__ float pool_mask(const float *raw, const uint8_t *dec, int B, int w,
+                                           int j) {
+    const int h = w >> 1;
+    float best = -INFINITY;
+    const int lo = max(0, j - h), hi = min(B - 1, j + h);
+    for (int t = lo; t <= hi; ++t) best = fmaxf(best, raw[t]);
+    return dec[j] ? -INFINITY : best;
+}
+
+// One CTA per request.  From the per-kv-head column sums of both layers (fused
+// path) or from a pooled delta (stand-alone select): I0, I1, dI, MaxPool1D,
+// mask, top-k, then the k kept hidden rows copied with 16-byte vectors.
+__global__ void __launch_bounds__(256) select_compact_kernel(const SelectParams p) {
+    __shared__ float raw_s[128];
+    __shared__ float val_s[128];
+    __shared__ uint8_t dec_s[128];
+    __shared__ int sel_s[128];
+    __shared__ int kept_s[128];
+    const int r = blockIdx.x;
+    const int B = p.B;
+    const int j = threadIdx.x;
+    const size_t rb = static_cast<size_t>(r) * B;
+
+    if (j < B) dec_s[j] = p.decoded[rb + j];
+    if (p.partial) {
+        if (j < B) {
+            const size_t lstride = static_cast<size_t>(p.R) * p.Hkv * p.MT * B;
+            float i0 = 0.f, i1 = 0.f;
+            for (int g = 0; g < p.Hkv * p.MT; ++g) {
+                const size_t idx = (rb * p.Hkv * p.MT) + static_cast<size_t>(g) * B + j;
+                i0 += p.partial[idx];
+                i1 += p.partial[lstride + idx];
+            }
+            raw_s[j] = i1 - i0;
+            if (p.i0_out) p.i0_out[rb + j] = i0;
+            if (p.i1_out) p.i1_out[rb + j] = i1;
+            if (p.raw_out) p.raw_out[rb + j] = i1 - i0;
+        }
+        __syncthreads();
+        if (j < B) {
+            const float d = pool_mask(raw_s, dec_s, B, p.pool_window, j);
+            val_s[j] = d;
+            if (p.delta_out) p.delta_out[rb + j] = d;
+        }
+    } else {
+        if (j < B) val_s[j] = p.delta_in[rb + j];
+    }
+    __syncthreads();
+
+    const long long base = p.cu_seqlens[r];
+    const int k = static_cast<int>(p.cu_seqlens[r + 1] - base);
+    select_block(val_s, dec_s, B, k, base, p.capacity, sel_s, kept_s, p.kept_idx, p.status);
+    __syncthreads();
+
+    if (p.hidden) {
+        const int rows = static_cast<int>(max(0ll, min(static_cast<long long>(k), p.capacity - base)));
+        const int nvec = p.H / 8;  // 16-byte vectors per row
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.hidden) + rb * nvec;
+        uint4 *dst = reinterpret_cast<uint4 *>(p.packed) + static_cast<size_t>(base) * nvec;
+        const int total = rows * nvec;
+        for (int v = threadIdx.x; v < total; v += blockDim.x) {
+            const int t = v / nvec;
+            const int c = v - t * nvec;
+            const int jj = kept_s[t];
+            if (jj < 0) {  // fewer than k selected: non-finite values (out of contract)
+                if (c == 0) atomicOr(p.status, FOCUS_DEV_BAD_INPUT);
+                continue;
+            }
+            dst[static_cast<size_t>(t) * nvec + c] = __ldg(src + static_cast<size_t>(jj) * nvec + c);
+        }
+    }
+}
+
+// Stand-alone importance delta + MaxPool1D + mask, one CTA (128 threads) per request.
+__global__ void __launch_bounds__(128) delta_kernel(const DeltaParams p) {
+    __shared__ float raw_s[128];
+    __shared__ uint8_t dec_s[128];
+    const int r = blockIdx.x, j = threadIdx.x, B = p.B;
+    const size_t rb = static_cast<size_t>(r) * B;
+    if (j < B) {
+        const float d = p.i1[rb + j] - p.i0[rb + j];
+        raw_s[j] = d;
+        dec_s[j] = p.decoded[rb + j];
+        if (p.raw) p.raw[rb + j] = d;
+    }
+    __syncthreads();
+    if (j < B) p.delta[rb + j] = pool_mask(raw_s, dec_s, B, p.pool_window, j);
+}
+
+// importance[r][j] = sum over kv heads and row tiles (fixed order) of the column sums.
+__global__ void __launch_bounds__(128) reduce_kernel(const ReduceParams p) {
+    const int r = blockIdx.x, j = threadIdx.x, B = p.B;
+    if (j >= B) return;
+    const size_t rb = static_cast<size_t>(r) * B;
+    float s = 0.f;
+    for (int g = 0; g < p.Hkv * p.MT; ++g) s += p.partial[rb * p.Hkv * p.MT + static_cast<size_t>(g) * B + j];
+    p.importance[rb + j] = s;
+}
+
+// Stand-alone compaction: one warp per packed row, request found by binary search.
+__global__ void __launch_bounds__(256) compact_kernel(const CompactParams p) {
+    const int warps = blockDim.x >> 5;
+    const long long total = min(static_cast<long long>(p.cu_seqlens[p.R]), p.capacity);
+    if (blockIdx.x == 0 && threadIdx.x == 0 && p.cu_seqlens[p.R] > p.capacity)
+        atomicOr(p.status, FOCUS_DEV_CAPACITY);
+    const int lane = threadIdx.x & 31;
+    const int nvec = p.H / 8;
+    for (long long row = static_cast<long long>(blockIdx.x) * warps + (threadIdx.x >> 5); row < total;
+         row += static_cast<long long>(gridDim.x) * warps) {
+        int lo = 0, hi = p.R - 1;  // largest r with cu[r] <= row
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.cu_seqlens[mid] <= row) lo = mid; else hi = mid - 1;
+        }
+        const int jj = p.kept_idx[row];
+        if (jj < 0 || jj >= p.B) {
+            if (lane == 0) atomicOr(p.status, FOCUS_DEV_BAD_INPUT);
+            continue;
+        }
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.hidden) +
+                           (static_cast<size_t>(lo) * p.B + jj) * nvec;
+        uint4 *dst = reinterpret_cast<uint4 *>(p.packed) + static_cast<size_t>(row) * nvec;
+        for (int c = lane; c < nvec; c += 32) dst[c] = __ldg(src + c);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_plan(const PlanParams &p, cudaStream_t stream) {
+    plan_kernel<<<1, kPlanThreads, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select_compact(const SelectParams &p, cudaStream_t stream) {
+    select_compact_kernel<<<p.R, 256, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_delta(const DeltaParams &p, cudaStream_t stream) {
+    delta_kernel<<<p.R, 128, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_reduce(const ReduceParams &p, cudaStream_t stream) {
+    reduce_kernel<<<p.R, 128, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_compact(const CompactParams &p, cudaStream_t stream) {
+    long long blocks = (p.capacity + 7) / 8;
+    if (blocks < 1) blocks = 1;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    compact_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace focus

@@ -1,0 +1,435 @@
+#!/usr/bin/env python
+"""Throughput of the FOCUS importance-delta token eviction step on B200.
+
+One step = one fused focus_evict call over a batch of blocks: layer-0 and
+layer-1 attention importance, delta, MaxPool1D, mask, top-K, compaction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--config C]
+
+Default workload: SDAR-8B shape, 256 requests, B = 32, prefix lengths
+U[1024, 4096], Hq = 32, Hkv = 8, d = 128, hidden = 4096 (seeded synthetic bf16).
+N > 1 runs under torchrun, one rank per GPU; every rank processes its own batch
+(independent requests: weak scaling, no collective on the data path); the
+time is the max over ranks.  Prints one JSON line on rank 0.
+
+--impl reference times the float64 CPU oracle (the checker the tests use) on
+the host cores, on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "eviction blocks/s at SDAR-8B shape, batch 256, B=32; % of HBM roofline"
+UNIT = "blocks/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+ATTN_SOURCES = ["attn_stats.cu", "focus_device.cuh", "focus_kernels.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_stats_traffic.txt")
+
+
+# ---------------------------------------------------------------- accounting
+
+def algorithmic_counts(p) -> dict:
+    """Work the method must do per step (not what an implementation happens to do).
+
+    attention: both layers read every prefix and block key once (Hkv x d bf16 per
+    key) and every block query once; flops 2*d per (query row, key) per layer;
+    one exp per (query row, key) per layer.  Select/compact: the mask, budget,
+    kept indices, cu_seqlens, and the kept hidden rows read once and written once.
+    """
+    L = p.prefix_len.astype(np.int64)
+    N = L + p.B
+    dec = p.decoded.cpu().numpy()
+    masked = (dec == 0).sum(1).astype(np.int64)
+    k = np.minimum(np.clip(p.budget.cpu().numpy().astype(np.int64), 0, None), masked)
+    attn = 2 * (N * p.Hkv * p.d * 2 + p.B * p.Hq * p.d * 2)
+    rest = p.B + 4 + 4 * k + 4 + k * p.H * 2 * 2
+    return dict(attn_bytes=int(attn.sum()), bytes=int(attn.sum() + rest.sum() + 4),
+                flops=int((2 * 2 * p.Hq * p.B * N * p.d).sum()),
+                exps=int((2 * p.Hq * p.B * N).sum()), decisions=int(masked.sum()),
+                kept_rows=int(k.sum()), blocks=int(p.R))
+
+
+def read_peaks() -> tuple[dict, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def attn_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ATTN_SOURCES:
+        with open(os.path.join(ROOT, "attention_delta_token_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, or None when
+    the kernel sources changed since the counters were taken."""
+    try:
+        kv = {}
+        for line in open(TRAFFIC_FILE):
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+        if kv.get("kernel_sources_sha256_16") != attn_source_hash():
+            return None
+        return int(kv[f"dram_bytes_per_launch[{workload}]"])
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------- clocks
+
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+           0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+           0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Reads SM clock and clock-event reasons through NVML every `period` seconds
+    while the timed region runs.  Read-only: it changes no GPU setting."""
+
+    def __init__(self, device_index: int, period: float = 0.02):
+        self.samples = []
+        self.period = period
+        self.ok = False
+        self.sm_max = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                if not uuid.startswith("GPU-"):
+                    uuid = "GPU-" + uuid
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.sm_max = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                sm = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((sm, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self) -> dict:
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.sm_max, "reasons": [], "samples": 0}
+        sms = [s for s, _ in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= int(r)
+        names = [n for b, n in REASONS.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(sms)), "sm_max_mhz": self.sm_max,
+                "reasons": names, "samples": len(sms)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def make_outputs(p, cap, dev):
+    kept = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)[:cap]
+    cu = torch.empty(p.R + 1, dtype=torch.int32, device=dev)
+    packed = torch.empty(max(cap, 1), p.H, dtype=torch.bfloat16, device=dev)[:cap]
+    return kept, cu, packed
+
+
+def run_ours(args, rank, world, local_rank):
+    import attention_delta_token_b200 as F
+    dist = torch.distributed if world > 1 else None
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = synth.CONFIGS[args.config]
+    seed = args.config + 1000 * rank
+    p = synth.make_problem(cfg, seed=seed, device=dev)
+    counts = algorithmic_counts(p)
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+    ws = F.Workspace(dims, dev)
+    cap = F.plan_capacity(p.decoded, p.budget)
+    kept, cu, packed = make_outputs(p, cap, dev)
+    stream = torch.cuda.current_stream(dev)
+    in_bytes = sum(t.numel() * t.element_size() for t in p.tensors().values())
+
+    def step():
+        F.focus_evict(dims, p.q0, p.k0_prefix, p.k0_block, p.q1, p.k1_prefix, p.k1_block,
+                      p.cu_prefix, p.hidden, p.decoded, p.budget, kept, cu, packed, ws)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if dist:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if not dist:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- device-resident timing
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        for _ in range(args.warmup):
+            step()
+        barrier()
+        ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for e in ev_a + ev_b:
+            e.record(stream)
+        start = torch.cuda.Event(enable_timing=True)
+        stop = torch.cuda.Event(enable_timing=True)
+        barrier()
+        start.record(stream)
+        for k in range(args.steps):
+            F.focus_set_trace_events(ev_a[k], ev_b[k])
+            step()
+        stop.record(stream)
+        F.focus_set_trace_events(None, None)
+        barrier()
+    status = F.focus_read_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {F.focus_status_string(status)}")
+    elapsed = start.elapsed_time(stop) / 1e3
+    attn_s = sum(a.elapsed_time(b) for a, b in zip(ev_a, ev_b)) / 1e3 / args.steps
+    elapsed_max = max_over_ranks(elapsed)
+    attn_s_max = max_over_ranks(attn_s)
+    step_s = elapsed_max / args.steps
+
+    # ---- end to end: pinned host inputs -> device, the C-ABI call, result -> host
+    e2e = None
+    if not args.no_e2e:
+        host = {k: v.to("cpu").pin_memory() for k, v in p.tensors().items()}
+        dev_t = p.tensors()
+        out_kept = torch.empty(kept.shape, dtype=kept.dtype).pin_memory()
+        out_cu = torch.empty(cu.shape, dtype=cu.dtype).pin_memory()
+        out_packed = torch.empty(packed.shape, dtype=packed.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = sum(t.numel() * t.element_size() for t in (out_kept, out_cu, out_packed))
+        n_e2e = max(1, min(args.steps, args.e2e_steps))
+
+        def e2e_step():
+            for k, t in host.items():
+                dev_t[k].copy_(t, non_blocking=True)
+            step()
+            out_kept.copy_(kept, non_blocking=True)
+            out_cu.copy_(cu, non_blocking=True)
+            out_packed.copy_(packed, non_blocking=True)
+
+        e2e_step()
+        barrier()
+        s2 = torch.cuda.Event(enable_timing=True)
+        t2 = torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        t2.record(stream)
+        barrier()
+        e2e_s = max_over_ranks(s2.elapsed_time(t2) / 1e3) / n_e2e
+        e2e = {"value": world * p.R / e2e_s, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "steps": n_e2e, "ms_per_step": e2e_s * 1e3,
+               "path": "pinned host -> cudaMemcpyAsync -> focus_evict -> host"}
+        if F.focus_read_device_status(ws) != 0:
+            raise RuntimeError("device status after e2e")
+
+    result = None
+    if rank == 0:
+        peaks, peak_src = read_peaks()
+        hbm = float(peaks["hbm_gbs"])
+        tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        achieved = counts["attn_bytes"] / attn_s_max / 1e9
+        t_hbm = counts["bytes"] / (hbm * 1e9)
+        t_tc = counts["flops"] / (tc * 1e12)
+        workload = cfg.name
+        clocks = sampler.summary()
+        sm_hz = (clocks["sm_mhz"] or 1965.0) * 1e6
+        result = {
+            "metric": METRIC, "value": world * p.R / step_s, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {
+                "workload": workload, "R": p.R, "B": p.B, "Hq": p.Hq, "Hkv": p.Hkv, "d": p.d,
+                "hidden": p.H, "prefix": list(cfg.prefix), "total_prefix": p.total_prefix,
+                "seed": seed, "kept_rows": counts["kept_rows"],
+                "input_bytes_per_step": int(in_bytes),
+                "l2": f"no flush: {in_bytes / 2**30:.2f} GiB of inputs per step > 126 MB L2",
+                "accumulate": "fp32", "parallelism": f"dp{world} (request-sharded replicas)",
+            },
+            "decisions_per_s": world * counts["decisions"] / step_s,
+            "roofline": {
+                "bound": "hbm", "kernel": "attn_stats_kernel", "achieved": achieved,
+                "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": read_traffic(workload),
+                "algorithmic_bytes_per_launch": counts["attn_bytes"],
+                "ms_per_launch": attn_s_max * 1e3, "peak_source": f"{peak_src} (hbm_gbs)",
+                "note": f"frac of {peak_src} HBM copy bandwidth",
+            },
+            "roofline_step": {
+                "t_hbm_us": t_hbm * 1e6, "t_tensor_us": t_tc * 1e6,
+                "t_mufu_us": counts["exps"] / (16 * 148 * sm_hz) * 1e6,
+                "frac": max(t_hbm, t_tc) / step_s, "bytes": counts["bytes"],
+                "flops": counts["flops"], "exps": counts["exps"],
+                "peaks": f"{peak_src}: hbm {hbm} GB/s, bf16 {tc} TFLOP/s",
+            },
+            "clocks": clocks,
+            "gpu_launches": 3 * args.steps,
+            "e2e": e2e,
+            "impl": "ours",
+        }
+    return result, p
+
+
+def cpu_baseline(p, target_s: float = 12.0) -> dict:
+    """The oracle as it stands, on a bounded sample of the same workload (rank 0, N=1)."""
+    import oracle
+    threads = oracle.num_threads()
+    n0 = max(1, min(p.R, threads // max(1, p.Hkv)))
+    cpu_p = p.subset(range(n0)).to("cpu")
+    t0 = time.perf_counter()
+    oracle.evict(cpu_p)
+    t = time.perf_counter() - t0
+    n = n0
+    if t < target_s / 2 and n0 < p.R:
+        n = int(min(p.R, max(n0 + 1, round(n0 * target_s / max(t, 1e-3)))))
+        cpu_p = p.subset(range(n)).to("cpu")
+        t0 = time.perf_counter()
+        oracle.evict(cpu_p)
+        t = time.perf_counter() - t0
+    return {"value": n / t, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "seconds": t,
+            "sample": f"requests 0..{n - 1} ({n} of {p.R} blocks) of the same workload; "
+                      f"both layers' importance, delta, pooling, mask, top-K, compaction in "
+                      f"float64 (OpenMP over request x kv-head pairs)"}
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The float64 CPU oracle on host cores; each step a bounded sample of the workload."""
+    import oracle
+    cfg = synth.CONFIGS[args.config]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    p = synth.make_problem(cfg, seed=args.config, device=dev)
+    threads = oracle.num_threads()
+    n = max(1, min(p.R, threads // max(1, p.Hkv)))
+    subsets = {}
+
+    def sample(step_idx):
+        start = (step_idx * n) % p.R
+        req = [(start + i) % p.R for i in range(n)]
+        key = tuple(req)
+        if key not in subsets:
+            subsets[key] = p.subset(req).to("cpu")
+        return subsets[key]
+
+    for w in range(args.warmup):
+        oracle.evict(sample(w))
+    total = 0.0
+    for s in range(args.steps):
+        sp = sample(args.warmup + s)
+        t0 = time.perf_counter()
+        oracle.evict(sp)
+        total += time.perf_counter() - t0
+    step_s = total / max(1, args.steps)
+    value = n / step_s
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "R": p.R, "B": p.B, "Hq": p.Hq, "Hkv": p.Hkv, "d": p.d,
+                   "hidden": p.H, "prefix": list(cfg.prefix), "seed": args.config},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{n} requests per step, cycling through the {p.R}-block "
+                                   f"workload; float64, OpenMP over request x kv-head pairs"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=synth.METRIC_CONFIG)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=300),
+            device_id=torch.device("cuda", local_rank))
+    try:
+        result, p = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                result["cpu_baseline"] = cpu_baseline(p)
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

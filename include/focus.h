@@ -1,0 +1,196 @@
+/*
+ * focus.h -- C ABI of libfocus: FOCUS importance-delta token eviction on B200 (sm_100a).
+ *
+ * The method ("FOCUS: DLLMs Know How to Tame Their Compute Bound", pith.science
+ * review page, section "What carries the argument"): for every request's block
+ * of B tokens, I_j is the column sum, over the block's queries and over the
+ * query heads, of the row-wise softmax attention weights token j receives (the
+ * softmax of a query row runs over the request's prefix keys followed by the B
+ * block keys; Referee Report, minor comment on Eq. (2), reads the softmax as
+ * row-wise).  I is taken at layer 0 and from the layer-1 Q/K projections
+ * (Figure 5 caption: eviction happens right after the layer-1 QKProj).  The
+ * importance delta dI = I(layer 1) - I(layer 0) (Eq. 3) is smoothed with
+ * MaxPool1D (window 3, stride 1, same padding; Free-Parameter Ledger, Eq. 15),
+ * already-decoded positions are masked, the top-K still-masked tokens under a
+ * per-request budget K are kept (ties to the lower position), and the kept
+ * tokens' hidden rows are packed into a varlen batch with cu_seqlens
+ * ("The pith": the remaining layers run only on the retained candidates).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor arguments are DEVICE pointers owned by the caller, row-major,
+ *    contiguous.  bf16 tensors are passed as `const void*` holding IEEE bfloat16
+ *    and must be 16-byte aligned; int32/float32 arrays 4-byte aligned; the
+ *    workspace 256-byte aligned.  The library allocates nothing and
+ *    keeps no state between calls; it is thread-safe as long as concurrent
+ *    calls use different workspaces.
+ *  - `stream` is a cudaStream_t (passed as void*; NULL = legacy default stream).
+ *    Every call only enqueues work on `stream` and returns without
+ *    synchronising.  The return value reports host-side validation and launch
+ *    errors.  Problems that only the device can see (budget rows beyond
+ *    `capacity`, malformed cu_prefix, a kernel wait that timed out) are OR-ed
+ *    into a status word inside the workspace; read it with
+ *    focus_read_device_status().
+ *  - Shapes: 1 <= B <= 128; head_dim in {64, 128}; Hq % Hkv == 0 and
+ *    G = Hq / Hkv divides 128; hidden % 8 == 0; pool_window odd and >= 1;
+ *    R >= 1.  Other shapes return FOCUS_ERR_UNSUPPORTED_SHAPE.
+ *  - Per-request budgets are clamped to [0, masked_r] on the device, so
+ *    k_r = min(max(budget[r], 0), masked_r).  k_r depends only on `decoded`
+ *    and `budget`, never on the attention data, so the host scheduler that
+ *    owns both can size `capacity` = sum_r k_r exactly.
+ *  - Kept positions are written in ascending order per request; requests are
+ *    packed in order: request r owns rows cu_seqlens[r] .. cu_seqlens[r+1]-1.
+ */
+#ifndef FOCUS_H_
+#define FOCUS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FOCUS_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define FOCUS_API __attribute__((visibility("default")))
+#else
+#define FOCUS_API
+#endif
+
+typedef enum {
+    FOCUS_OK = 0,
+    FOCUS_ERR_INVALID_ARGUMENT = 1,  /* null/misaligned pointer, negative size, bad scale   */
+    FOCUS_ERR_UNSUPPORTED_SHAPE = 2, /* shape outside the supported set above              */
+    FOCUS_ERR_CAPACITY = 3,          /* device: sum k_r > capacity (extra rows not written) */
+    FOCUS_ERR_WORKSPACE = 4,         /* workspace null, misaligned or too small            */
+    FOCUS_ERR_CUDA = 5,              /* a CUDA runtime/driver call failed                  */
+    FOCUS_ERR_DEVICE_CHECK = 6,      /* device: malformed cu_prefix or kept index          */
+    FOCUS_ERR_TIMEOUT = 7            /* device wait gave up, or status read timed out      */
+} focus_status_t;
+
+/* Problem dimensions, shared by all entry points. */
+typedef struct {
+    int32_t R;             /* requests (blocks) in the batch                          */
+    int32_t B;             /* block size                                              */
+    int32_t Hq;            /* query heads                                             */
+    int32_t Hkv;           /* key/value heads (GQA: query head h reads kv head h/(Hq/Hkv)) */
+    int32_t head_dim;      /* d                                                       */
+    int32_t hidden;        /* hidden size H of the rows that are compacted            */
+    float softmax_scale;   /* logit = softmax_scale * q.k (usually 1/sqrt(d)); finite, >= 0 */
+    int32_t pool_window;   /* MaxPool1D window (odd; the method uses 3)               */
+} focus_dims_t;
+
+/* Bytes of workspace every entry point below needs for `dims` (256-byte aligned). */
+FOCUS_API size_t focus_workspace_size(const focus_dims_t *dims);
+
+/* Zero the workspace's device status word (enqueued on `stream`).  Call once
+ * before the first use of a workspace and whenever the status should restart. */
+FOCUS_API focus_status_t focus_clear_device_status(void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Wait (up to timeout_ms; < 0 waits forever) for the work enqueued so far on
+ * `stream` and return the workspace's device status: FOCUS_OK, or the first of
+ * FOCUS_ERR_TIMEOUT (a kernel wait gave up), FOCUS_ERR_DEVICE_CHECK,
+ * FOCUS_ERR_CAPACITY that is set.  Returns FOCUS_ERR_TIMEOUT without reading
+ * when the stream has not finished in time.  This is the only call that
+ * synchronises.
+ */
+FOCUS_API focus_status_t focus_read_device_status(const void *workspace, void *stream, int timeout_ms);
+
+/*
+ * Attention importance of ONE layer (method step "Delta Calculation", first half):
+ *   I[r][j] = sum over query heads h and block queries i of
+ *             softmax_i( softmax_scale * q[r,i,h,:] . key[:] )[prefix_len_r + j]
+ * where the keys of request r are its prefix rows k_prefix[cu_prefix[r] ..
+ * cu_prefix[r+1]-1, h/G, :] followed by its block rows k_block[r, 0..B-1, h/G, :].
+ *
+ *   q            [R, B, Hq, d]        bf16
+ *   k_prefix     [total_prefix, Hkv, d] bf16 (may be NULL when total_prefix == 0)
+ *   cu_prefix    [R + 1] int32        cu_prefix[0] = 0, non-decreasing, cu_prefix[R] <= total_prefix
+ *   total_prefix rows of k_prefix
+ *   k_block      [R, B, Hkv, d]       bf16
+ *   importance   [R, B] float32       output
+ * A malformed cu_prefix entry sets FOCUS_ERR_DEVICE_CHECK in the device status
+ * and that request is computed with no prefix.
+ */
+FOCUS_API focus_status_t focus_attn_stats(const focus_dims_t *dims, const void *q, const void *k_prefix,
+                                const int32_t *cu_prefix, int64_t total_prefix,
+                                const void *k_block, float *importance, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+/*
+ * Importance delta, smoothing and mask (method steps Eq. 3, MaxPool1D, mask):
+ *   delta[r][j] = max_{|t-j| <= pool_window/2, 0 <= t < B} (i1[r][t] - i0[r][t])
+ *   delta[r][j] = -inf where decoded[r][j] != 0
+ *   i0, i1 [R, B] float32; decoded [R, B] uint8 (nonzero = decoded); delta [R, B] float32 out.
+ * raw_delta (nullable) receives i1 - i0 before pooling.
+ */
+FOCUS_API focus_status_t focus_importance_delta(const focus_dims_t *dims, const float *i0, const float *i1,
+                                      const uint8_t *decoded, float *delta, float *raw_delta,
+                                      void *stream);
+
+/*
+ * Top-K candidate selection (method step "Token Eviction", selection half):
+ *   k_r = min(max(budget[r], 0), #{j : decoded[r][j] == 0})
+ *   kept_idx[cu_seqlens[r] ..] = the k_r positions ranked first by
+ *                                (delta desc, position asc), in ascending position order
+ *   cu_seqlens[0] = 0, cu_seqlens[r+1] = cu_seqlens[r] + k_r
+ *   delta [R, B] float32 (as produced by focus_importance_delta); budget [R] int32;
+ *   kept_idx [capacity] int32 out; cu_seqlens [R + 1] int32 out.
+ * Rows beyond `capacity` are not written and FOCUS_ERR_CAPACITY is set in the
+ * device status (cu_seqlens is still complete).
+ */
+FOCUS_API focus_status_t focus_topk_select(const focus_dims_t *dims, const float *delta,
+                                 const uint8_t *decoded, const int32_t *budget, int32_t *kept_idx,
+                                 int32_t *cu_seqlens, int64_t capacity, void *workspace,
+                                 size_t workspace_bytes, void *stream);
+
+/*
+ * Compaction (method step "Token Eviction", eviction half): bit copy
+ *   packed[cu_seqlens[r] + t][:] = hidden[r][kept_idx[cu_seqlens[r] + t]][:]
+ *   hidden [R, B, H] bf16; kept_idx, cu_seqlens as above; packed [capacity, H] bf16 out.
+ * Rows at or beyond `capacity` are skipped (FOCUS_ERR_CAPACITY in the device
+ * status); a kept index outside [0, B) skips its row (FOCUS_ERR_DEVICE_CHECK).
+ */
+FOCUS_API focus_status_t focus_compact(const focus_dims_t *dims, const void *hidden, const int32_t *kept_idx,
+                             const int32_t *cu_seqlens, void *packed, int64_t capacity,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The whole eviction step, fused, on one stream: layer-0 and layer-1
+ * importance, delta, MaxPool1D, mask, top-K, compaction.  Arguments as in the
+ * calls above; q0/k0_* are layer 0, q1/k1_* the layer-1 Q/K projections, both
+ * layers share cu_prefix/total_prefix.  delta_out (pooled and masked), i0_out
+ * and i1_out ([R, B] float32) are optional (NULL skips them).
+ */
+FOCUS_API focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void *k0_prefix,
+                           const void *k0_block, const void *q1, const void *k1_prefix,
+                           const void *k1_block, const int32_t *cu_prefix, int64_t total_prefix,
+                           const void *hidden, const uint8_t *decoded, const int32_t *budget,
+                           int32_t *kept_idx, int32_t *cu_seqlens, void *packed, int64_t capacity,
+                           float *delta_out, float *i0_out, float *i1_out, void *workspace,
+                           size_t workspace_bytes, void *stream);
+
+/*
+ * Tracing hook: when `start_event` and `stop_event` (cudaEvent_t, passed as void*)
+ * are non-NULL, every later focus_evict / focus_attn_stats call records
+ * start_event on its stream right before its attention-statistics kernel and
+ * stop_event right after it, so the caller can time that kernel alone with
+ * cudaEventElapsedTime.  NULL, NULL turns the hook off.  The setting is
+ * process-wide; set it from the thread that issues the calls.
+ */
+FOCUS_API void focus_set_trace_events(void *start_event, void *stop_event);
+
+/* Human-readable name of a status code (static string). */
+FOCUS_API const char *focus_status_string(focus_status_t status);
+
+/* FOCUS_ABI_VERSION of the loaded library. */
+FOCUS_API int focus_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FOCUS_H_ */

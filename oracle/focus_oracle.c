@@ -33,7 +33,8 @@
  * Arithmetic is float64 throughout.  bf16 inputs are widened exactly.  Each
  * function is a direct transcription of its definition: no blocking, fusion or
  * reordering beyond what the definition states.  OpenMP (when compiled with
- * -fopenmp) only splits the outer loop over independent requests.
+ * -fopenmp) only splits the outer loop over independent (request, kv head)
+ * pairs; their contributions to I are added afterwards in kv-head order.
  */
 #include <math.h>
 #include <stdint.h>
@@ -99,12 +100,19 @@ int focus_oracle_importance(int R, int B, int Hq, int Hkv, int d, double scale,
         if (cu_prefix[r + 1] < cu_prefix[r])
             return ORACLE_BAD_ARGUMENT;
     const int G = Hq / Hkv;
+    /* part[r][g][j]: the contribution of the G query heads that read kv head g. */
+    double *part = (double *)calloc((size_t)R * Hkv * B, sizeof(double));
+    if (!part)
+        return ORACLE_NO_MEMORY;
     int failed = 0;
 
 #pragma omp parallel for schedule(dynamic, 1)
-    for (int r = 0; r < R; ++r) {
+    for (long long task = 0; task < (long long)R * Hkv; ++task) {
+        const int r = (int)(task / Hkv);
+        const int g = (int)(task % Hkv);
         const int L = cu_prefix[r + 1] - cu_prefix[r];
         const int N = L + B;
+        double *acc = part + ((size_t)r * Hkv + g) * B;
         double *s = (double *)malloc(sizeof(double) * (size_t)N);
         double *qrow = (double *)malloc(sizeof(double) * (size_t)d);
         double *keys = (double *)malloc(sizeof(double) * (size_t)N * (size_t)d);
@@ -114,46 +122,50 @@ int focus_oracle_importance(int R, int B, int Hq, int Hkv, int d, double scale,
             failed = 1;
             continue;
         }
-        for (int j = 0; j < B; ++j)
-            out[(size_t)r * B + j] = 0.0;
-
-        for (int g = 0; g < Hkv; ++g) {
-            /* Key list of kv head g: prefix keys, then block keys. */
-            for (int j = 0; j < N; ++j) {
-                const uint16_t *src;
-                if (j < L)
-                    src = k_prefix + (((size_t)cu_prefix[r] + j) * Hkv + g) * d;
-                else
-                    src = k_block + (((size_t)r * B + (j - L)) * Hkv + g) * d;
+        /* Key list of kv head g: prefix keys, then block keys. */
+        for (int j = 0; j < N; ++j) {
+            const uint16_t *src;
+            if (j < L)
+                src = k_prefix + (((size_t)cu_prefix[r] + j) * Hkv + g) * d;
+            else
+                src = k_block + (((size_t)r * B + (j - L)) * Hkv + g) * d;
+            for (int c = 0; c < d; ++c)
+                keys[(size_t)j * d + c] = bf16_bits_to_double(src[c]);
+        }
+        for (int h = g * G; h < (g + 1) * G; ++h) {
+            for (int i = 0; i < B; ++i) {
+                const uint16_t *qs = q + (((size_t)r * B + i) * Hq + h) * d;
                 for (int c = 0; c < d; ++c)
-                    keys[(size_t)j * d + c] = bf16_bits_to_double(src[c]);
-            }
-            for (int h = g * G; h < (g + 1) * G; ++h) {
-                for (int i = 0; i < B; ++i) {
-                    const uint16_t *qs = q + (((size_t)r * B + i) * Hq + h) * d;
+                    qrow[c] = bf16_bits_to_double(qs[c]);
+                double m = -INFINITY;
+                for (int j = 0; j < N; ++j) {
+                    double dot = 0.0;
                     for (int c = 0; c < d; ++c)
-                        qrow[c] = bf16_bits_to_double(qs[c]);
-                    double m = -INFINITY;
-                    for (int j = 0; j < N; ++j) {
-                        double dot = 0.0;
-                        for (int c = 0; c < d; ++c)
-                            dot += qrow[c] * keys[(size_t)j * d + c];
-                        s[j] = scale * dot;
-                        if (s[j] > m)
-                            m = s[j];
-                    }
-                    double Z = 0.0;
-                    for (int j = 0; j < N; ++j)
-                        Z += exp(s[j] - m);
-                    for (int j = 0; j < B; ++j)
-                        out[(size_t)r * B + j] += exp(s[L + j] - m) / Z;
+                        dot += qrow[c] * keys[(size_t)j * d + c];
+                    s[j] = scale * dot;
+                    if (s[j] > m)
+                        m = s[j];
                 }
+                double Z = 0.0;
+                for (int j = 0; j < N; ++j)
+                    Z += exp(s[j] - m);
+                for (int j = 0; j < B; ++j)
+                    acc[j] += exp(s[L + j] - m) / Z;
             }
         }
         free(s);
         free(qrow);
         free(keys);
     }
+    /* I[r][j] = sum over kv heads g (in order) of the group contributions. */
+    for (int r = 0; r < R; ++r)
+        for (int j = 0; j < B; ++j) {
+            double sum = 0.0;
+            for (int g = 0; g < Hkv; ++g)
+                sum += part[((size_t)r * Hkv + g) * B + j];
+            out[(size_t)r * B + j] = sum;
+        }
+    free(part);
     return failed ? ORACLE_NO_MEMORY : ORACLE_OK;
 }
 

@@ -1,0 +1,148 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point the header
+declares, and its host-side validation rejects bad arguments before touching
+CUDA.  No call here reaches a kernel launch."""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import attention_delta_token_b200 as F
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "focus.h")
+
+OK, INVALID, UNSUPPORTED, CAPACITY, WORKSPACE, CUDA, DEVCHECK, TIMEOUT = range(8)
+A = 0x100000  # a 256-byte-aligned fake device address (never dereferenced here)
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return re.findall(r"FOCUS_API\s+[\w\s\*]*?\b(focus_\w+)\s*\(", src)
+
+
+def test_header_declares_the_entry_points():
+    names = set(declared_functions())
+    for want in ("focus_attn_stats", "focus_importance_delta", "focus_topk_select",
+                 "focus_compact", "focus_evict", "focus_workspace_size",
+                 "focus_read_device_status", "focus_clear_device_status"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(F.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version():
+    for code, name in F.STATUS.items():
+        assert F.focus_status_string(code) == name
+    assert F.focus_abi_version() == 1
+
+
+def dims(**kw):
+    base = dict(R=4, B=32, Hq=32, Hkv=8, head_dim=128, hidden=4096, softmax_scale=None,
+                pool_window=3)
+    base.update(kw)
+    return F.make_dims(**base)
+
+
+def test_workspace_size():
+    d = dims()
+    n = F.focus_workspace_size(d)
+    # status (256) + order (R int32, rounded to 256) + 2 layers x R x Hkv x MT x B fp32
+    assert n == 256 + 256 + 2 * 4 * 8 * 1 * 32 * 4
+    d3 = dims(B=128)  # G*B = 512 -> 4 row tiles
+    assert F.focus_workspace_size(d3) == 256 + 256 + 2 * 4 * 8 * 4 * 128 * 4
+    assert F._lib.focus_workspace_size(None) == 0
+    assert F._lib.focus_workspace_size(ctypes.byref(dims(B=0))) == 0
+
+
+BAD_DIMS = [
+    (dict(R=0), INVALID), (dict(B=0), INVALID), (dict(Hq=0), INVALID),
+    (dict(softmax_scale=-1.0), INVALID), (dict(softmax_scale=math.nan), INVALID),
+    (dict(softmax_scale=math.inf), INVALID), (dict(pool_window=0), INVALID),
+    (dict(B=129), UNSUPPORTED), (dict(head_dim=96), UNSUPPORTED), (dict(head_dim=256), UNSUPPORTED),
+    (dict(Hq=30, Hkv=8), UNSUPPORTED), (dict(Hq=24, Hkv=8), UNSUPPORTED),
+    (dict(Hq=256, Hkv=1), UNSUPPORTED), (dict(hidden=4092), UNSUPPORTED),
+    (dict(pool_window=2), UNSUPPORTED),
+]
+
+
+def evict_args(d, **over):
+    ws = F.focus_workspace_size(dims()) if F._lib.focus_workspace_size(ctypes.byref(d)) == 0 \
+        else F.focus_workspace_size(d)
+    a = dict(q0=A, k0p=A, k0b=A, q1=A, k1p=A, k1b=A, cu=A, total=100, hidden=A, dec=A,
+             budget=A, kept=A, cu_s=A, packed=A, cap=16, delta=None, i0=None, i1=None,
+             ws=A, ws_bytes=ws, stream=None)
+    a.update(over)
+    return a
+
+
+def call_evict(d, a):
+    return F._lib.focus_evict(ctypes.byref(d), a["q0"], a["k0p"], a["k0b"], a["q1"], a["k1p"],
+                              a["k1b"], a["cu"], a["total"], a["hidden"], a["dec"], a["budget"],
+                              a["kept"], a["cu_s"], a["packed"], a["cap"], a["delta"], a["i0"],
+                              a["i1"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("over,code", BAD_DIMS)
+def test_bad_dims_rejected_everywhere(over, code):
+    d = dims(**over)
+    if "softmax_scale" in over:
+        d.softmax_scale = over["softmax_scale"]
+    assert call_evict(d, evict_args(d)) == code
+    assert F._lib.focus_attn_stats(ctypes.byref(d), A, A, A, 100, A, A, A, 1 << 20, None) == code
+    assert F._lib.focus_importance_delta(ctypes.byref(d), A, A, A, A, None, None) == code
+    assert F._lib.focus_topk_select(ctypes.byref(d), A, A, A, A, A, 16, A, 1 << 20, None) == code
+    assert F._lib.focus_compact(ctypes.byref(d), A, A, A, A, 16, A, 1 << 20, None) == code
+
+
+BAD_PTRS = [
+    (dict(q0=None), INVALID), (dict(q1=A + 8), INVALID), (dict(k0b=None), INVALID),
+    (dict(k1p=None), INVALID), (dict(cu=None), INVALID), (dict(cu=A + 2), INVALID),
+    (dict(hidden=A + 4), INVALID), (dict(dec=None), INVALID), (dict(budget=None), INVALID),
+    (dict(kept=None), INVALID), (dict(packed=A + 8), INVALID), (dict(cu_s=None), INVALID),
+    (dict(delta=A + 1), INVALID), (dict(i0=A + 2), INVALID), (dict(total=-1), INVALID),
+    (dict(total=1 << 40), INVALID), (dict(cap=-1), INVALID),
+    (dict(ws=None), WORKSPACE), (dict(ws=A + 16), WORKSPACE), (dict(ws_bytes=100), WORKSPACE),
+]
+
+
+@pytest.mark.parametrize("over,code", BAD_PTRS)
+def test_bad_pointers_rejected(over, code):
+    d = dims()
+    assert call_evict(d, evict_args(d, **over)) == code
+
+
+def test_other_entry_points_check_pointers():
+    d = dims()
+    ws = F.focus_workspace_size(d)
+    L = F._lib
+    assert L.focus_attn_stats(ctypes.byref(d), None, A, A, 100, A, A, A, ws, None) == INVALID
+    assert L.focus_attn_stats(ctypes.byref(d), A, None, A, 100, A, A, A, ws, None) == INVALID
+    assert L.focus_attn_stats(ctypes.byref(d), A, A, A, 100, A, A + 2, A, ws, None) == INVALID
+    assert L.focus_attn_stats(ctypes.byref(d), A, A, A, 100, A, A, A, ws - 4, None) == WORKSPACE
+    assert L.focus_importance_delta(ctypes.byref(d), A, None, A, A, None, None) == INVALID
+    assert L.focus_importance_delta(ctypes.byref(d), A, A, A, A + 1, None, None) == INVALID
+    assert L.focus_topk_select(ctypes.byref(d), A, A, None, A, A, 16, A, ws, None) == INVALID
+    assert L.focus_topk_select(ctypes.byref(d), A, A, A, A, A, -3, A, ws, None) == INVALID
+    assert L.focus_topk_select(ctypes.byref(d), A, A, A, A, A, 16, None, ws, None) == WORKSPACE
+    assert L.focus_compact(ctypes.byref(d), A + 8, A, A, A, 16, A, ws, None) == INVALID
+    assert L.focus_compact(ctypes.byref(d), A, A, A, A, 16, A, 8, None) == WORKSPACE
+    assert L.focus_read_device_status(None, None, 10) == WORKSPACE
+    assert L.focus_clear_device_status(None, 1024, None) == WORKSPACE
+
+
+def test_plan_capacity_matches_oracle_counts():
+    import oracle
+    import synth
+    for cfg in range(5):
+        p = synth.make_problem(cfg, overrides=dict(R=min(synth.CONFIGS[cfg].R, 12), d=64,
+                                                   prefix=("fixed", 0)))
+        _, cu, _ = oracle.select(np.zeros((p.R, p.B)), p.decoded, p.budget)
+        assert F.plan_capacity(p.decoded, p.budget) == int(cu[-1])

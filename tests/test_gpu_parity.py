@@ -1,0 +1,217 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle.
+
+Small cases are compared element by element; they span several 128-key tiles,
+ragged tails, several 128-row query tiles, both head dims, GQA group sizes
+1..16, odd block sizes and empty prefixes.  The five full-size workloads run in
+the launch configuration the benchmark times and are compared on sampled
+requests, which the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from focus_testutil import (assert_close_delta, assert_close_importance, check_packed,
+                            check_selection, hidden_bits, run_evict)
+
+pytestmark = pytest.mark.gpu
+
+SMALL_CASES = {
+    "tiny": (0, {}, False),
+    "tiny_wide": (0, {}, True),
+    "sdar_r6_ragged": (1, dict(R=6, prefix=("uniform", 0, 700)), False),
+    "sdar_r6_ragged_wide": (1, dict(R=6, prefix=("uniform", 0, 700)), True),
+    "block128_mt4": (3, dict(R=3, prefix=("uniform", 100, 400)), True),
+    "ragged_g8_ties": (4, dict(R=8, prefix=("loguniform", 600)), True),
+    "d64_g1_b20": (0, dict(R=5, B=20, Hq=4, Hkv=4, d=64, H=64, prefix=("uniform", 0, 300),
+                          decoded=("uniform", 0.0, 0.8), lift=("frac", 0.2),
+                          budget=("ceil", 0.3)), True),
+    "g16_b16_mt2": (1, dict(R=3, B=16, Hq=32, Hkv=2, prefix=("uniform", 1, 260)), True),
+    "b1_g1": (0, dict(R=4, B=1, Hq=8, Hkv=8, d=64, H=64, prefix=("uniform", 0, 200),
+                      decoded=("exact", 0), lift=("count", 0), budget=("fixed", 1)), True),
+    "no_prefix": (1, dict(R=4, prefix=("fixed", 0)), True),
+    "g2_b32_neighbours": (0, dict(R=3, prefix=("uniform", 0, 300)), True),
+    "d64_b128": (3, dict(R=2, d=64, Hq=8, Hkv=2, prefix=("uniform", 0, 300)), True),
+}
+
+
+@pytest.fixture(scope="module")
+def orc():
+    import oracle
+    return oracle.default()
+
+
+def _compare_full(p, out, ref):
+    assert out["status"] == 0, out["status"]
+    assert_close_importance(out["i0"], ref["i0"], "I0")
+    assert_close_importance(out["i1"], ref["i1"], "I1")
+    assert_close_delta(out["delta"], ref["pooled"])
+    np.testing.assert_array_equal(out["cu_seqlens"], ref["cu_seqlens"])
+    check_selection(out["kept"], out["cu_seqlens"], ref["pooled"], p.decoded.cpu().numpy(),
+                    p.budget.cpu().numpy())
+    check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))
+
+
+@pytest.mark.parametrize("case", sorted(SMALL_CASES))
+def test_small_elementwise(case, orc):
+    cfg, ov, wide = SMALL_CASES[case]
+    p = synth.make_problem(cfg, seed=100 + sorted(SMALL_CASES).index(case), wide_logits=wide,
+                           overrides=ov)
+    ref = orc.evict(p)
+    out = run_evict(p.to("cuda"))
+    _compare_full(p, out, ref)
+
+
+def _sample_requests(p, n=6):
+    L = p.prefix_len
+    dec = p.decoded.cpu().numpy()
+    masked = (dec == 0).sum(1)
+    pick = [int(np.argmax(L)), int(np.argmin(L)), int(np.argmax(masked)), int(np.argmin(masked))]
+    pick += [r for (r, _, _) in p.tie_pairs[:2]]
+    rng = np.random.default_rng(0)
+    pick += rng.choice(p.R, size=min(p.R, n), replace=False).tolist()
+    return sorted(set(pick))
+
+
+@pytest.mark.parametrize("cfg", [0, 1, 2, 3, 4])
+def test_full_config_sampled(cfg, orc):
+    """The benchmark's launch configuration on the full workload; the oracle checks a
+    sample of requests one by one, and cu_seqlens in full."""
+    p = synth.make_problem(cfg)
+    out = run_evict(p.to("cuda"))
+    assert out["status"] == 0
+    req = _sample_requests(p)
+    sub = p.subset(req)
+    ref = orc.evict(sub)
+    assert_close_importance(out["i0"][req], ref["i0"], "I0")
+    assert_close_importance(out["i1"][req], ref["i1"], "I1")
+    assert_close_delta(out["delta"][req], ref["pooled"])
+    # cu_seqlens in full: the kept counts do not depend on the attention data
+    _, cu_all, _ = orc.select(np.zeros((p.R, p.B)), p.decoded, p.budget)
+    np.testing.assert_array_equal(out["cu_seqlens"], cu_all)
+    check_selection(out["kept"], out["cu_seqlens"], ref["pooled"], p.decoded.cpu().numpy(),
+                    p.budget.cpu().numpy(), requests=req)
+    check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))
+    # every request: valid selection shape
+    assert np.isfinite(out["i0"]).all() and np.isfinite(out["i1"]).all()
+
+
+def test_duplicate_keys_give_equal_columns():
+    """A duplicated block key (same K rows at both layers) gets bit-equal I columns."""
+    p = synth.make_problem(4, overrides=dict(R=24, prefix=("loguniform", 900), tie_frac=0.5))
+    assert p.tie_pairs
+    out = run_evict(p.to("cuda"))
+    for (r, a, b) in p.tie_pairs:
+        assert out["i0"][r, a] == out["i0"][r, b], (r, a, b)
+        assert out["i1"][r, a] == out["i1"][r, b], (r, a, b)
+
+
+def test_deterministic():
+    p = synth.make_problem(1, overrides=dict(R=8), wide_logits=True).to("cuda")
+    a, b = run_evict(p), run_evict(p)
+    for k in ("i0", "i1", "delta", "kept", "cu_seqlens", "packed"):
+        np.testing.assert_array_equal(a[k], b[k], err_msg=k)
+
+
+def test_standalone_chain_matches_fused():
+    """attn_stats x2 -> importance_delta -> topk_select -> compact reproduces
+    focus_evict bit for bit (same reduction order everywhere)."""
+    import attention_delta_token_b200 as F
+    p = synth.make_problem(4, overrides=dict(R=16, prefix=("loguniform", 1500)),
+                           wide_logits=True).to("cuda")
+    fused = run_evict(p)
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+    ws = F.Workspace(dims)
+    i0 = torch.empty(p.R, p.B, device="cuda")
+    i1 = torch.empty_like(i0)
+    F.focus_attn_stats(dims, p.q0, p.k0_prefix, p.cu_prefix, p.k0_block, i0, ws)
+    F.focus_attn_stats(dims, p.q1, p.k1_prefix, p.cu_prefix, p.k1_block, i1, ws)
+    delta = torch.empty_like(i0)
+    raw = torch.empty_like(i0)
+    F.focus_importance_delta(dims, i0, i1, p.decoded, delta, raw)
+    cap = F.plan_capacity(p.decoded, p.budget)
+    kept = torch.empty(cap, dtype=torch.int32, device="cuda")
+    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+    F.focus_topk_select(dims, delta, p.decoded, p.budget, kept, cu, ws)
+    packed = torch.empty(cap, p.H, dtype=torch.bfloat16, device="cuda")
+    F.focus_compact(dims, p.hidden, kept, cu, packed, ws)
+    assert F.focus_read_device_status(ws) == 0
+    np.testing.assert_array_equal(i0.cpu().numpy(), fused["i0"].astype(np.float32))
+    np.testing.assert_array_equal(i1.cpu().numpy(), fused["i1"].astype(np.float32))
+    np.testing.assert_array_equal(delta.cpu().numpy(), fused["delta"].astype(np.float32))
+    np.testing.assert_array_equal((i1 - i0).cpu().numpy(), raw.cpu().numpy())
+    np.testing.assert_array_equal(kept.cpu().numpy(), fused["kept"])
+    np.testing.assert_array_equal(cu.cpu().numpy(), fused["cu_seqlens"])
+    np.testing.assert_array_equal(packed.view(torch.int16).cpu().numpy().view(np.uint16),
+                                  fused["packed"])
+
+
+def test_standalone_steps_vs_oracle(orc):
+    """Each stand-alone entry point against the oracle's step of the same name."""
+    import attention_delta_token_b200 as F
+    p = synth.make_problem(1, overrides=dict(R=5, prefix=("uniform", 0, 500)), wide_logits=True)
+    g = p.to("cuda")
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+    ws = F.Workspace(dims)
+    i0 = torch.empty(p.R, p.B, device="cuda")
+    F.focus_attn_stats(dims, g.q0, g.k0_prefix, g.cu_prefix, g.k0_block, i0, ws)
+    want = orc.importance(p.q0, p.k0_prefix, p.cu_prefix, p.k0_block, Hq=p.Hq, Hkv=p.Hkv,
+                          scale=p.scale)
+    assert_close_importance(i0.cpu().numpy(), want, "attn_stats")
+    # delta / pool / mask on exact float32 inputs: exact
+    rng = np.random.default_rng(3)
+    a = rng.normal(size=(p.R, p.B)).astype(np.float32)
+    b = rng.normal(size=(p.R, p.B)).astype(np.float32)
+    delta = torch.empty(p.R, p.B, device="cuda")
+    F.focus_importance_delta(dims, torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda(),
+                             g.decoded, delta)
+    _, pooled = orc.delta_pool_mask(a.astype(np.float64), b.astype(np.float64), p.decoded)
+    np.testing.assert_array_equal(delta.cpu().numpy(),
+                                  pooled.astype(np.float32))  # b - a is exact in fp64 -> fp32 rounding once
+    # select on a coarse grid (many exact ties): bit-exact
+    vals = (rng.integers(-3, 4, size=(p.R, p.B)) * 0.5).astype(np.float32)
+    vals[p.decoded.numpy() != 0] = -np.inf
+    cap = F.plan_capacity(p.decoded, p.budget)
+    kept = torch.empty(cap, dtype=torch.int32, device="cuda")
+    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+    F.focus_topk_select(dims, torch.from_numpy(vals).cuda(), g.decoded, g.budget, kept, cu, ws)
+    okept, ocu, _ = orc.select(vals.astype(np.float64), p.decoded, p.budget)
+    np.testing.assert_array_equal(kept.cpu().numpy(), okept)
+    np.testing.assert_array_equal(cu.cpu().numpy(), ocu)
+    packed = torch.empty(cap, p.H, dtype=torch.bfloat16, device="cuda")
+    F.focus_compact(dims, g.hidden, kept, cu, packed, ws)
+    want_packed = orc.compact(p.hidden, okept, ocu)
+    np.testing.assert_array_equal(packed.view(torch.int16).cpu().numpy().view(np.uint16), want_packed)
+    assert F.focus_read_device_status(ws) == 0
+
+
+def test_zero_budget_and_all_decoded(orc):
+    p = synth.make_problem(1, overrides=dict(R=4, prefix=("uniform", 0, 300)))
+    p.budget = torch.tensor([0, -5, 3, 40], dtype=torch.int32)
+    dec = p.decoded.clone()
+    dec[2] = 1  # request 2 fully decoded: nothing to keep
+    p.decoded = dec
+    ref = orc.evict(p)
+    out = run_evict(p.to("cuda"))
+    _compare_full(p, out, ref)
+    assert out["cu_seqlens"][1] == 0 and out["cu_seqlens"][2] == 0
+
+
+def test_capacity_overflow_reports_and_stays_in_bounds():
+    import attention_delta_token_b200 as F
+    p = synth.make_problem(1, overrides=dict(R=4, prefix=("uniform", 0, 300))).to("cuda")
+    need = F.plan_capacity(p.decoded, p.budget)
+    assert need >= 3
+    out = run_evict(p, capacity=need - 2)
+    assert out["status"] == 3  # FOCUS_ERR_CAPACITY
+    assert out["cu_seqlens"][-1] == need
+
+
+def test_malformed_cu_prefix_reports():
+    import attention_delta_token_b200 as F
+    p = synth.make_problem(1, overrides=dict(R=3, prefix=("uniform", 10, 100))).to("cuda")
+    bad = p.cu_prefix.clone()
+    bad[2] = bad[3] + 5  # beyond total_prefix and decreasing
+    p.cu_prefix = bad
+    out = run_evict(p)
+    assert out["status"] == 6  # FOCUS_ERR_DEVICE_CHECK

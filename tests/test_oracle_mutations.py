@@ -15,8 +15,8 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "focus_oracle.c")
 MUTATIONS = {
     "scale_dropped": ("s[j] = scale * dot;", "s[j] = dot;"),
     "prefix_left_out_of_denominator": (
-        "for (int j = 0; j < N; ++j)\n                        Z += exp",
-        "for (int j = L; j < N; ++j)\n                        Z += exp"),
+        "for (int j = 0; j < N; ++j)\n                    Z += exp",
+        "for (int j = L; j < N; ++j)\n                    Z += exp"),
     "prefix_column_read": ("exp(s[L + j] - m) / Z", "exp(s[j] - m) / Z"),
     "head_mapping_modulo": ("for (int h = g * G; h < (g + 1) * G; ++h)",
                             "for (int h = g; h < Hq; h += Hkv)"),
