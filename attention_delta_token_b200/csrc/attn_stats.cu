@@ -7,22 +7,28 @@
 // row (query) wise.  Each query row's softmax runs over the request's prefix
 // keys followed by its B block keys; I_j also sums over the query heads.
 //
-// One CTA handles one (layer, request, kv head, 128-row query tile) in a single
-// pass over the keys:
-//   warp 0      TMA producer: the Q tile once, then 128-key tiles of the prefix
-//               and finally the block keys, through a 2-stage shared-memory ring;
-//   warp 1      allocates TMEM and issues tcgen05.mma (M=128 rows, N=128 keys,
-//               K=d, bf16 in, fp32 out) into two ping-pong TMEM S buffers;
-//   warps 2-5   one TMEM lane (= one query row) per thread: online row max m
-//               and sum-exp l over every key tile (exp2 on the SFU).  The block
-//               tile comes last, so when it arrives m and l are final and the
-//               row's weights p_ij = 2^(s_ij - m)/l of the B block columns are
-//               formed straight from the same S values, without a second pass.
-//               Column sums over the 128 rows (warp butterfly, then the four
-//               warps in fixed order) go to `partial`; no float atomics, so the
-//               result is deterministic and equal keys give bit-equal columns.
-// Two CTAs fit on an SM (99 KB shared memory and 256 TMEM columns each), so one
-// CTA's prologue/epilogue overlaps the other's streaming.
+// Work item = one (layer, request, kv head, 128-row query tile).  The kernel is
+// persistent: two CTAs per SM, each walking the items (longest prefix first) with
+// a stride of the grid size.  Per CTA (10 warps):
+//   warp 0      TMA producer: the item's Q tile (once per item, as soon as the
+//               previous item's MMAs have released it), then 128-key tiles of the
+//               prefix and finally the block keys, through a 2-stage ring;
+//   warp 1      allocates TMEM and issues tcgen05.mma (M=128 query rows, N=128
+//               keys, K=d; bf16 in, fp32 out) into two ping-pong TMEM S buffers;
+//   warps 2-9   two softmax warpgroups.  Warpgroup h reads columns [64h, 64h+64)
+//               of every S tile (one TMEM lane = one query row per thread) and
+//               keeps an online row max m and sum-exp l over its columns.  The
+//               block tile comes last: the two halves' (m, l) are merged through
+//               shared memory, the row's weights p_ij = 2^(s_ij - M)/L of the B
+//               block columns are formed straight from the S values already in
+//               registers (no second pass over the keys), and their column sums
+//               over the 128 rows (warp butterfly, then the four lane quadrants in
+//               fixed order) go to `partial`.  No float atomics: the result is
+//               deterministic and equal keys give bit-equal columns.
+// A fraction of each full tile's exponentials runs on the FMA pipe (2^x by
+// Cody-Waite style range reduction to [-1/2, 1/2] and a degree-3 minimax
+// polynomial fitted for this file, max relative error 7.5e-5), the rest on the
+// SFU, so neither pipe is the bottleneck.
 #include <math.h>
 
 #include "focus_device.cuh"
@@ -33,6 +39,15 @@ namespace focus {
 namespace {
 
 constexpr uint32_t kChunkBytes = kTileRows * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
+constexpr int kHalf = kTileKeys / 2;               // S columns per softmax warpgroup
+
+#ifndef FOCUS_EXP_MODE
+#define FOCUS_EXP_MODE 0  // full prefix tiles: 0 fp32 SFU exp2, 1 packed f16 pairs, 2 f16 quads
+#endif
+
+#ifndef FOCUS_POLY_EVERY
+#define FOCUS_POLY_EVERY 0  // > 0: every n-th column pair of a full tile uses the FMA-pipe exp2
+#endif
 
 template <int HEAD_DIM>
 struct AttnSmem {
@@ -42,9 +57,59 @@ struct AttnSmem {
     static constexpr uint32_t kKOff = kTileBytes;
     static constexpr uint32_t kBarOff = kKOff + kStages * kTileBytes;
     static constexpr uint32_t kRedOff = kBarOff + 256;
-    static constexpr uint32_t kBytes = kRedOff + 4 * 128 * sizeof(float);
+    static constexpr uint32_t kStatOff = kRedOff + 4 * 128 * sizeof(float);
+    static constexpr uint32_t kBytes = kStatOff + 2 * 128 * sizeof(float2);
     static constexpr uint32_t kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
+
+struct Item {
+    int layer, r, kvh, mt, pstart, L, n_pre;
+    bool bad;
+};
+
+__device__ __forceinline__ Item decode_item(const AttnParams &p, int it) {
+    Item w;
+    const int per_req = p.n_layers * p.Hkv * p.MT;
+    const int rank = it / per_req;
+    int rem = it - rank * per_req;
+    w.layer = rem / (p.Hkv * p.MT);
+    rem -= w.layer * p.Hkv * p.MT;
+    w.kvh = rem / p.MT;
+    w.mt = rem - w.kvh * p.MT;
+    w.r = p.order ? p.order[rank] : rank;
+    w.pstart = p.cu_prefix[w.r];
+    w.L = p.cu_prefix[w.r + 1] - w.pstart;
+    w.bad = w.pstart < 0 || w.L < 0 || static_cast<long long>(w.pstart) + w.L > p.total_prefix;
+    if (w.bad) {
+        w.L = 0;
+        w.pstart = 0;
+    }
+    w.n_pre = (w.L + kTileKeys - 1) / kTileKeys;
+    return w;
+}
+
+// 2^x for x <= 0 on the FMA/ALU pipes.  x = n + f with n = round(x) (the 1.5*2^23
+// shifter leaves n in the low mantissa bits of t), f in [-1/2, 1/2];
+// 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 (relative-error minimax fit on [-1/2, 1/2]);
+// 2^n is applied by adding n to the exponent field.  x is clamped at -125 so the
+// result stays a normal float (2^-125 is negligible against a sum >= 1).
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+    constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f;
+    constexpr float c2 = 0.2426111400127411f, c3 = 0.0551716573536396f;
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 t = __fadd2_rn(x, make_float2(kShift, kShift));
+    const float2 n = __fadd2_rn(t, make_float2(-kShift, -kShift));
+    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+    float2 q = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+    q = __ffma2_rn(q, f, make_float2(c1, c1));
+    q = __ffma2_rn(q, f, make_float2(c0, c0));
+    float2 y;
+    y.x = __int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23));
+    y.y = __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23));
+    return y;
+}
 
 // Loads 32 TMEM columns of this thread's lane into v[OFF .. OFF+31].
 template <int OFF>
@@ -69,6 +134,55 @@ __device__ __forceinline__ float warp_colsum32(float *x, int lane) {
     return x[0];
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Max of v[0..63] with three-input max, four independent chains.
+__device__ __forceinline__ float max64(const float *v) {
+    float a = fmaxf(v[0], v[1]), b = fmaxf(v[2], v[3]), c = fmaxf(v[4], v[5]), d = fmaxf(v[6], v[7]);
+#pragma unroll
+    for (int j = 8; j < kHalf; j += 8) {
+        a = fmax3(a, v[j + 0], v[j + 1]);
+        b = fmax3(b, v[j + 2], v[j + 3]);
+        c = fmax3(c, v[j + 4], v[j + 5]);
+        d = fmax3(d, v[j + 6], v[j + 7]);
+    }
+    return fmaxf(fmaxf(a, b), fmaxf(c, d));
+}
+
+// 2^xa + 2^xb for xa, xb <= 0 with one SFU instruction: both arguments are
+// rounded to f16, exponentiated as a packed f16 pair (relative error about
+// 2^-10 per term), and the pair is added back into the fp32 sums.
+__device__ __forceinline__ void ex2_f16x2_acc(float xa, float xb, float &acc0, float &acc1) {
+    asm("{\n\t.reg .b32 h, e;\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.f16x2.f32 h, %3, %2;\n\t"
+        "ex2.approx.f16x2 e, h;\n\t"
+        "mov.b32 {lo, hi}, e;\n\t"
+        "add.rn.f32.f16 %0, lo, %0;\n\t"
+        "add.rn.f32.f16 %1, hi, %1;\n\t}"
+        : "+f"(acc0), "+f"(acc1)
+        : "f"(xa), "f"(xb));
+}
+
+// Same for two pairs, the two f16 pairs first added in f16 (one more 2^-11
+// rounding) so only one pair of fp32 additions is needed per four terms.
+__device__ __forceinline__ void ex2_f16x2_acc4(float2 xa, float2 xb, float &acc0, float &acc1) {
+    asm("{\n\t.reg .b32 ha, hb, ea, eb, s;\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.f16x2.f32 ha, %3, %2;\n\t"
+        "cvt.rn.f16x2.f32 hb, %5, %4;\n\t"
+        "ex2.approx.f16x2 ea, ha;\n\t"
+        "ex2.approx.f16x2 eb, hb;\n\t"
+        "add.rn.f16x2 s, ea, eb;\n\t"
+        "mov.b32 {lo, hi}, s;\n\t"
+        "add.rn.f32.f16 %0, lo, %0;\n\t"
+        "add.rn.f32.f16 %1, hi, %1;\n\t}"
+        : "+f"(acc0), "+f"(acc1)
+        : "f"(xa.x), "f"(xa.y), "f"(xb.x), "f"(xb.y));
+}
+
 template <int HEAD_DIM>
 __global__ void __launch_bounds__(kAttnThreads, 2)
 attn_stats_kernel(const __grid_constant__ AttnParams p) {
@@ -82,35 +196,19 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
     uint64_t *full = bars;                 // [kStages] key tile landed
     uint64_t *empty = bars + kStages;      // [kStages] key tile consumed by the MMAs
     uint64_t *q_full = bars + 2 * kStages; // Q tile landed
-    uint64_t *s_full = q_full + 1;         // [2] S buffer written by the MMAs
-    uint64_t *s_empty = s_full + 2;        // [2] S buffer read out by the softmax warps
-    uint64_t *red_bar = s_empty + 2;       // column partial sums of the 4 softmax warps ready
+    uint64_t *q_empty = q_full + 1;        // Q tile released by the item's last MMAs
+    uint64_t *s_full = q_empty + 1;        // [2] S buffer written by the MMAs
+    uint64_t *s_empty = s_full + 2;        // [2] S buffer read out by the 8 softmax warps
+    uint64_t *stat_bar = s_empty + 2;      // both halves' (m, l) of the item are in smem
+    uint64_t *red_bar = stat_bar + 1;      // column partial sums of the item are in smem
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(red_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    float *red = reinterpret_cast<float *>(smem + S::kRedOff);  // [4][128]
+    float *red = reinterpret_cast<float *>(smem + S::kRedOff);     // [4 quadrants][128 columns]
+    float2 *stat = reinterpret_cast<float2 *>(smem + S::kStatOff); // [2 halves][128 rows]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    // ---- work item
-    const int per_req = p.n_layers * p.Hkv * p.MT;
-    const int rank = blockIdx.x / per_req;
-    int rem = blockIdx.x - rank * per_req;
-    const int layer = rem / (p.Hkv * p.MT);
-    rem -= layer * p.Hkv * p.MT;
-    const int kvh = rem / p.MT;
-    const int mt = rem - kvh * p.MT;
-    const int r = p.order ? p.order[rank] : rank;
-
-    int pstart = p.cu_prefix[r];
-    int L = p.cu_prefix[r + 1] - pstart;
-    if (pstart < 0 || L < 0 || static_cast<long long>(pstart) + L > p.total_prefix) {
-        if (threadIdx.x == 0) atomicOr(p.status, FOCUS_DEV_BAD_INPUT);
-        L = 0;
-        pstart = 0;
-    }
-    const int n_pre = (L + kTileKeys - 1) / kTileKeys;
-    const int n_tiles = n_pre + 1;  // + the block tile, always last
+    const int n_items = p.R * p.n_layers * p.Hkv * p.MT;
 
     // ---- setup
     if (threadIdx.x == 0) {
@@ -119,18 +217,22 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
             mbar_init(&empty[s], 1);
         }
         mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&s_empty[b], 4);
+            mbar_init(&s_empty[b], kSoftmaxWarps);
         }
-        mbar_init(red_bar, 4);
+        mbar_init(stat_bar, kSoftmaxWarps);
+        mbar_init(red_bar, kSoftmaxWarps);
         *abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&p.tm_q[layer]);
-        tma_prefetch_desc(&p.tm_kp[layer]);
-        tma_prefetch_desc(&p.tm_kb[layer]);
+        for (int l = 0; l < p.n_layers; ++l) {
+            tma_prefetch_desc(&p.tm_q[l]);
+            tma_prefetch_desc(&p.tm_kp[l]);
+            tma_prefetch_desc(&p.tm_kb[l]);
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -147,36 +249,48 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
             // Key tiles of a single row tile are read once: stream them past L2.  With
             // several row tiles per kv head the siblings re-read them from L2.
             const uint64_t pol = p.MT == 1 ? l2_policy_evict_first() : l2_policy_evict_normal();
-            mbar_arrive_expect_tx(q_full, S::kTileBytes);
+            uint32_t kt = 0;   // key tiles issued by this CTA
+            int last_q = -1;   // item count of the last Q load issued
+            int k = 0;
+            for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++k) {
+                const Item w = decode_item(p, it);
+                if (w.bad) atomicOr(p.status, FOCUS_DEV_BAD_INPUT);
+                if (!mbar_wait(q_empty, (k & 1) ^ 1, p.status, abort_flag)) break;
+                mbar_arrive_expect_tx(q_full, S::kTileBytes);
 #pragma unroll
-            for (int c = 0; c < S::kChunks; ++c)
-                tma_load_3d(sQ + c * kChunkBytes, &p.tm_q[layer], q_full, c * 64, kvh * p.G,
-                            r * p.B + mt * p.tok_per_tile, pol);
-            int last = -1;
-            for (int t = 0; t < n_tiles; ++t) {
-                const int s = t % kStages;
-                const uint32_t ph = (t / kStages) & 1;
-                if (!mbar_wait(&empty[s], ph ^ 1, p.status, abort_flag)) break;
-                uint8_t *dst = sK + s * S::kTileBytes;
-                if (t < n_pre) {
-                    mbar_arrive_expect_tx(&full[s], S::kTileBytes);
+                for (int c = 0; c < S::kChunks; ++c)
+                    tma_load_3d(sQ + c * kChunkBytes, &p.tm_q[w.layer], q_full, c * 64, w.kvh * p.G,
+                                w.r * p.B + w.mt * p.tok_per_tile, pol);
+                last_q = k;
+                bool ok = true;
+                for (int t = 0; t <= w.n_pre; ++t, ++kt) {
+                    const int s = kt % kStages;
+                    const uint32_t ph = (kt / kStages) & 1;
+                    if (!mbar_wait(&empty[s], ph ^ 1, p.status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *dst = sK + s * S::kTileBytes;
+                    if (t < w.n_pre) {
+                        mbar_arrive_expect_tx(&full[s], S::kTileBytes);
 #pragma unroll
-                    for (int c = 0; c < S::kChunks; ++c)
-                        tma_load_3d(dst + c * kChunkBytes, &p.tm_kp[layer], &full[s], c * 64, kvh,
-                                    pstart + t * kTileKeys, pol);
-                } else {
-                    mbar_arrive_expect_tx(&full[s], p.n_blk * 128 * S::kChunks);
+                        for (int c = 0; c < S::kChunks; ++c)
+                            tma_load_3d(dst + c * kChunkBytes, &p.tm_kp[w.layer], &full[s], c * 64,
+                                        w.kvh, w.pstart + t * kTileKeys, pol);
+                    } else {
+                        mbar_arrive_expect_tx(&full[s], p.n_blk * 128 * S::kChunks);
 #pragma unroll
-                    for (int c = 0; c < S::kChunks; ++c)
-                        tma_load_3d(dst + c * kChunkBytes, &p.tm_kb[layer], &full[s], c * 64, kvh,
-                                    r * p.B, pol);
+                        for (int c = 0; c < S::kChunks; ++c)
+                            tma_load_3d(dst + c * kChunkBytes, &p.tm_kb[w.layer], &full[s], c * 64,
+                                        w.kvh, w.r * p.B, pol);
+                    }
                 }
-                last = t;
+                if (!ok) break;
             }
             // Drain: every copy this thread issued has landed before the CTA exits.
-            mbar_wait_drain(q_full, 0);
-            for (int t = last - kStages + 1; t <= last; ++t)
-                if (t >= 0) mbar_wait_drain(&full[t % kStages], (t / kStages) & 1);
+            if (last_q >= 0) mbar_wait_drain(q_full, last_q & 1);
+            for (uint32_t u = kt > kStages ? kt - kStages : 0; u < kt; ++u)
+                mbar_wait_drain(&full[u % kStages], (u / kStages) & 1);
         }
     } else if (warp == 1) {
         // ======================= MMA issuer
@@ -184,17 +298,25 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
             const uint32_t idesc_pre = umma_idesc_bf16_f32(kTileRows, kTileKeys);
             const uint32_t idesc_blk = umma_idesc_bf16_f32(kTileRows, p.n_blk);
             const uint32_t a_base = smem_u32(sQ);
-            int last = -1;
-            if (mbar_wait(q_full, 0, p.status, abort_flag)) {
-                for (int t = 0; t < n_tiles; ++t) {
-                    const int s = t % kStages;
-                    const uint32_t ph = (t / kStages) & 1;
-                    const int buf = t & 1;
-                    const uint32_t bph = (t >> 1) & 1;
-                    if (!mbar_wait(&s_empty[buf], bph ^ 1, p.status, abort_flag)) break;
-                    if (!mbar_wait(&full[s], ph, p.status, abort_flag)) break;
+            uint32_t kt = 0;  // key tiles consumed
+            uint32_t st = 0;  // S tiles produced
+            int k = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++k) {
+                const Item w = decode_item(p, it);
+                if (!mbar_wait(q_full, k & 1, p.status, abort_flag)) break;
+                for (int t = 0; t <= w.n_pre; ++t, ++kt, ++st) {
+                    const int s = kt % kStages;
+                    const uint32_t ph = (kt / kStages) & 1;
+                    const int buf = st & 1;
+                    const uint32_t bph = (st >> 1) & 1;
+                    if (!mbar_wait(&s_empty[buf], bph ^ 1, p.status, abort_flag) ||
+                        !mbar_wait(&full[s], ph, p.status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
-                    const uint32_t idesc = (t < n_pre) ? idesc_pre : idesc_blk;
+                    const uint32_t idesc = (t < w.n_pre) ? idesc_pre : idesc_blk;
                     const uint32_t d_tmem = tmem_base + buf * kTileKeys;
                     const uint32_t b_base = smem_u32(sK + s * S::kTileBytes);
 #pragma unroll
@@ -205,114 +327,159 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
                     }
                     umma_commit(&empty[s]);
                     umma_commit(&s_full[buf]);
-                    last = t;
                 }
+                if (ok) umma_commit(q_empty);  // Q may be overwritten once these MMAs finish
             }
             // Drain: the last MMAs have finished writing TMEM.
-            if (last >= 0) mbar_wait_drain(&s_full[last & 1], (last >> 1) & 1);
+            if (st > 0) mbar_wait_drain(&s_full[(st - 1) & 1], ((st - 1) >> 1) & 1);
         }
     } else {
-        // ======================= softmax statistics, one query row per thread
-        const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+        // ======================= softmax statistics: warpgroup h, one query row per thread
+        const int sw = warp - 2;         // 0..7
+        const int h = sw >> 2;           // column half of every S tile
+        const int quad = warp & 3;       // TMEM lane quadrant this warp may access
         const int row = quad * 32 + lane;
-        const int rows_valid = min(kTileRows, p.G * p.B - mt * kTileRows);
+        const int col0 = h * kHalf;
         const float c = p.scale_log2;
-        float m = -INFINITY;  // running max of the scaled logits (log2 domain)
-        float l = 0.f;        // running sum of 2^(x - m)
-        for (int t = 0; t < n_tiles; ++t) {
-            const int buf = t & 1;
-            const uint32_t bph = (t >> 1) & 1;
-            if (!mbar_wait(&s_full[buf], bph, p.status, abort_flag)) break;
-            tc_fence_after();
-            const uint32_t ta = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                                static_cast<uint32_t>(buf * kTileKeys);
-            float v[kTileKeys];
-            tmem_ld32<0>(ta, v);
-            tmem_ld32<32>(ta, v);
-            tmem_ld32<64>(ta, v);
-            tmem_ld32<96>(ta, v);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_empty[buf]);
-
-            if (t < n_pre) {
-                const int nv = min(kTileKeys, L - t * kTileKeys);
-                float mx = -INFINITY;
-                if (nv == kTileKeys) {
-#pragma unroll
-                    for (int j = 0; j < kTileKeys; ++j) mx = fmaxf(mx, v[j]);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < kTileKeys; ++j)
-                        if (j < nv) mx = fmaxf(mx, v[j]);
+        const float2 c2 = make_float2(c, c);
+        uint32_t st = 0;
+        int k = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++k) {
+            const Item w = decode_item(p, it);
+            const int rows_valid = min(kTileRows, p.G * p.B - w.mt * kTileRows);
+            float m = -INFINITY;  // running max of the scaled logits (log2 domain), this half
+            float l = 0.f;        // running sum of 2^(x - m), this half
+            for (int t = 0; t <= w.n_pre; ++t, ++st) {
+                const int buf = st & 1;
+                const uint32_t bph = (st >> 1) & 1;
+                if (!mbar_wait(&s_full[buf], bph, p.status, abort_flag)) {
+                    ok = false;
+                    break;
                 }
-                const float m_new = fmaxf(m, mx * c);
-                const float neg = -m_new;
-                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-                if (nv == kTileKeys) {
-#pragma unroll
-                    for (int j = 0; j < kTileKeys; j += 4) {
-                        a0 += ex2(fmaf(v[j + 0], c, neg));
-                        a1 += ex2(fmaf(v[j + 1], c, neg));
-                        a2 += ex2(fmaf(v[j + 2], c, neg));
-                        a3 += ex2(fmaf(v[j + 3], c, neg));
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < kTileKeys; j += 4) {
-                        a0 += (j + 0 < nv) ? ex2(fmaf(v[j + 0], c, neg)) : 0.f;
-                        a1 += (j + 1 < nv) ? ex2(fmaf(v[j + 1], c, neg)) : 0.f;
-                        a2 += (j + 2 < nv) ? ex2(fmaf(v[j + 2], c, neg)) : 0.f;
-                        a3 += (j + 3 < nv) ? ex2(fmaf(v[j + 3], c, neg)) : 0.f;
-                    }
+                tc_fence_after();
+                const int ncols = (t < w.n_pre) ? min(kTileKeys, w.L - t * kTileKeys) : p.B;
+                const int nh = min(max(ncols - col0, 0), kHalf);  // valid columns in this half
+                float v[kHalf];
+                if (nh > 0) {
+                    const uint32_t ta = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                                        static_cast<uint32_t>(buf * kTileKeys + col0);
+                    tmem_ld32<0>(ta, v);
+                    tmem_ld32<32>(ta, v);
+                    tmem_wait_ld();
                 }
-                l = l * ex2(m - m_new) + ((a0 + a1) + (a2 + a3));
-                m = m_new;
-            } else {
-                // Block tile: finish m and l, then the weights of the B block columns.
-                const int nb = p.B;
-                float mx = -INFINITY;
-#pragma unroll
-                for (int j = 0; j < kTileKeys; ++j)
-                    if (j < nb) mx = fmaxf(mx, v[j]);
-                const float m_new = fmaxf(m, mx * c);
-                const float neg = -m_new;
-                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-                for (int j = 0; j < kTileKeys; j += 4) {
-                    v[j + 0] = (j + 0 < nb) ? ex2(fmaf(v[j + 0], c, neg)) : 0.f;
-                    v[j + 1] = (j + 1 < nb) ? ex2(fmaf(v[j + 1], c, neg)) : 0.f;
-                    v[j + 2] = (j + 2 < nb) ? ex2(fmaf(v[j + 2], c, neg)) : 0.f;
-                    v[j + 3] = (j + 3 < nb) ? ex2(fmaf(v[j + 3], c, neg)) : 0.f;
-                    a0 += v[j + 0];
-                    a1 += v[j + 1];
-                    a2 += v[j + 2];
-                    a3 += v[j + 3];
-                }
-                l = l * ex2(m - m_new) + ((a0 + a1) + (a2 + a3));
-                m = m_new;
-                const bool row_ok = row < rows_valid;
-                const float inv = 1.f / l;
-#pragma unroll
-                for (int j = 0; j < kTileKeys; ++j) v[j] = row_ok ? v[j] * inv : 0.f;
-                // Column sums over this warp's 32 rows, one 32-column group at a time.
-#pragma unroll
-                for (int g = 0; g < kTileKeys / 32; ++g) {
-                    if (g * 32 < nb) {
-                        const float col = warp_colsum32(v + g * 32, lane);
-                        red[quad * 128 + g * 32 + lane] = col;
-                    }
-                }
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(red_bar);
-                if (mbar_wait(red_bar, 0, p.status, abort_flag)) {
-                    const int j = (warp - 2) * 32 + lane;  // 128 threads cover up to 128 columns
-                    if (j < nb) {
+                if (lane == 0) mbar_arrive(&s_empty[buf]);
+
+                if (t < w.n_pre) {
+                    if (nh == kHalf) {
+                        const float m_new = fmaxf(m, max64(v) * c);
+                        const float2 nm = make_float2(-m_new, -m_new);
+                        float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
+#if FOCUS_EXP_MODE == 2
+#pragma unroll
+                        for (int q = 0; q < kHalf / 2; q += 2) {
+                            const float2 xa = __ffma2_rn(make_float2(v[2 * q], v[2 * q + 1]), c2, nm);
+                            const float2 xb = __ffma2_rn(make_float2(v[2 * q + 2], v[2 * q + 3]), c2, nm);
+                            if (q & 2)
+                                ex2_f16x2_acc4(xa, xb, acc1.x, acc1.y);
+                            else
+                                ex2_f16x2_acc4(xa, xb, acc0.x, acc0.y);
+                        }
+#else
+#pragma unroll
+                        for (int q = 0; q < kHalf / 2; ++q) {
+                            const float2 x = __ffma2_rn(make_float2(v[2 * q], v[2 * q + 1]), c2, nm);
+#if FOCUS_EXP_MODE == 1
+                            if (q & 1)
+                                ex2_f16x2_acc(x.x, x.y, acc1.x, acc1.y);
+                            else
+                                ex2_f16x2_acc(x.x, x.y, acc0.x, acc0.y);
+#else
+                            float2 e;
+                            if (FOCUS_POLY_EVERY > 0 && (q % (FOCUS_POLY_EVERY > 0 ? FOCUS_POLY_EVERY : 1)) ==
+                                                            FOCUS_POLY_EVERY - 1) {
+                                e = ex2_poly2(x);
+                            } else {
+                                e.x = ex2(x.x);
+                                e.y = ex2(x.y);
+                            }
+                            if (q & 1)
+                                acc1 = __fadd2_rn(acc1, e);
+                            else
+                                acc0 = __fadd2_rn(acc0, e);
+#endif
+                        }
+#endif
+                        l = l * ex2(m - m_new) + ((acc0.x + acc0.y) + (acc1.x + acc1.y));
+                        m = m_new;
+                    } else if (nh > 0) {
+#pragma unroll
+                        for (int j = 0; j < kHalf; ++j)
+                            if (j >= nh) v[j] = -INFINITY;
+                        const float m_new = fmaxf(m, max64(v) * c);
+                        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                        for (int j = 0; j < kHalf; j += 2) {
+                            a0 += (j < nh) ? ex2(fmaf(v[j], c, -m_new)) : 0.f;
+                            a1 += (j + 1 < nh) ? ex2(fmaf(v[j + 1], c, -m_new)) : 0.f;
+                        }
+                        l = l * ex2(m - m_new) + (a0 + a1);
+                        m = m_new;
+                    }
+                } else {
+                    // ---- block tile: finish this half, merge halves, weights, column sums
+                    if (nh > 0) {
+#pragma unroll
+                        for (int j = 0; j < kHalf; ++j)
+                            if (j >= nh) v[j] = -INFINITY;
+                        const float m_new = fmaxf(m, max64(v) * c);
+                        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                        for (int j = 0; j < kHalf; j += 2) {
+                            v[j] = (j < nh) ? ex2(fmaf(v[j], c, -m_new)) : 0.f;
+                            v[j + 1] = (j + 1 < nh) ? ex2(fmaf(v[j + 1], c, -m_new)) : 0.f;
+                            a0 += v[j];
+                            a1 += v[j + 1];
+                        }
+                        l = l * ex2(m - m_new) + (a0 + a1);
+                        m = m_new;
+                    }
+                    stat[h * 128 + row] = make_float2(m, l);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(stat_bar);
+                    if (!mbar_wait(stat_bar, k & 1, p.status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const float2 s0 = stat[row], s1 = stat[128 + row];
+                    const float M = fmaxf(s0.x, s1.x);  // finite: half 0 always has a column
+                    const float Ltot = s0.y * ex2(s0.x - M) + s1.y * ex2(s1.x - M);
+                    if (nh > 0) {
+                        const float scale = (row < rows_valid) ? ex2(m - M) / Ltot : 0.f;
+#pragma unroll
+                        for (int j = 0; j < kHalf; ++j) v[j] *= scale;
+#pragma unroll
+                        for (int g = 0; g < kHalf / 32; ++g) {
+                            if (g * 32 < nh) {
+                                const float col = warp_colsum32(v + g * 32, lane);
+                                red[quad * 128 + col0 + g * 32 + lane] = col;
+                            }
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(red_bar);
+                    if (!mbar_wait(red_bar, k & 1, p.status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const int j = sw * 32 + lane;
+                    if (j < p.B) {
                         const float sum = ((red[0 * 128 + j] + red[1 * 128 + j]) + red[2 * 128 + j]) +
                                           red[3 * 128 + j];
                         const size_t idx =
-                            ((((size_t)layer * p.R + r) * p.Hkv + kvh) * p.MT + mt) * p.B + j;
+                            ((((size_t)w.layer * p.R + w.r) * p.Hkv + w.kvh) * p.MT + w.mt) * p.B + j;
                         p.partial[idx] = sum;
                     }
                 }
@@ -329,6 +496,14 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
     }
 }
 
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return 148;
+    return n;
+}
+
 }  // namespace
 
 size_t attn_smem_bytes(int head_dim) {
@@ -336,8 +511,9 @@ size_t attn_smem_bytes(int head_dim) {
 }
 
 cudaError_t launch_attn_stats(const AttnParams &p, int head_dim, cudaStream_t stream) {
-    const long long grid = static_cast<long long>(p.R) * p.n_layers * p.Hkv * p.MT;
-    if (grid <= 0) return cudaSuccess;
+    const long long items = static_cast<long long>(p.R) * p.n_layers * p.Hkv * p.MT;
+    if (items <= 0) return cudaSuccess;
+    const long long grid = items < 2ll * sm_count() ? items : 2ll * sm_count();
     if (head_dim == 64) {
         const int smem = AttnSmem<64>::kAlloc;
         cudaError_t e = cudaFuncSetAttribute(attn_stats_kernel<64>,

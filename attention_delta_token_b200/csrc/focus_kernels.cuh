@@ -8,14 +8,16 @@
 namespace focus {
 
 // ---------------------------------------------------------------- attention statistics
-// One CTA = one (layer, request, kv head, 128-row query tile).  Its 128 query
-// rows are the G = Hq/Hkv query heads of that kv head for 128/G consecutive
-// block tokens (row = token * G + head-in-group), so every key tile that TMA
-// brings in is used by all query heads that read it.
+// Work item = one (layer, request, kv head, 128-row query tile); persistent CTAs
+// walk the items.  An item's 128 query rows are the G = Hq/Hkv query heads of
+// that kv head for 128/G consecutive block tokens (row = token * G + head-in-
+// group), so every key tile that TMA brings in is used by all query heads that
+// read it.
 constexpr int kTileRows = 128;   // UMMA M: query rows per CTA
 constexpr int kTileKeys = 128;   // UMMA N: keys per prefix tile
 constexpr int kStages = 2;       // key-tile ring depth (two CTAs share an SM)
-constexpr int kAttnThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 softmax
+constexpr int kAttnThreads = 320;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-9 softmax
+constexpr int kSoftmaxWarps = 8;   // two warpgroups, one per half of the S tile columns
 constexpr int kTmemCols = 256;   // two 128-column fp32 S buffers
 
 struct AttnParams {

@@ -184,6 +184,9 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     cfg = synth.CONFIGS[args.config]
+    if args.requests:
+        cfg = synth.FocusConfig(**{**cfg.__dict__, "R": args.requests,
+                                   "name": f"{cfg.name}_r{args.requests}"})
     seed = args.config + 1000 * rank
     p = synth.make_problem(cfg, seed=seed, device=dev)
     counts = algorithmic_counts(p)
@@ -399,6 +402,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=synth.METRIC_CONFIG)
+    ap.add_argument("--requests", type=int, default=0,
+                    help="override the workload's request count (same shape; for profiling)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
