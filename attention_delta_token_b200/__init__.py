@@ -23,7 +23,7 @@ __all__ = [
     "focus_clear_device_status", "focus_read_device_status", "focus_attn_stats",
     "focus_importance_delta", "focus_topk_select", "focus_compact", "focus_evict",
     "focus_status_string", "focus_abi_version", "focus_set_trace_events", "plan_capacity",
-    "LIB_PATH", "STATUS",
+    "focus_evict_static_scratch", "STATIC_SCRATCH_BYTES", "LIB_PATH", "STATUS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfocus.so")
@@ -67,6 +67,8 @@ def _load() -> ctypes.CDLL:
         "focus_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "focus_abi_version": (ctypes.c_int, []),
         "focus_set_trace_events": (None, [P, P]),
+        "focus_evict_static_scratch": (ctypes.c_int, [D, P, P, P, P, P, P, P, i64, P, P, P, P, P,
+                                                      P, i64, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -211,6 +213,33 @@ def focus_evict(dims, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block, cu_prefi
         _ptr(packed, bf, "packed"), int(packed.shape[0]),
         _ptr(delta_out, f32, "delta_out"), _ptr(i0_out, f32, "i0_out"),
         _ptr(i1_out, f32, "i1_out"), ws.ptr, ws.nbytes, _stream(stream)), "focus_evict")
+
+
+STATIC_SCRATCH_BYTES = 8 << 20
+
+
+def focus_evict_static_scratch(dims, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block, cu_prefix,
+                               hidden, decoded, budget, kept_idx, cu_seqlens, packed,
+                               device_status=None, delta_out=None, i0_out=None, i1_out=None,
+                               stream=None):
+    """focus_evict without a workspace argument, for callers that cannot allocate:
+    the scratch is the library's own fixed device array (STATIC_SCRATCH_BYTES).
+    `device_status` (optional int32 CUDA tensor of one element) receives the raw
+    device status bits (0 = fine)."""
+    bf, f32 = torch.bfloat16, torch.float32
+    if k0_prefix.shape[0] != k1_prefix.shape[0]:
+        raise ValueError("k0_prefix and k1_prefix must have the same number of rows")
+    _ok(_lib.focus_evict_static_scratch(
+        ctypes.byref(dims), _ptr(q0, bf, "q0"), _ptr(k0_prefix, bf, "k0_prefix"),
+        _ptr(k0_block, bf, "k0_block"), _ptr(q1, bf, "q1"), _ptr(k1_prefix, bf, "k1_prefix"),
+        _ptr(k1_block, bf, "k1_block"), _ptr(cu_prefix, torch.int32, "cu_prefix"),
+        int(k0_prefix.shape[0]), _ptr(hidden, bf, "hidden"),
+        _ptr(decoded, torch.uint8, "decoded"), _ptr(budget, torch.int32, "budget"),
+        _ptr(kept_idx, torch.int32, "kept_idx"), _ptr(cu_seqlens, torch.int32, "cu_seqlens"),
+        _ptr(packed, bf, "packed"), int(packed.shape[0]),
+        _ptr(delta_out, f32, "delta_out"), _ptr(i0_out, f32, "i0_out"),
+        _ptr(i1_out, f32, "i1_out"), _ptr(device_status, torch.int32, "device_status"),
+        _stream(stream)), "focus_evict_static_scratch")
 
 
 def plan_capacity(decoded, budget) -> int:

@@ -183,6 +183,44 @@ FOCUS_API focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, c
  */
 FOCUS_API void focus_set_trace_events(void *start_event, void *stop_event);
 
+/*
+ * The fused step for callers that cannot allocate device memory.  (The FOCUS
+ * pages have no counterpart: this is a deployment variant of focus_evict.)
+ *
+ * focus_evict needs a caller-allocated workspace.  A caller that cannot make
+ * allocations -- e.g. a serving engine that has reserved nearly all HBM for its
+ * KV cache and must not request more while it decodes, or a plug-in that only
+ * sees this C ABI and has no access to its host framework's memory pool -- can
+ * call this instead: the scratch lives in a device array of
+ * FOCUS_STATIC_SCRATCH_BYTES (8 MiB) that the library owns, and that every GPU
+ * which loads the library keeps until the process exits.  The call allocates
+ * nothing (no cudaMalloc/cudaFree, no allocating library routine); the caller
+ * still passes every input and output, as for focus_evict.
+ *
+ *  - Arguments and results are those of focus_evict, minus the workspace.
+ *  - device_status (nullable, device pointer, 4-byte aligned) receives the
+ *    call's raw device status bits: 1 = rows beyond `capacity`, 2 = malformed
+ *    cu_prefix or kept index, 4 = a kernel wait gave up; 0 = fine.  It is written
+ *    on `stream` after the kernels.
+ *  - Returns FOCUS_ERR_WORKSPACE when focus_workspace_size(dims) exceeds
+ *    FOCUS_STATIC_SCRATCH_BYTES (shapes that large need focus_evict), otherwise
+ *    the same codes as focus_evict.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current; `stream` must belong to
+ *    the current device).  Make that first call before any stream capture.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents: each call clears the status word and rewrites the rest before
+ *    reading it.  Calls whose kernels overlap on the GPU (different streams, or
+ *    threads without ordering) race on the array; serialise them.
+ */
+#define FOCUS_STATIC_SCRATCH_BYTES (8u << 20)
+FOCUS_API focus_status_t focus_evict_static_scratch(
+    const focus_dims_t *dims, const void *q0, const void *k0_prefix, const void *k0_block,
+    const void *q1, const void *k1_prefix, const void *k1_block, const int32_t *cu_prefix,
+    int64_t total_prefix, const void *hidden, const uint8_t *decoded, const int32_t *budget,
+    int32_t *kept_idx, int32_t *cu_seqlens, void *packed, int64_t capacity, float *delta_out,
+    float *i0_out, float *i1_out, uint32_t *device_status, void *stream);
+
 /* Human-readable name of a status code (static string). */
 FOCUS_API const char *focus_status_string(focus_status_t status);
 
