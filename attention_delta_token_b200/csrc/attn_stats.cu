@@ -25,10 +25,10 @@
 //               over the 128 rows (warp butterfly, then the four lane quadrants in
 //               fixed order) go to `partial`.  No float atomics: the result is
 //               deterministic and equal keys give bit-equal columns.
-// A fraction of each full tile's exponentials runs on the FMA pipe (2^x by
-// Cody-Waite style range reduction to [-1/2, 1/2] and a degree-3 minimax
-// polynomial fitted for this file, max relative error 7.5e-5), the rest on the
-// SFU, so neither pipe is the bottleneck.
+// Exponentials run on the SFU (ex2.approx, fp32); the FMA-pipe polynomial exp2,
+// packed-f16 SFU exps and a lazily updated reference max were measured and lost:
+// at the metric shape the kernel runs at the board power cap, so extra
+// instructions cost clock rather than buying throughput.
 #include <math.h>
 
 #include "focus_device.cuh"
@@ -40,14 +40,6 @@ namespace {
 
 constexpr uint32_t kChunkBytes = kTileRows * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr int kHalf = kTileKeys / 2;               // S columns per softmax warpgroup
-
-#ifndef FOCUS_EXP_MODE
-#define FOCUS_EXP_MODE 0  // full prefix tiles: 0 fp32 SFU exp2, 1 packed f16 pairs, 2 f16 quads
-#endif
-
-#ifndef FOCUS_POLY_EVERY
-#define FOCUS_POLY_EVERY 0  // > 0: every n-th column pair of a full tile uses the FMA-pipe exp2
-#endif
 
 template <int HEAD_DIM>
 struct AttnSmem {
@@ -86,29 +78,6 @@ __device__ __forceinline__ Item decode_item(const AttnParams &p, int it) {
     }
     w.n_pre = (w.L + kTileKeys - 1) / kTileKeys;
     return w;
-}
-
-// 2^x for x <= 0 on the FMA/ALU pipes.  x = n + f with n = round(x) (the 1.5*2^23
-// shifter leaves n in the low mantissa bits of t), f in [-1/2, 1/2];
-// 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 (relative-error minimax fit on [-1/2, 1/2]);
-// 2^n is applied by adding n to the exponent field.  x is clamped at -125 so the
-// result stays a normal float (2^-125 is negligible against a sum >= 1).
-__device__ __forceinline__ float2 ex2_poly2(float2 x) {
-    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-    constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f;
-    constexpr float c2 = 0.2426111400127411f, c3 = 0.0551716573536396f;
-    x.x = fmaxf(x.x, -125.f);
-    x.y = fmaxf(x.y, -125.f);
-    const float2 t = __fadd2_rn(x, make_float2(kShift, kShift));
-    const float2 n = __fadd2_rn(t, make_float2(-kShift, -kShift));
-    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-    float2 q = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
-    q = __ffma2_rn(q, f, make_float2(c1, c1));
-    q = __ffma2_rn(q, f, make_float2(c0, c0));
-    float2 y;
-    y.x = __int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23));
-    y.y = __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23));
-    return y;
 }
 
 // Loads 32 TMEM columns of this thread's lane into v[OFF .. OFF+31].
@@ -151,36 +120,6 @@ __device__ __forceinline__ float max64(const float *v) {
         d = fmax3(d, v[j + 6], v[j + 7]);
     }
     return fmaxf(fmaxf(a, b), fmaxf(c, d));
-}
-
-// 2^xa + 2^xb for xa, xb <= 0 with one SFU instruction: both arguments are
-// rounded to f16, exponentiated as a packed f16 pair (relative error about
-// 2^-10 per term), and the pair is added back into the fp32 sums.
-__device__ __forceinline__ void ex2_f16x2_acc(float xa, float xb, float &acc0, float &acc1) {
-    asm("{\n\t.reg .b32 h, e;\n\t.reg .b16 lo, hi;\n\t"
-        "cvt.rn.f16x2.f32 h, %3, %2;\n\t"
-        "ex2.approx.f16x2 e, h;\n\t"
-        "mov.b32 {lo, hi}, e;\n\t"
-        "add.rn.f32.f16 %0, lo, %0;\n\t"
-        "add.rn.f32.f16 %1, hi, %1;\n\t}"
-        : "+f"(acc0), "+f"(acc1)
-        : "f"(xa), "f"(xb));
-}
-
-// Same for two pairs, the two f16 pairs first added in f16 (one more 2^-11
-// rounding) so only one pair of fp32 additions is needed per four terms.
-__device__ __forceinline__ void ex2_f16x2_acc4(float2 xa, float2 xb, float &acc0, float &acc1) {
-    asm("{\n\t.reg .b32 ha, hb, ea, eb, s;\n\t.reg .b16 lo, hi;\n\t"
-        "cvt.rn.f16x2.f32 ha, %3, %2;\n\t"
-        "cvt.rn.f16x2.f32 hb, %5, %4;\n\t"
-        "ex2.approx.f16x2 ea, ha;\n\t"
-        "ex2.approx.f16x2 eb, hb;\n\t"
-        "add.rn.f16x2 s, ea, eb;\n\t"
-        "mov.b32 {lo, hi}, s;\n\t"
-        "add.rn.f32.f16 %0, lo, %0;\n\t"
-        "add.rn.f32.f16 %1, hi, %1;\n\t}"
-        : "+f"(acc0), "+f"(acc1)
-        : "f"(xa.x), "f"(xa.y), "f"(xb.x), "f"(xb.y));
 }
 
 template <int HEAD_DIM>
@@ -377,41 +316,17 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
                         const float m_new = fmaxf(m, max64(v) * c);
                         const float2 nm = make_float2(-m_new, -m_new);
                         float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
-#if FOCUS_EXP_MODE == 2
-#pragma unroll
-                        for (int q = 0; q < kHalf / 2; q += 2) {
-                            const float2 xa = __ffma2_rn(make_float2(v[2 * q], v[2 * q + 1]), c2, nm);
-                            const float2 xb = __ffma2_rn(make_float2(v[2 * q + 2], v[2 * q + 3]), c2, nm);
-                            if (q & 2)
-                                ex2_f16x2_acc4(xa, xb, acc1.x, acc1.y);
-                            else
-                                ex2_f16x2_acc4(xa, xb, acc0.x, acc0.y);
-                        }
-#else
 #pragma unroll
                         for (int q = 0; q < kHalf / 2; ++q) {
                             const float2 x = __ffma2_rn(make_float2(v[2 * q], v[2 * q + 1]), c2, nm);
-#if FOCUS_EXP_MODE == 1
-                            if (q & 1)
-                                ex2_f16x2_acc(x.x, x.y, acc1.x, acc1.y);
-                            else
-                                ex2_f16x2_acc(x.x, x.y, acc0.x, acc0.y);
-#else
                             float2 e;
-                            if (FOCUS_POLY_EVERY > 0 && (q % (FOCUS_POLY_EVERY > 0 ? FOCUS_POLY_EVERY : 1)) ==
-                                                            FOCUS_POLY_EVERY - 1) {
-                                e = ex2_poly2(x);
-                            } else {
-                                e.x = ex2(x.x);
-                                e.y = ex2(x.y);
-                            }
+                            e.x = ex2(x.x);
+                            e.y = ex2(x.y);
                             if (q & 1)
                                 acc1 = __fadd2_rn(acc1, e);
                             else
                                 acc0 = __fadd2_rn(acc0, e);
-#endif
                         }
-#endif
                         l = l * ex2(m - m_new) + ((acc0.x + acc0.y) + (acc1.x + acc1.y));
                         m = m_new;
                     } else if (nh > 0) {

@@ -20,16 +20,31 @@ namespace focus {
 namespace {
 
 constexpr int kPlanThreads = 1024;
-constexpr int kMaxSortR = 4096;  // requests ordered on the device; larger batches keep input order
+constexpr int kRankSortR = 1024; // up to here the order is a rank count
+constexpr int kMaxSortR = 4096;  // up to here a bitonic sort; larger batches keep input order
+
+// masked_r = number of zero bytes in decoded[r*B .. r*B+B); 16-byte loads when
+// the row is 16-byte aligned.
+__device__ __forceinline__ int masked_count(const uint8_t *decoded, int r, int B) {
+    const uint8_t *d = decoded + static_cast<size_t>(r) * B;
+    int masked = 0;
+    if ((reinterpret_cast<uintptr_t>(d) & 15u) == 0 && (B & 15) == 0) {
+        const uint4 *d4 = reinterpret_cast<const uint4 *>(d);
+        for (int i = 0; i < B / 16; ++i) {
+            const uint4 w = __ldg(d4 + i);
+            masked += __popc(__vcmpeq4(w.x, 0u)) + __popc(__vcmpeq4(w.y, 0u)) +
+                      __popc(__vcmpeq4(w.z, 0u)) + __popc(__vcmpeq4(w.w, 0u));
+        }
+        return masked >> 3;  // __vcmpeq4 sets 8 bits per equal byte
+    }
+    for (int j = 0; j < B; ++j) masked += d[j] == 0;
+    return masked;
+}
 
 // k_r = min(max(budget_r, 0), masked_r)
 __device__ __forceinline__ int kept_count(const uint8_t *decoded, const int32_t *budget, int r,
                                           int B) {
-    int masked = 0;
-    const uint8_t *d = decoded + static_cast<size_t>(r) * B;
-    for (int j = 0; j < B; ++j) masked += d[j] == 0;
-    const int K = budget[r];
-    return min(max(K, 0), masked);
+    return min(max(budget[r], 0), masked_count(decoded, r, B));
 }
 
 // Exclusive block-wide scan of one int per thread (kPlanThreads threads).
@@ -61,16 +76,30 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int *warp_tot, int &t
     return ex;
 }
 
-// One CTA: (a) the processing order of the requests, longest prefix first (a
-// bitonic sort of (L desc, r asc) keys), so the attention CTAs of the longest
-// requests start in the first wave; (b) k_r and cu_seqlens (depend only on
-// decoded and budget) and the capacity check.
+// One CTA: (a) the processing order of the requests, longest prefix first
+// (ranks of (L desc, r asc) keys), so the attention CTAs of the longest requests
+// start in the first wave; (b) k_r and cu_seqlens (depend only on decoded and
+// budget) and the capacity check.
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) {
     __shared__ unsigned long long keys[kMaxSortR];
     __shared__ int warp_tot[33];
     const int R = p.R;
 
-    if (p.order) {
+    if (p.order && R <= kRankSortR) {
+        // Rank of each request under (L desc, r asc): a plain count, no sort passes.
+        for (int i = threadIdx.x; i < R; i += blockDim.x) {
+            const int L = max(p.cu_prefix[i + 1] - p.cu_prefix[i], 0);
+            keys[i] = (static_cast<unsigned long long>(0x7fffffffu - static_cast<uint32_t>(L)) << 32) |
+                      static_cast<uint32_t>(i);
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < R; i += blockDim.x) {
+            const unsigned long long ki = keys[i];
+            int rank = 0;
+            for (int j = 0; j < R; ++j) rank += keys[j] < ki;
+            p.order[rank] = i;
+        }
+    } else if (p.order) {
         if (R <= kMaxSortR) {
             int n = 1;
             while (n < R) n <<= 1;

@@ -178,6 +178,26 @@ def make_outputs(p, cap, dev):
     return kept, cu, packed
 
 
+def rank_seed(config: int, rank: int) -> int:
+    """Each rank draws its own batch of the same shape (independent requests)."""
+    return config + 1000 * rank
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """The slowest rank's time (all ranks must call this in the same order)."""
+    dist = torch.distributed
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, blocks_per_rank: int, seconds_per_step: float) -> float:
+    """Whole-job blocks/s: every rank processes `blocks_per_rank` blocks per step."""
+    return world * blocks_per_rank / seconds_per_step
+
+
 def run_ours(args, rank, world, local_rank):
     import attention_delta_token_b200 as F
     dist = torch.distributed if world > 1 else None
@@ -187,7 +207,7 @@ def run_ours(args, rank, world, local_rank):
     if args.requests:
         cfg = synth.FocusConfig(**{**cfg.__dict__, "R": args.requests,
                                    "name": f"{cfg.name}_r{args.requests}"})
-    seed = args.config + 1000 * rank
+    seed = rank_seed(args.config, rank)
     p = synth.make_problem(cfg, seed=seed, device=dev)
     counts = algorithmic_counts(p)
     dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
@@ -205,13 +225,6 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize(dev)
         if dist:
             dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if not dist:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     # ---- device-resident timing
     sampler = ClockSampler(local_rank)
@@ -238,8 +251,8 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device status {F.focus_status_string(status)}")
     elapsed = start.elapsed_time(stop) / 1e3
     attn_s = sum(a.elapsed_time(b) for a, b in zip(ev_a, ev_b)) / 1e3 / args.steps
-    elapsed_max = max_over_ranks(elapsed)
-    attn_s_max = max_over_ranks(attn_s)
+    elapsed_max = max_over_ranks(elapsed, dev)
+    attn_s_max = max_over_ranks(attn_s, dev)
     step_s = elapsed_max / args.steps
 
     # ---- end to end: pinned host inputs -> device, the C-ABI call, result -> host
@@ -271,8 +284,8 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
         t2.record(stream)
         barrier()
-        e2e_s = max_over_ranks(s2.elapsed_time(t2) / 1e3) / n_e2e
-        e2e = {"value": world * p.R / e2e_s, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+        e2e_s = max_over_ranks(s2.elapsed_time(t2) / 1e3, dev) / n_e2e
+        e2e = {"value": job_throughput(world, p.R, e2e_s), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "steps": n_e2e, "ms_per_step": e2e_s * 1e3,
                "path": "pinned host -> cudaMemcpyAsync -> focus_evict -> host"}
         if F.focus_read_device_status(ws) != 0:
@@ -290,7 +303,8 @@ def run_ours(args, rank, world, local_rank):
         clocks = sampler.summary()
         sm_hz = (clocks["sm_mhz"] or 1965.0) * 1e6
         result = {
-            "metric": METRIC, "value": world * p.R / step_s, "unit": UNIT, "n_gpus": world,
+            "metric": METRIC, "value": job_throughput(world, p.R, step_s), "unit": UNIT,
+            "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
@@ -319,7 +333,7 @@ def run_ours(args, rank, world, local_rank):
                 "peaks": f"{peak_src}: hbm {hbm} GB/s, bf16 {tc} TFLOP/s",
             },
             "clocks": clocks,
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": 3 * args.steps,  # plan, attention statistics, select + compact
             "e2e": e2e,
             "impl": "ours",
         }
