@@ -25,10 +25,12 @@
 //               over the 128 rows (warp butterfly, then the four lane quadrants in
 //               fixed order) go to `partial`.  No float atomics: the result is
 //               deterministic and equal keys give bit-equal columns.
-// Exponentials run on the SFU (ex2.approx, fp32); the FMA-pipe polynomial exp2,
-// packed-f16 SFU exps and a lazily updated reference max were measured and lost:
-// at the metric shape the kernel runs at the board power cap, so extra
-// instructions cost clock rather than buying throughput.
+// Exponentials run on the SFU (ex2.approx, fp32).  After a half-row's first full
+// tile the exps are taken against the running reference max without computing
+// each tile's max (the tile's sum reveals a rise).  At the metric shape the
+// kernel runs at the board power cap, so fewer instructions per (row, key) is
+// what buys throughput; moving exps to the FMA pipe or packing them as f16
+// pairs was measured and did not.
 #include <math.h>
 
 #include "focus_device.cuh"
@@ -181,6 +183,9 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // Everything above overlaps the planner; the request order it writes is read below.
+    pdl_launch_dependents();
+    pdl_wait();
 
     if (warp == 0) {
         // ======================= TMA producer
@@ -312,20 +317,42 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
                 if (lane == 0) mbar_arrive(&s_empty[buf]);
 
                 if (t < w.n_pre) {
-                    if (nh == kHalf) {
+                    if (nh == kHalf && m != -INFINITY) {
+                        // Against the running reference m, no tile max is needed: a tile whose
+                        // values rose far above m shows up as a large sum (>= 2^20), and only
+                        // then is the tile redone against its exact max.  Values that fell far
+                        // below m underflow to 0, as they do against the exact max.
+                        const float2 nm = make_float2(-m, -m);
+                        float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+                        for (int q = 0; q < kHalf / 2; ++q) {
+                            const float2 x = __ffma2_rn(make_float2(v[2 * q], v[2 * q + 1]), c2, nm);
+                            float2 e; e.x = ex2(x.x); e.y = ex2(x.y);
+                            if (q & 1) acc1 = __fadd2_rn(acc1, e); else acc0 = __fadd2_rn(acc0, e);
+                        }
+                        const float sum = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+                        if (sum <= 1048576.f) {
+                            l += sum;
+                        } else {
+                            const float m_new = fmaxf(m, max64(v) * c);
+                            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                            for (int j = 0; j < kHalf; j += 2) {
+                                a0 += ex2(fmaf(v[j], c, -m_new));
+                                a1 += ex2(fmaf(v[j + 1], c, -m_new));
+                            }
+                            l = l * ex2(m - m_new) + (a0 + a1);
+                            m = m_new;
+                        }
+                    } else if (nh == kHalf) {
                         const float m_new = fmaxf(m, max64(v) * c);
                         const float2 nm = make_float2(-m_new, -m_new);
                         float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
 #pragma unroll
                         for (int q = 0; q < kHalf / 2; ++q) {
                             const float2 x = __ffma2_rn(make_float2(v[2 * q], v[2 * q + 1]), c2, nm);
-                            float2 e;
-                            e.x = ex2(x.x);
-                            e.y = ex2(x.y);
-                            if (q & 1)
-                                acc1 = __fadd2_rn(acc1, e);
-                            else
-                                acc0 = __fadd2_rn(acc0, e);
+                            float2 e; e.x = ex2(x.x); e.y = ex2(x.y);
+                            if (q & 1) acc1 = __fadd2_rn(acc1, e); else acc0 = __fadd2_rn(acc0, e);
                         }
                         l = l * ex2(m - m_new) + ((acc0.x + acc0.y) + (acc1.x + acc1.y));
                         m = m_new;
@@ -425,7 +452,7 @@ size_t attn_smem_bytes(int head_dim) {
     return head_dim == 64 ? AttnSmem<64>::kAlloc : AttnSmem<128>::kAlloc;
 }
 
-cudaError_t launch_attn_stats(const AttnParams &p, int head_dim, cudaStream_t stream) {
+cudaError_t launch_attn_stats(const AttnParams &p, int head_dim, cudaStream_t stream, bool pdl) {
     const long long items = static_cast<long long>(p.R) * p.n_layers * p.Hkv * p.MT;
     if (items <= 0) return cudaSuccess;
     const long long grid = items < 2ll * sm_count() ? items : 2ll * sm_count();
@@ -434,13 +461,17 @@ cudaError_t launch_attn_stats(const AttnParams &p, int head_dim, cudaStream_t st
         cudaError_t e = cudaFuncSetAttribute(attn_stats_kernel<64>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        attn_stats_kernel<64><<<static_cast<unsigned>(grid), kAttnThreads, smem, stream>>>(p);
+        e = launch_kernel(attn_stats_kernel<64>, dim3(static_cast<unsigned>(grid)), dim3(kAttnThreads),
+                          smem, stream, pdl, p);
+        if (e != cudaSuccess) return e;
     } else {
         const int smem = AttnSmem<128>::kAlloc;
         cudaError_t e = cudaFuncSetAttribute(attn_stats_kernel<128>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        attn_stats_kernel<128><<<static_cast<unsigned>(grid), kAttnThreads, smem, stream>>>(p);
+        e = launch_kernel(attn_stats_kernel<128>, dim3(static_cast<unsigned>(grid)), dim3(kAttnThreads),
+                          smem, stream, pdl, p);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }

@@ -92,10 +92,12 @@ focus_status_t check_ws(const focus_dims_t &d, const void *ws, size_t bytes) {
 std::atomic<cudaEvent_t> g_trace_start{nullptr};
 std::atomic<cudaEvent_t> g_trace_stop{nullptr};
 
-cudaError_t launch_attn_traced(const AttnParams &p, int head_dim, cudaStream_t s) {
+cudaError_t launch_attn_traced(const AttnParams &p, int head_dim, cudaStream_t s, bool pdl = false) {
     cudaEvent_t a = g_trace_start.load(), b = g_trace_stop.load();
     if (a && b && cudaEventRecord(a, s) != cudaSuccess) return cudaErrorInvalidResourceHandle;
-    cudaError_t e = focus::launch_attn_stats(p, head_dim, s);
+    // An event between two kernels would cut the programmatic overlap, so a traced
+    // launch is an ordinary one.
+    cudaError_t e = focus::launch_attn_stats(p, head_dim, s, pdl && !(a && b));
     if (e != cudaSuccess) return e;
     if (a && b) return cudaEventRecord(b, s);
     return cudaSuccess;
@@ -392,16 +394,15 @@ focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void 
     pp.R = d.R;
     pp.B = d.B;
     FOCUS_CUDA(focus::launch_plan(pp, s));
-    FOCUS_CUDA(launch_attn_traced(p, d.head_dim, s));
+    FOCUS_CUDA(launch_attn_traced(p, d.head_dim, s, /*pdl=*/true));
 
+    // Selection per request, then the row copy spread over the whole GPU.
     focus::SelectParams sp;
     memset(&sp, 0, sizeof sp);
     sp.partial = p.partial;
     sp.decoded = decoded;
     sp.cu_seqlens = cu_seqlens;
     sp.kept_idx = kept_idx;
-    sp.hidden = static_cast<const uint16_t *>(hidden);
-    sp.packed = static_cast<uint16_t *>(packed);
     sp.delta_out = delta_out;
     sp.i0_out = i0_out;
     sp.i1_out = i1_out;
@@ -413,7 +414,11 @@ focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void 
     sp.MT = p.MT;
     sp.H = d.hidden;
     sp.pool_window = d.pool_window;
-    FOCUS_CUDA(focus::launch_select_compact(sp, s));
+    FOCUS_CUDA(focus::launch_select_compact(sp, s, /*pdl=*/true));
+    focus::CompactParams cp{static_cast<const uint16_t *>(hidden), kept_idx, cu_seqlens,
+                            static_cast<uint16_t *>(packed), p.status, capacity, d.R, d.B,
+                            d.hidden};
+    FOCUS_CUDA(focus::launch_compact(cp, s, /*pdl=*/true));
     return FOCUS_OK;
 }
 

@@ -5,7 +5,29 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace focus {
+
+// Launches `kernel` on `stream`; with `pdl` the launch carries the programmatic
+// stream serialization attribute, so it may start while the previous kernel on
+// the stream is still running (the kernel itself waits with griddepcontrol.wait
+// before touching that kernel's outputs).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t stream, bool pdl, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ---------------------------------------------------------------- attention statistics
 // Work item = one (layer, request, kv head, 128-row query tile); persistent CTAs
@@ -36,7 +58,8 @@ struct AttnParams {
 };
 
 size_t attn_smem_bytes(int head_dim);
-cudaError_t launch_attn_stats(const AttnParams &p, int head_dim, cudaStream_t stream);
+cudaError_t launch_attn_stats(const AttnParams &p, int head_dim, cudaStream_t stream,
+                              bool pdl = false);
 
 // ---------------------------------------------------------------- planning
 struct PlanParams {
@@ -65,7 +88,7 @@ struct SelectParams {
     long long capacity;
     int R, B, Hkv, MT, H, pool_window;
 };
-cudaError_t launch_select_compact(const SelectParams &p, cudaStream_t stream);
+cudaError_t launch_select_compact(const SelectParams &p, cudaStream_t stream, bool pdl = false);
 
 struct DeltaParams {
     const float *i0, *i1;
@@ -90,6 +113,6 @@ struct CompactParams {
     long long capacity;
     int R, B, H;
 };
-cudaError_t launch_compact(const CompactParams &p, cudaStream_t stream);
+cudaError_t launch_compact(const CompactParams &p, cudaStream_t stream, bool pdl = false);
 
 }  // namespace focus

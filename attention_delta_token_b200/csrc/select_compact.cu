@@ -84,6 +84,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
     __shared__ unsigned long long keys[kMaxSortR];
     __shared__ int warp_tot[33];
     const int R = p.R;
+    pdl_launch_dependents();  // the attention kernel may set up while this runs
 
     if (p.order && R <= kRankSortR) {
         // Rank of each request under (L desc, r asc): a plain count, no sort passes.
@@ -199,6 +200,8 @@ __device__ __forceinline__ float pool_mask(const float *raw, const uint8_t *dec,
 // path) or from a pooled delta (stand-alone select): I0, I1, dI, MaxPool1D,
 // mask, top-k, then the k kept hidden rows copied with 16-byte vectors.
 __global__ void __launch_bounds__(256) select_compact_kernel(const SelectParams p) {
+    pdl_launch_dependents();
+    pdl_wait();  // column sums / delta and cu_seqlens come from the previous kernels
     __shared__ float raw_s[128];
     __shared__ float val_s[128];
     __shared__ uint8_t dec_s[128];
@@ -287,6 +290,7 @@ __global__ void __launch_bounds__(128) reduce_kernel(const ReduceParams p) {
 
 // Stand-alone compaction: one warp per packed row, request found by binary search.
 __global__ void __launch_bounds__(256) compact_kernel(const CompactParams p) {
+    pdl_wait();  // kept_idx and cu_seqlens come from the previous kernels
     const int warps = blockDim.x >> 5;
     const long long total = min(static_cast<long long>(p.cu_seqlens[p.R]), p.capacity);
     if (blockIdx.x == 0 && threadIdx.x == 0 && p.cu_seqlens[p.R] > p.capacity)
@@ -305,10 +309,19 @@ __global__ void __launch_bounds__(256) compact_kernel(const CompactParams p) {
             if (lane == 0) atomicOr(p.status, FOCUS_DEV_BAD_INPUT);
             continue;
         }
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.hidden) +
-                           (static_cast<size_t>(lo) * p.B + jj) * nvec;
-        uint4 *dst = reinterpret_cast<uint4 *>(p.packed) + static_cast<size_t>(row) * nvec;
-        for (int c = lane; c < nvec; c += 32) dst[c] = __ldg(src + c);
+        const uint4 *__restrict__ src = reinterpret_cast<const uint4 *>(p.hidden) +
+                                        (static_cast<size_t>(lo) * p.B + jj) * nvec;
+        uint4 *__restrict__ dst = reinterpret_cast<uint4 *>(p.packed) + static_cast<size_t>(row) * nvec;
+        int c = lane;
+        for (; c + 96 < nvec; c += 128) {  // four 16-byte loads in flight per lane
+            const uint4 x0 = __ldg(src + c), x1 = __ldg(src + c + 32), x2 = __ldg(src + c + 64),
+                        x3 = __ldg(src + c + 96);
+            dst[c] = x0;
+            dst[c + 32] = x1;
+            dst[c + 64] = x2;
+            dst[c + 96] = x3;
+        }
+        for (; c < nvec; c += 32) dst[c] = __ldg(src + c);
     }
 }
 
@@ -319,9 +332,10 @@ cudaError_t launch_plan(const PlanParams &p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_select_compact(const SelectParams &p, cudaStream_t stream) {
-    select_compact_kernel<<<p.R, 256, 0, stream>>>(p);
-    return cudaGetLastError();
+cudaError_t launch_select_compact(const SelectParams &p, cudaStream_t stream, bool pdl) {
+    // Without a row copy only the B <= 128 column threads have work.
+    return launch_kernel(select_compact_kernel, dim3(p.R), dim3(p.hidden ? 256 : 128), 0, stream,
+                         pdl, p);
 }
 
 cudaError_t launch_delta(const DeltaParams &p, cudaStream_t stream) {
@@ -334,12 +348,12 @@ cudaError_t launch_reduce(const ReduceParams &p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_compact(const CompactParams &p, cudaStream_t stream) {
-    long long blocks = (p.capacity + 7) / 8;
+cudaError_t launch_compact(const CompactParams &p, cudaStream_t stream, bool pdl) {
+    long long blocks = (p.capacity + 7) / 8;  // one warp per packed row
     if (blocks < 1) blocks = 1;
     if (blocks > 148 * 16) blocks = 148 * 16;
-    compact_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(compact_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
+                         pdl, p);
 }
 
 }  // namespace focus
