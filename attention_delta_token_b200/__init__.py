@@ -23,7 +23,8 @@ __all__ = [
     "focus_clear_device_status", "focus_read_device_status", "focus_attn_stats",
     "focus_importance_delta", "focus_topk_select", "focus_compact", "focus_evict",
     "focus_status_string", "focus_abi_version", "focus_set_trace_events", "plan_capacity",
-    "focus_evict_static_scratch", "STATIC_SCRATCH_BYTES", "LIB_PATH", "STATUS",
+    "focus_evict_static_scratch", "STATIC_SCRATCH_BYTES", "focus_selftest_wait_timeout",
+    "LIB_PATH", "STATUS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfocus.so")
@@ -69,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "focus_set_trace_events": (None, [P, P]),
         "focus_evict_static_scratch": (ctypes.c_int, [D, P, P, P, P, P, P, P, i64, P, P, P, P, P,
                                                       P, i64, P, P, P, P, P]),
+        "focus_selftest_wait_timeout": (ctypes.c_int, [P, ctypes.c_uint64, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -240,6 +242,14 @@ def focus_evict_static_scratch(dims, q0, k0_prefix, k0_block, q1, k1_prefix, k1_
         _ptr(delta_out, f32, "delta_out"), _ptr(i0_out, f32, "i0_out"),
         _ptr(i1_out, f32, "i1_out"), _ptr(device_status, torch.int32, "device_status"),
         _stream(stream)), "focus_evict_static_scratch")
+
+
+def focus_selftest_wait_timeout(status, elapsed_ns, limit_ns: int, stream=None):
+    """Runs the bounded wait on a barrier that never completes (see include/focus.h).
+    `status`: int32 CUDA tensor [1]; `elapsed_ns`: int64 CUDA tensor [1]."""
+    _ok(_lib.focus_selftest_wait_timeout(_ptr(status, torch.int32, "status"), int(limit_ns),
+                                         _ptr(elapsed_ns, torch.int64, "elapsed_ns"),
+                                         _stream(stream)), "focus_selftest_wait_timeout")
 
 
 def plan_capacity(decoded, budget) -> int:

@@ -18,7 +18,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfocus.so")
-SOURCES = ["focus_api.cu", "attn_stats.cu", "select_compact.cu", "focus_static_scratch.cu"]
+SOURCES = ["focus_api.cu", "attn_stats.cu", "select_compact.cu", "focus_static_scratch.cu",
+           "focus_selftest.cu"]
 HEADERS = ["focus_device.cuh", "focus_kernels.cuh"]
 
 NVCC_FLAGS = [

@@ -70,14 +70,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // FOCUS_DEV_TIMEOUT in *status plus *abort_flag) when the limit passes or when
 // another role of the CTA has already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *status,
-                                          volatile int *abort_flag) {
+                                          volatile int *abort_flag,
+                                          uint64_t limit_ns = FOCUS_WAIT_LIMIT_NS) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 255u) == 0) {
             if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > FOCUS_WAIT_LIMIT_NS) {
+            if (global_timer_ns() - t0 > limit_ns) {
                 atomicOr(status, FOCUS_DEV_TIMEOUT);
                 *abort_flag = 1;
                 return false;

@@ -221,6 +221,18 @@ FOCUS_API focus_status_t focus_evict_static_scratch(
     int32_t *kept_idx, int32_t *cu_seqlens, void *packed, int64_t capacity, float *delta_out,
     float *i0_out, float *i1_out, uint32_t *device_status, void *stream);
 
+/*
+ * Self-test of the failure-detection path (no FOCUS counterpart; a test hook).
+ * Launches one warp that waits, with the same bounded mbarrier wait the eviction
+ * kernels use, on a barrier that never completes.  After `limit_ns`
+ * (1 .. 2e9 nanoseconds) the wait gives up: FOCUS_DEV_TIMEOUT (4) is OR-ed into
+ * the device word *status, and *elapsed_ns (device) receives how long it waited.
+ * Nothing faults, traps or hangs; the context stays usable.
+ */
+FOCUS_API focus_status_t focus_selftest_wait_timeout(uint32_t *status, uint64_t limit_ns,
+                                                     unsigned long long *elapsed_ns,
+                                                     void *stream);
+
 /* Human-readable name of a status code (static string). */
 FOCUS_API const char *focus_status_string(focus_status_t status);
 

@@ -215,3 +215,20 @@ def test_malformed_cu_prefix_reports():
     p.cu_prefix = bad
     out = run_evict(p)
     assert out["status"] == 6  # FOCUS_ERR_DEVICE_CHECK
+
+
+def test_bounded_wait_times_out_and_reports():
+    """A kernel waiting on a barrier that never completes gives up after its limit,
+    reports FOCUS_DEV_TIMEOUT in the status word, and leaves the context usable."""
+    import attention_delta_token_b200 as F
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    elapsed = torch.zeros(1, dtype=torch.int64, device="cuda")
+    limit = 50_000_000  # 50 ms
+    F.focus_selftest_wait_timeout(status, elapsed, limit)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 4  # FOCUS_DEV_TIMEOUT, and the barrier never completed
+    assert limit <= int(elapsed.item()) < limit + 200_000_000
+    # the context still runs the eviction step correctly
+    p = synth.make_problem(0).to("cuda")
+    out = run_evict(p)
+    assert out["status"] == 0
