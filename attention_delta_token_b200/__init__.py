@@ -45,7 +45,12 @@ class FocusError(RuntimeError):
 class FocusDims(ctypes.Structure):
     _fields_ = [("R", ctypes.c_int32), ("B", ctypes.c_int32), ("Hq", ctypes.c_int32),
                 ("Hkv", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("hidden", ctypes.c_int32),
-                ("softmax_scale", ctypes.c_float), ("pool_window", ctypes.c_int32)]
+                ("softmax_scale", ctypes.c_float), ("pool_window", ctypes.c_int32),
+                ("constraints", ctypes.c_int32)]
+
+
+KEEP_PREDECESSOR = 1               # retain each candidate's immediate predecessor
+KEEP_MASKED_BEFORE_RIGHTMOST = 2   # retain masked tokens left of the rightmost candidate
 
 
 def _load() -> ctypes.CDLL:
@@ -82,11 +87,12 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 
 
-def make_dims(R, B, Hq, Hkv, head_dim, hidden, softmax_scale=None, pool_window=3) -> FocusDims:
+def make_dims(R, B, Hq, Hkv, head_dim, hidden, softmax_scale=None, pool_window=3,
+              constraints=0) -> FocusDims:
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(head_dim)
     return FocusDims(int(R), int(B), int(Hq), int(Hkv), int(head_dim), int(hidden),
-                     float(softmax_scale), int(pool_window))
+                     float(softmax_scale), int(pool_window), int(constraints))
 
 
 def _ptr(t: torch.Tensor | None, dtype=None, name="tensor"):
@@ -252,12 +258,20 @@ def focus_selftest_wait_timeout(status, elapsed_ns, limit_ns: int, stream=None):
                                          _stream(stream)), "focus_selftest_wait_timeout")
 
 
-def plan_capacity(decoded, budget) -> int:
-    """Rows the packed batch needs: sum_r min(max(budget_r, 0), masked_r).
+def plan_capacity(decoded, budget, constraints: int = 0) -> int:
+    """Rows the packed batch needs: sum_r k_r with k_r = min(max(budget_r, 0), masked_r).
 
     Host-side planning helper for the scheduler that owns `decoded` and
-    `budget`: the kept-row counts never depend on the attention data."""
+    `budget`: without structural constraints the kept-row counts never depend on
+    the attention data, so this is exact.  With constraints it is the upper bound
+    sum_r min(B, masked_r + k_r) over requests with k_r > 0 (candidates, their
+    predecessors and the other masked tokens)."""
     dec = decoded.detach().cpu()
     bud = budget.detach().cpu().to(torch.int64)
     masked = (dec == 0).sum(dim=1).to(torch.int64)
-    return int(torch.minimum(bud.clamp(min=0), masked).sum())
+    k = torch.minimum(bud.clamp(min=0), masked)
+    if not constraints:
+        return int(k.sum())
+    B = dec.shape[1]
+    bound = torch.where(k > 0, torch.clamp(masked + k, max=B), torch.zeros_like(k))
+    return int(bound.sum())

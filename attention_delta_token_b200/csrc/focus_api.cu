@@ -34,8 +34,9 @@ int row_tiles(const focus_dims_t &d) {
 }
 
 // Workspace: [status 256 B][order: R int32][partial: 2 x R x Hkv x MT x B fp32]
+//            [lists: R x B int32][counts: R int32]   (retained positions under constraints)
 struct WsLayout {
-    size_t status, order, partial, total;
+    size_t status, order, partial, lists, counts, total;
 };
 
 WsLayout ws_layout(const focus_dims_t &d) {
@@ -44,7 +45,9 @@ WsLayout ws_layout(const focus_dims_t &d) {
     w.order = kAlign;
     w.partial = w.order + round_up(sizeof(int32_t) * static_cast<size_t>(d.R), kAlign);
     const size_t np = 2ull * d.R * d.Hkv * row_tiles(d) * d.B;
-    w.total = w.partial + round_up(sizeof(float) * np, kAlign);
+    w.lists = w.partial + round_up(sizeof(float) * np, kAlign);
+    w.counts = w.lists + round_up(sizeof(int32_t) * static_cast<size_t>(d.R) * d.B, kAlign);
+    w.total = w.counts + round_up(sizeof(int32_t) * static_cast<size_t>(d.R), kAlign);
     return w;
 }
 
@@ -54,6 +57,7 @@ focus_status_t check_dims(const focus_dims_t *d) {
         d->pool_window < 1)
         return FOCUS_ERR_INVALID_ARGUMENT;
     if (!isfinite(d->softmax_scale) || d->softmax_scale < 0.f) return FOCUS_ERR_INVALID_ARGUMENT;
+    if (d->constraints < 0 || d->constraints > 3) return FOCUS_ERR_INVALID_ARGUMENT;
     if (d->B > 128 || (d->head_dim != 64 && d->head_dim != 128) || d->Hq % d->Hkv != 0 ||
         d->hidden % 8 != 0 || d->pool_window % 2 == 0)
         return FOCUS_ERR_UNSUPPORTED_SHAPE;
@@ -300,17 +304,7 @@ focus_status_t focus_topk_select(const focus_dims_t *dims, const float *delta,
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint32_t *status = reinterpret_cast<uint32_t *>(ws + ws_layout(d).status);
 
-    focus::PlanParams pp;
-    memset(&pp, 0, sizeof pp);
-    pp.decoded = decoded;
-    pp.budget = budget;
-    pp.cu_seqlens = cu_seqlens;
-    pp.status = status;
-    pp.capacity = capacity;
-    pp.R = d.R;
-    pp.B = d.B;
-    FOCUS_CUDA(focus::launch_plan(pp, s));
-
+    const WsLayout w = ws_layout(d);
     focus::SelectParams sp;
     memset(&sp, 0, sizeof sp);
     sp.delta_in = delta;
@@ -322,6 +316,31 @@ focus_status_t focus_topk_select(const focus_dims_t *dims, const float *delta,
     sp.R = d.R;
     sp.B = d.B;
     sp.pool_window = d.pool_window;
+    if (d.constraints) {
+        // Retained lists per request, then cu_seqlens, then kept_idx from the lists.
+        sp.constraints = d.constraints;
+        sp.budget = budget;
+        sp.lists = reinterpret_cast<int32_t *>(ws + w.lists);
+        sp.counts = reinterpret_cast<int32_t *>(ws + w.counts);
+        FOCUS_CUDA(focus::launch_select_compact(sp, s));
+        focus::ScanParams sc{sp.counts, cu_seqlens, status, capacity, d.R};
+        FOCUS_CUDA(focus::launch_scan(sc, s, /*pdl=*/true));
+        focus::CompactParams cp{nullptr, nullptr, cu_seqlens, nullptr, status, capacity,
+                                d.R, d.B, d.hidden, sp.lists, kept_idx};
+        FOCUS_CUDA(focus::launch_compact(cp, s, /*pdl=*/true));
+        return FOCUS_OK;
+    }
+
+    focus::PlanParams pp;
+    memset(&pp, 0, sizeof pp);
+    pp.decoded = decoded;
+    pp.budget = budget;
+    pp.cu_seqlens = cu_seqlens;
+    pp.status = status;
+    pp.capacity = capacity;
+    pp.R = d.R;
+    pp.B = d.B;
+    FOCUS_CUDA(focus::launch_plan(pp, s));
     FOCUS_CUDA(focus::launch_select_compact(sp, s));
     return FOCUS_OK;
 }
@@ -343,7 +362,7 @@ focus_status_t focus_compact(const focus_dims_t *dims, const void *hidden, const
     focus::CompactParams p{static_cast<const uint16_t *>(hidden), kept_idx, cu_seqlens,
                            static_cast<uint16_t *>(packed),
                            reinterpret_cast<uint32_t *>(ws + ws_layout(d).status), capacity,
-                           d.R, d.B, d.hidden};
+                           d.R, d.B, d.hidden, nullptr, nullptr};
     FOCUS_CUDA(focus::launch_compact(p, static_cast<cudaStream_t>(stream)));
     return FOCUS_OK;
 }
@@ -388,7 +407,7 @@ focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void 
     pp.decoded = decoded;
     pp.budget = budget;
     pp.order = const_cast<int32_t *>(p.order);
-    pp.cu_seqlens = cu_seqlens;
+    pp.cu_seqlens = d.constraints ? nullptr : cu_seqlens;  // with constraints: after selection
     pp.status = p.status;
     pp.capacity = capacity;
     pp.R = d.R;
@@ -414,10 +433,25 @@ focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void 
     sp.MT = p.MT;
     sp.H = d.hidden;
     sp.pool_window = d.pool_window;
+    if (d.constraints) {
+        const WsLayout w = ws_layout(d);
+        sp.constraints = d.constraints;
+        sp.budget = budget;
+        sp.lists = reinterpret_cast<int32_t *>(ws + w.lists);
+        sp.counts = reinterpret_cast<int32_t *>(ws + w.counts);
+        FOCUS_CUDA(focus::launch_select_compact(sp, s, /*pdl=*/true));
+        focus::ScanParams sc{sp.counts, cu_seqlens, p.status, capacity, d.R};
+        FOCUS_CUDA(focus::launch_scan(sc, s, /*pdl=*/true));
+        focus::CompactParams cp{static_cast<const uint16_t *>(hidden), nullptr, cu_seqlens,
+                                static_cast<uint16_t *>(packed), p.status, capacity, d.R, d.B,
+                                d.hidden, sp.lists, kept_idx};
+        FOCUS_CUDA(focus::launch_compact(cp, s, /*pdl=*/true));
+        return FOCUS_OK;
+    }
     FOCUS_CUDA(focus::launch_select_compact(sp, s, /*pdl=*/true));
     focus::CompactParams cp{static_cast<const uint16_t *>(hidden), kept_idx, cu_seqlens,
                             static_cast<uint16_t *>(packed), p.status, capacity, d.R, d.B,
-                            d.hidden};
+                            d.hidden, nullptr, nullptr};
     FOCUS_CUDA(focus::launch_compact(cp, s, /*pdl=*/true));
     return FOCUS_OK;
 }

@@ -87,7 +87,23 @@ struct SelectParams {
     uint32_t *status;
     long long capacity;
     int R, B, Hkv, MT, H, pool_window;
+    // Structural constraints (constraints != 0): the retained positions of request r
+    // go to lists[r*B ..] and their number to counts[r]; kept_idx/cu_seqlens are
+    // written later by the scan and list-driven compaction.
+    int constraints;
+    const int32_t *budget;     // [R]
+    int32_t *lists;            // [R*B]
+    int32_t *counts;           // [R]
 };
+
+struct ScanParams {
+    const int32_t *counts;     // [R]
+    int32_t *cu_seqlens;       // [R+1]
+    uint32_t *status;
+    long long capacity;
+    int R;
+};
+cudaError_t launch_scan(const ScanParams &p, cudaStream_t stream, bool pdl = false);
 cudaError_t launch_select_compact(const SelectParams &p, cudaStream_t stream, bool pdl = false);
 
 struct DeltaParams {
@@ -106,12 +122,14 @@ struct ReduceParams {
 cudaError_t launch_reduce(const ReduceParams &p, cudaStream_t stream);
 
 struct CompactParams {
-    const uint16_t *hidden;
+    const uint16_t *hidden;    // null: write kept_idx from lists only, copy nothing
     const int32_t *kept_idx, *cu_seqlens;
     uint16_t *packed;
     uint32_t *status;
     long long capacity;
     int R, B, H;
+    const int32_t *lists;      // non-null: row t of request r is lists[r*B + t], written to kept_out
+    int32_t *kept_out;
 };
 cudaError_t launch_compact(const CompactParams &p, cudaStream_t stream, bool pdl = false);
 

@@ -238,6 +238,39 @@ __global__ void __launch_bounds__(256) select_compact_kernel(const SelectParams 
     }
     __syncthreads();
 
+    if (p.constraints) {
+        // Candidates, then the structural constraints; the retained positions go to a
+        // per-request list (their count depends on the data: cu_seqlens comes later).
+        __shared__ int rightmost;
+        const int masked = __syncthreads_count(j < B && dec_s[j] == 0);
+        const int k = min(max(p.budget[r], 0), masked);
+        if (j == 0) rightmost = -1;
+        if (j < B) {
+            const float v = val_s[j];
+            int rank = 0;
+            for (int t = 0; t < B; ++t) {
+                const float u = val_s[t];
+                rank += dec_s[t] == 0 && ((u > v) || (u == v && t < j));
+            }
+            sel_s[j] = (dec_s[j] == 0 && rank < k) ? 1 : 0;
+        }
+        __syncthreads();
+        if (j < B && sel_s[j]) atomicMax(&rightmost, j);
+        __syncthreads();
+        const bool keep = j < B && (sel_s[j] ||
+                                    ((p.constraints & 1) && j + 1 < B && sel_s[j + 1]) ||
+                                    ((p.constraints & 2) && dec_s[j] == 0 && j < rightmost));
+        if (j < 128) kept_s[j] = keep ? 1 : 0;
+        const int n = __syncthreads_count(keep);
+        if (keep) {
+            int slot = 0;
+            for (int t = 0; t < j; ++t) slot += kept_s[t];
+            p.lists[rb + slot] = j;
+        }
+        if (j == 0) p.counts[r] = n;
+        return;
+    }
+
     const long long base = p.cu_seqlens[r];
     const int k = static_cast<int>(p.cu_seqlens[r + 1] - base);
     select_block(val_s, dec_s, B, k, base, p.capacity, sel_s, kept_s, p.kept_idx, p.status);
@@ -304,11 +337,19 @@ __global__ void __launch_bounds__(256) compact_kernel(const CompactParams p) {
             const int mid = (lo + hi + 1) >> 1;
             if (p.cu_seqlens[mid] <= row) lo = mid; else hi = mid - 1;
         }
-        const int jj = p.kept_idx[row];
+        int jj;
+        if (p.lists) {  // structural constraints: row t of request lo is its t-th list entry
+            const long long t = row - p.cu_seqlens[lo];
+            jj = (t >= 0 && t < p.B) ? p.lists[static_cast<size_t>(lo) * p.B + t] : -1;
+            if (lane == 0 && jj >= 0 && jj < p.B) p.kept_out[row] = jj;
+        } else {
+            jj = p.kept_idx[row];
+        }
         if (jj < 0 || jj >= p.B) {
             if (lane == 0) atomicOr(p.status, FOCUS_DEV_BAD_INPUT);
             continue;
         }
+        if (!p.hidden) continue;
         const uint4 *__restrict__ src = reinterpret_cast<const uint4 *>(p.hidden) +
                                         (static_cast<size_t>(lo) * p.B + jj) * nvec;
         uint4 *__restrict__ dst = reinterpret_cast<uint4 *>(p.packed) + static_cast<size_t>(row) * nvec;
@@ -325,7 +366,30 @@ __global__ void __launch_bounds__(256) compact_kernel(const CompactParams p) {
     }
 }
 
+// cu_seqlens from per-request counts (one CTA; chunks of kPlanThreads), capacity check.
+__global__ void __launch_bounds__(kPlanThreads) scan_kernel(const ScanParams p) {
+    __shared__ int warp_tot[33];
+    pdl_launch_dependents();
+    pdl_wait();  // counts come from the selection kernel
+    int running = 0;
+    if (threadIdx.x == 0) p.cu_seqlens[0] = 0;
+    for (int base = 0; base < p.R; base += kPlanThreads) {
+        const int r = base + threadIdx.x;
+        const int c = r < p.R ? p.counts[r] : 0;
+        int total;
+        const int ex = block_exclusive_scan(c, warp_tot, total);
+        if (r < p.R) p.cu_seqlens[r + 1] = running + ex + c;
+        running += total;
+    }
+    if (threadIdx.x == 0 && static_cast<long long>(running) > p.capacity)
+        atomicOr(p.status, FOCUS_DEV_CAPACITY);
+}
+
 }  // namespace
+
+cudaError_t launch_scan(const ScanParams &p, cudaStream_t stream, bool pdl) {
+    return launch_kernel(scan_kernel, dim3(1), dim3(kPlanThreads), 0, stream, pdl, p);
+}
 
 cudaError_t launch_plan(const PlanParams &p, cudaStream_t stream) {
     plan_kernel<<<1, kPlanThreads, 0, stream>>>(p);

@@ -211,9 +211,9 @@ def run_ours(args, rank, world, local_rank):
     seed = rank_seed(args.config, rank)
     p = synth.make_problem(cfg, seed=seed, device=dev)
     counts = algorithmic_counts(p)
-    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, args.constraints)
     ws = F.Workspace(dims, dev)
-    cap = F.plan_capacity(p.decoded, p.budget)
+    cap = F.plan_capacity(p.decoded, p.budget, args.constraints)
     kept, cu, packed = make_outputs(p, cap, dev)
     stream = torch.cuda.current_stream(dev)
     in_bytes = sum(t.numel() * t.element_size() for t in p.tensors().values())
@@ -321,6 +321,7 @@ def run_ours(args, rank, world, local_rank):
                 "input_bytes_per_step": int(in_bytes),
                 "l2": f"no flush: {in_bytes / 2**30:.2f} GiB of inputs per step > 126 MB L2",
                 "accumulate": "fp32", "parallelism": f"dp{world} (request-sharded replicas)",
+                "constraints": args.constraints,
             },
             "decisions_per_s": world * counts["decisions"] / step_s,
             "roofline": {
@@ -340,7 +341,8 @@ def run_ours(args, rank, world, local_rank):
                 "peaks": f"{peak_src}: hbm {hbm} GB/s, bf16 {tc} TFLOP/s",
             },
             "clocks": clocks,
-            "gpu_launches": 4 * args.steps,  # plan, attention statistics, select, compact
+            # plan, attention statistics, select, (scan,) compact
+            "gpu_launches": (5 if args.constraints else 4) * args.steps,
             "e2e": e2e,
             "impl": "ours",
         }
@@ -425,6 +427,9 @@ def main():
     ap.add_argument("--config", type=int, default=synth.METRIC_CONFIG)
     ap.add_argument("--requests", type=int, default=0,
                     help="override the workload's request count (same shape; for profiling)")
+    ap.add_argument("--constraints", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="structural constraints on the retained set (bit 1: predecessors, "
+                         "bit 2: masked tokens left of the rightmost candidate)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -33,11 +33,13 @@
  *    focus_read_device_status().
  *  - Shapes: 1 <= B <= 128; head_dim in {64, 128}; Hq % Hkv == 0 and
  *    G = Hq / Hkv divides 128; hidden % 8 == 0; pool_window odd and >= 1;
- *    R >= 1.  Other shapes return FOCUS_ERR_UNSUPPORTED_SHAPE.
+ *    R >= 1; constraints in 0..3 (else FOCUS_ERR_INVALID_ARGUMENT).  Other shapes
+ *    return FOCUS_ERR_UNSUPPORTED_SHAPE.
  *  - Per-request budgets are clamped to [0, masked_r] on the device, so
- *    k_r = min(max(budget[r], 0), masked_r).  k_r depends only on `decoded`
- *    and `budget`, never on the attention data, so the host scheduler that
- *    owns both can size `capacity` = sum_r k_r exactly.
+ *    k_r = min(max(budget[r], 0), masked_r).  Without structural constraints
+ *    (dims.constraints == 0) k_r depends only on `decoded` and `budget`, never on
+ *    the attention data, so the host scheduler that owns both can size
+ *    `capacity` = sum_r k_r exactly.
  *  - Kept positions are written in ascending order per request; requests are
  *    packed in order: request r owns rows cu_seqlens[r] .. cu_seqlens[r+1]-1.
  */
@@ -51,7 +53,7 @@
 extern "C" {
 #endif
 
-#define FOCUS_ABI_VERSION 1
+#define FOCUS_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define FOCUS_API __attribute__((visibility("default")))
@@ -80,7 +82,25 @@ typedef struct {
     int32_t hidden;        /* hidden size H of the rows that are compacted            */
     float softmax_scale;   /* logit = softmax_scale * q.k (usually 1/sqrt(d)); finite, >= 0 */
     int32_t pool_window;   /* MaxPool1D window (odd; the method uses 3)               */
+    int32_t constraints;   /* structural constraints on the retained set, bit mask:
+                              FOCUS_KEEP_PREDECESSOR | FOCUS_KEEP_MASKED_BEFORE_RIGHTMOST;
+                              0 keeps exactly the top-K candidates                   */
 } focus_dims_t;
+
+/*
+ * Structural constraints ("What carries the argument": after the top-K candidates
+ * are chosen, each candidate's immediate predecessor and all masked tokens before
+ * the rightmost candidate are retained as well).  With either bit set:
+ *   retained_r = candidates_r
+ *              U {j - 1 : j a candidate, j >= 1}            (FOCUS_KEEP_PREDECESSOR;
+ *                                                          masked or decoded)
+ *              U {masked j : j < rightmost candidate}    (FOCUS_KEEP_MASKED_BEFORE_RIGHTMOST)
+ * in ascending order.  The retained count then depends on the attention data,
+ * so `capacity` must be an upper bound (sum over requests of
+ * min(B, masked_r + k_r) is one) and cu_seqlens is computed on the device.
+ */
+#define FOCUS_KEEP_PREDECESSOR 1
+#define FOCUS_KEEP_MASKED_BEFORE_RIGHTMOST 2
 
 /* Bytes of workspace every entry point below needs for `dims` (256-byte aligned). */
 FOCUS_API size_t focus_workspace_size(const focus_dims_t *dims);
@@ -136,7 +156,8 @@ FOCUS_API focus_status_t focus_importance_delta(const focus_dims_t *dims, const 
  *   k_r = min(max(budget[r], 0), #{j : decoded[r][j] == 0})
  *   kept_idx[cu_seqlens[r] ..] = the k_r positions ranked first by
  *                                (delta desc, position asc), in ascending position order
- *   cu_seqlens[0] = 0, cu_seqlens[r+1] = cu_seqlens[r] + k_r
+ *                                (plus the structural constraints of dims.constraints)
+ *   cu_seqlens[0] = 0, cu_seqlens[r+1] = cu_seqlens[r] + (rows kept for request r)
  *   delta [R, B] float32 (as produced by focus_importance_delta); budget [R] int32;
  *   kept_idx [capacity] int32 out; cu_seqlens [R + 1] int32 out.
  * Rows beyond `capacity` are not written and FOCUS_ERR_CAPACITY is set in the

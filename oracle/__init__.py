@@ -91,9 +91,11 @@ class Oracle:
         lib.focus_oracle_delta.argtypes = [i32, i32, i32, P, P, P, P, P]
         lib.focus_oracle_select.argtypes = [i32, i32, P, P, P, P, P, i64]
         lib.focus_oracle_compact.argtypes = [i32, i32, i32, P, P, P, P, i64]
+        lib.focus_oracle_select_structured.argtypes = [i32, i32, P, P, P, i32, P, P, i64]
         lib.focus_oracle_num_threads.argtypes = []
         for fn in (lib.focus_oracle_importance, lib.focus_oracle_delta, lib.focus_oracle_select,
-                   lib.focus_oracle_compact, lib.focus_oracle_num_threads):
+                   lib.focus_oracle_compact, lib.focus_oracle_num_threads,
+                   lib.focus_oracle_select_structured):
             fn.restype = ctypes.c_int
         self.lib = lib
 
@@ -145,6 +147,23 @@ class Oracle:
         n = min(cap, int(cu[-1]))
         return kept[:n], cu, st
 
+    def select_structured(self, pooled, decoded, budget, constraints: int, *,
+                          capacity: int | None = None):
+        """Top-k candidates plus the structural constraints (bit 1: each candidate's
+        predecessor; bit 2: masked tokens before the rightmost candidate).
+        Returns (kept [n] int32, cu_seqlens [R+1] int32, status)."""
+        pv = _arr(pooled, np.float64)
+        dec = _arr(decoded, np.uint8)
+        bud = _arr(budget, np.int32)
+        R, B = pv.shape
+        cap = R * B if capacity is None else int(capacity)
+        kept = np.full((max(cap, 1),), -1, np.int32)
+        cu = np.zeros((R + 1,), np.int32)
+        st = self.lib.focus_oracle_select_structured(R, B, _p(pv), _p(dec), _p(bud),
+                                                     int(constraints), _p(kept), _p(cu), cap)
+        _check(st, "select_structured", allow_capacity=True)
+        return kept[:min(cap, int(cu[-1]))], cu, st
+
     def compact(self, hidden, kept, cu_seqlens, *, capacity: int | None = None) -> np.ndarray:
         """packed [capacity, H] uint16 (bf16 bits) of the kept hidden rows."""
         hid = _u16(hidden)
@@ -159,7 +178,7 @@ class Oracle:
         _check(st, "compact")
         return packed[:capacity]
 
-    def evict(self, p) -> dict:
+    def evict(self, p, constraints: int = 0) -> dict:
         """The whole step on a problem object with the fields of ``synth.FocusProblem``.
 
         Returns float64 i0, i1, delta (raw), pooled (masked) [R, B]; int32 kept
@@ -170,7 +189,10 @@ class Oracle:
         i1 = self.importance(p.q1, p.k1_prefix, p.cu_prefix, p.k1_block, Hq=p.Hq, Hkv=p.Hkv,
                              scale=p.scale)
         raw, pooled = self.delta_pool_mask(i0, i1, p.decoded, window=p.pool_window)
-        kept, cu, st = self.select(pooled, p.decoded, p.budget)
+        if constraints:
+            kept, cu, st = self.select_structured(pooled, p.decoded, p.budget, constraints)
+        else:
+            kept, cu, st = self.select(pooled, p.decoded, p.budget)
         packed = self.compact(p.hidden, kept, cu)
         return dict(i0=i0, i1=i1, delta=raw, pooled=pooled, kept=kept, cu_seqlens=cu,
                     packed=packed)
@@ -207,5 +229,9 @@ def compact(*a, **k):
     return default().compact(*a, **k)
 
 
-def evict(p) -> dict:
-    return default().evict(p)
+def evict(p, constraints: int = 0) -> dict:
+    return default().evict(p, constraints)
+
+
+def select_structured(*a, **k):
+    return default().select_structured(*a, **k)

@@ -286,6 +286,77 @@ int focus_oracle_select(int R, int B, const double *pooled, const uint8_t *decod
 }
 
 /*
+ * Structural constraints on the retained set ("What carries the argument": after
+ * the top-K candidates are chosen, each candidate's immediate predecessor and all
+ * masked tokens before the rightmost candidate are retained as well).
+ *
+ *   S_r        = the top-k_r candidates of request r (focus_oracle_select's rule)
+ *   retained_r = S_r
+ *              U {j - 1 : j in S_r, j >= 1}                     (constraints & 1)
+ *              U {j : j < max S_r, decoded[r][j] == 0}          (constraints & 2)
+ *   written in ascending position order; cu[r+1] = cu[r] + |retained_r|.
+ *
+ * A predecessor is retained whether it is masked or decoded; the second rule adds
+ * masked positions only.  Returns ORACLE_CAPACITY (cu complete) past capacity.
+ */
+int focus_oracle_select_structured(int R, int B, const double *pooled, const uint8_t *decoded,
+                                   const int32_t *budget, int constraints, int32_t *kept,
+                                   int32_t *cu_seqlens, int64_t capacity)
+{
+    if (R < 0 || B <= 0 || capacity < 0 || constraints < 0 || constraints > 3)
+        return ORACLE_BAD_ARGUMENT;
+    int32_t *cand = (int32_t *)malloc(sizeof(int32_t) * (size_t)B);
+    int32_t cand_cu[2];
+    unsigned char *keep = (unsigned char *)malloc((size_t)B);
+    if (!cand || !keep) {
+        free(cand); free(keep);
+        return ORACLE_NO_MEMORY;
+    }
+    int status = ORACLE_OK;
+    cu_seqlens[0] = 0;
+    for (int r = 0; r < R; ++r) {
+        /* The candidates: the plain top-k selection of this one request. */
+        int st = focus_oracle_select(1, B, pooled + (size_t)r * B, decoded + (size_t)r * B,
+                                     budget + r, cand, cand_cu, B);
+        if (st != ORACLE_OK) {
+            free(cand); free(keep);
+            return st;
+        }
+        const int k = cand_cu[1];
+        for (int j = 0; j < B; ++j)
+            keep[j] = 0;
+        int rightmost = -1;
+        for (int t = 0; t < k; ++t) {
+            keep[cand[t]] = 1;
+            if (cand[t] > rightmost)
+                rightmost = cand[t];
+        }
+        if (constraints & 1)
+            for (int t = 0; t < k; ++t)
+                if (cand[t] >= 1)
+                    keep[cand[t] - 1] = 1;
+        if (constraints & 2)
+            for (int j = 0; j < rightmost; ++j)
+                if (decoded[(size_t)r * B + j] == 0)
+                    keep[j] = 1;
+        int64_t row = cu_seqlens[r];
+        for (int j = 0; j < B; ++j) {
+            if (!keep[j])
+                continue;
+            if (row < capacity)
+                kept[row] = j;
+            else
+                status = ORACLE_CAPACITY;
+            ++row;
+        }
+        cu_seqlens[r + 1] = (int32_t)row;
+    }
+    free(cand);
+    free(keep);
+    return status;
+}
+
+/*
  * Compaction of the retained tokens' hidden rows into a packed varlen batch:
  *   packed[cu[r] + t][:] = hidden[r][kept[cu[r] + t]][:]   (bit copy)
  */

@@ -18,13 +18,13 @@ RTOL = 1e-2
 TIE_TOL = 2e-3
 
 
-def run_evict(p, *, outputs=True, capacity=None, stream=None):
+def run_evict(p, *, outputs=True, capacity=None, stream=None, constraints=0):
     """focus_evict on a problem whose tensors live on the GPU.  Returns numpy arrays."""
     import attention_delta_token_b200 as F
     dev = p.q0.device
-    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, constraints)
     ws = F.Workspace(dims, dev)
-    cap = F.plan_capacity(p.decoded, p.budget) if capacity is None else capacity
+    cap = F.plan_capacity(p.decoded, p.budget, constraints) if capacity is None else capacity
     kept = torch.full((max(cap, 1),), -1, dtype=torch.int32, device=dev)[:cap]
     cu = torch.full((p.R + 1,), -7, dtype=torch.int32, device=dev)
     packed = torch.zeros((max(cap, 1), p.H), dtype=torch.bfloat16, device=dev)[:cap]
@@ -34,8 +34,9 @@ def run_evict(p, *, outputs=True, capacity=None, stream=None):
                   p.hidden, p.decoded, p.budget, kept, cu, packed, ws, delta_out=delta,
                   i0_out=i0, i1_out=i1, stream=stream)
     status = F.focus_read_device_status(ws, stream)
-    out = dict(kept=kept.cpu().numpy(), cu_seqlens=cu.cpu().numpy(),
-               packed=packed.view(torch.int16).cpu().numpy().view(np.uint16), status=status)
+    n = min(cap, int(cu[-1].item())) if constraints else cap
+    out = dict(kept=kept[:n].cpu().numpy(), cu_seqlens=cu.cpu().numpy(),
+               packed=packed[:n].view(torch.int16).cpu().numpy().view(np.uint16), status=status)
     if outputs:
         out.update(delta=delta.cpu().numpy().astype(np.float64), i0=i0.cpu().numpy().astype(np.float64),
                    i1=i1.cpu().numpy().astype(np.float64))
@@ -90,6 +91,33 @@ def check_selection(kept_gpu, cu_gpu, pooled_oracle, decoded, budget, requests=N
             f"differing positions {diff.tolist()} have pooled delta {orow[diff].tolist()}, k-th {kth}")
         tie_only += 1
     return exact, len(list(reqs)), tie_only
+
+
+def check_structured(kept_gpu, cu_gpu, kept_oracle, cu_oracle, pooled_oracle, decoded, budget,
+                     requests=None):
+    """Retained sets under structural constraints.  A request whose candidate set is
+    decided by a margin (oracle k-th and (k+1)-th pooled values more than 2e-3 apart)
+    must match the oracle exactly; requests inside the tie band only need a valid,
+    ascending, unique set.  Returns (n_exact, n_checked)."""
+    pooled_oracle = np.asarray(pooled_oracle, np.float64)
+    decoded = np.asarray(decoded)
+    budget = np.asarray(budget)
+    R, B = decoded.shape
+    reqs = range(R) if requests is None else requests
+    exact = 0
+    for i, r in enumerate(reqs):
+        got = kept_gpu[cu_gpu[r]:cu_gpu[r + 1]]
+        assert (np.diff(got) > 0).all() and ((got >= 0) & (got < B)).all(), (r, got)
+        orow = pooled_oracle[i]
+        masked = np.flatnonzero(decoded[r] == 0)
+        k = min(max(int(budget[r]), 0), masked.size)
+        vals = np.sort(orow[masked])[::-1]
+        decided = k == 0 or k == masked.size or vals[k - 1] - vals[k] > TIE_TOL
+        if decided:
+            want = kept_oracle[cu_oracle[i]:cu_oracle[i + 1]]
+            np.testing.assert_array_equal(got, want, err_msg=f"retained set of request {r}")
+            exact += 1
+    return exact, len(list(reqs))
 
 
 def check_packed(packed, kept, cu, hidden_bits, requests=None):

@@ -325,6 +325,55 @@ def pin_hand_evict(orc):
             packed, hidden[0, want].view(torch.int16).numpy().view(np.uint16).reshape(len(want), H))
 
 
+# --------------------------------------------------------------------------- structural constraints
+
+def _num(x):
+    return -np.inf if x == "-inf" else float(x)
+
+
+def pin_hand_structural(orc):
+    """Hand-worked retained sets for every constraint combination
+    (tests/golden/hand_structural_b8.json)."""
+    fx = json.load(open(os.path.join(GOLDEN, "hand_structural_b8.json")))
+    for case in fx["cases"]:
+        dec = np.array([case["decoded"]], np.uint8)
+        pooled = np.array([[_num(x) for x in case["pooled"]]])
+        bud = np.array([case["budget"]], np.int32)
+        for c, want in case["retained"].items():
+            kept, cu, st = orc.select_structured(pooled, dec, bud, int(c))
+            assert st == 0 and kept.tolist() == want, (case["derivation"], c, kept, want)
+            assert cu.tolist() == [0, len(want)]
+
+
+def pin_structural_properties(orc):
+    """On random blocks: constraints 0 equal the plain top-k; the retained set
+    contains the candidates, every candidate's predecessor (bit 1) and every masked
+    position left of the rightmost candidate (bit 2), and nothing else; it is
+    ascending and unique."""
+    rng = np.random.default_rng(16)
+    R, B = 30, 12
+    pooled = rng.integers(-3, 4, size=(R, B)).astype(np.float64)
+    dec = (rng.random((R, B)) < 0.3).astype(np.uint8)
+    pooled[dec != 0] = -np.inf
+    budget = rng.integers(0, 6, size=R).astype(np.int32)
+    cand, ccu, _ = orc.select(pooled, dec, budget)
+    k0, cu0, _ = orc.select_structured(pooled, dec, budget, 0)
+    np.testing.assert_array_equal(k0, cand)
+    np.testing.assert_array_equal(cu0, ccu)
+    for c in (1, 2, 3):
+        kept, cu, _ = orc.select_structured(pooled, dec, budget, c)
+        for r in range(R):
+            got = kept[cu[r]:cu[r + 1]].tolist()
+            S = set(cand[ccu[r]:ccu[r + 1]].tolist())
+            assert got == sorted(set(got))
+            want = set(S)
+            if c & 1:
+                want |= {j - 1 for j in S if j >= 1}
+            if c & 2 and S:
+                want |= {j for j in range(max(S)) if dec[r, j] == 0}
+            assert set(got) == want, (r, c, got, sorted(want))
+
+
 PINS = [
     pin_hand_two_tokens, pin_rows_sum_to_one_without_prefix, pin_prefix_takes_share,
     pin_zero_queries_uniform, pin_single_key_block, pin_prefix_permutation_invariance,
@@ -332,4 +381,5 @@ PINS = [
     pin_heads_sum, pin_requests_independent, pin_library_softmax_columns,
     pin_delta_sign_and_pool, pin_pool_spreads_decoded_neighbour, pin_topk_lexsort,
     pin_topk_bruteforce, pin_capacity_status, pin_compact_fancy_indexing, pin_hand_evict,
+    pin_hand_structural, pin_structural_properties,
 ]

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol():
 def test_status_strings_and_version():
     for code, name in F.STATUS.items():
         assert F.focus_status_string(code) == name
-    assert F.focus_abi_version() == 1
+    assert F.focus_abi_version() == 2
 
 
 def dims(**kw):
@@ -55,9 +55,10 @@ def test_workspace_size():
     d = dims()
     n = F.focus_workspace_size(d)
     # status (256) + order (R int32, rounded to 256) + 2 layers x R x Hkv x MT x B fp32
-    assert n == 256 + 256 + 2 * 4 * 8 * 1 * 32 * 4
+    # + retained lists (R x B int32) + counts (R int32), each rounded to 256
+    assert n == 256 + 256 + 2 * 4 * 8 * 1 * 32 * 4 + 512 + 256
     d3 = dims(B=128)  # G*B = 512 -> 4 row tiles
-    assert F.focus_workspace_size(d3) == 256 + 256 + 2 * 4 * 8 * 4 * 128 * 4
+    assert F.focus_workspace_size(d3) == 256 + 256 + 2 * 4 * 8 * 4 * 128 * 4 + 2048 + 256
     assert F._lib.focus_workspace_size(None) == 0
     assert F._lib.focus_workspace_size(ctypes.byref(dims(B=0))) == 0
 
@@ -66,6 +67,7 @@ BAD_DIMS = [
     (dict(R=0), INVALID), (dict(B=0), INVALID), (dict(Hq=0), INVALID),
     (dict(softmax_scale=-1.0), INVALID), (dict(softmax_scale=math.nan), INVALID),
     (dict(softmax_scale=math.inf), INVALID), (dict(pool_window=0), INVALID),
+    (dict(constraints=4), INVALID), (dict(constraints=-1), INVALID),
     (dict(B=129), UNSUPPORTED), (dict(head_dim=96), UNSUPPORTED), (dict(head_dim=256), UNSUPPORTED),
     (dict(Hq=30, Hkv=8), UNSUPPORTED), (dict(Hq=24, Hkv=8), UNSUPPORTED),
     (dict(Hq=256, Hkv=1), UNSUPPORTED), (dict(hidden=4092), UNSUPPORTED),
@@ -136,6 +138,21 @@ def test_other_entry_points_check_pointers():
     assert L.focus_compact(ctypes.byref(d), A, A, A, A, 16, A, 8, None) == WORKSPACE
     assert L.focus_read_device_status(None, None, 10) == WORKSPACE
     assert L.focus_clear_device_status(None, 1024, None) == WORKSPACE
+
+
+def test_plan_capacity_bounds_structured_counts():
+    """With structural constraints plan_capacity is an upper bound of the retained rows."""
+    import oracle
+    import synth
+    rng = np.random.default_rng(3)
+    for cfg in range(5):
+        p = synth.make_problem(cfg, overrides=dict(R=min(synth.CONFIGS[cfg].R, 12), d=64,
+                                                   prefix=("fixed", 0)))
+        pooled = rng.normal(size=(p.R, p.B))
+        pooled[p.decoded.numpy() != 0] = -np.inf
+        for c in (1, 2, 3):
+            _, cu, _ = oracle.select_structured(pooled, p.decoded, p.budget, c)
+            assert F.plan_capacity(p.decoded, p.budget, c) >= int(cu[-1])
 
 
 def test_plan_capacity_matches_oracle_counts():

@@ -232,3 +232,78 @@ def test_bounded_wait_times_out_and_reports():
     p = synth.make_problem(0).to("cuda")
     out = run_evict(p)
     assert out["status"] == 0
+
+
+STRUCTURED_CASES = {
+    "sdar_r8_wide": (1, dict(R=8, prefix=("uniform", 0, 600)), True),
+    "ragged_r10_ties": (4, dict(R=10, prefix=("loguniform", 500)), True),
+    "block128_r3": (3, dict(R=3, prefix=("uniform", 100, 300)), True),
+    "tiny": (0, {}, False),
+}
+
+
+@pytest.mark.parametrize("constraints", [1, 2, 3])
+@pytest.mark.parametrize("case", sorted(STRUCTURED_CASES))
+def test_structural_constraints_vs_oracle(case, constraints, orc):
+    """Retained sets with the structural constraints ("What carries the argument"):
+    candidates plus predecessors and/or masked tokens left of the rightmost one."""
+    from focus_testutil import check_structured
+    cfg, ov, wide = STRUCTURED_CASES[case]
+    p = synth.make_problem(cfg, seed=300 + constraints, wide_logits=wide, overrides=ov)
+    ref = orc.evict(p, constraints=constraints)
+    out = run_evict(p.to("cuda"), constraints=constraints)
+    assert out["status"] == 0, out["status"]
+    assert_close_importance(out["i0"], ref["i0"], "I0")
+    assert_close_importance(out["i1"], ref["i1"], "I1")
+    assert_close_delta(out["delta"], ref["pooled"])
+    exact, n = check_structured(out["kept"], out["cu_seqlens"], ref["kept"], ref["cu_seqlens"],
+                                ref["pooled"], p.decoded.numpy(), p.budget.numpy())
+    assert exact >= n // 2, (exact, n)
+    check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))
+
+
+def test_structural_topk_select_exact(orc):
+    """Stand-alone focus_topk_select with constraints on exact (grid) values: the
+    retained lists and cu_seqlens equal the oracle's bit for bit, ties included."""
+    import attention_delta_token_b200 as F
+    rng = np.random.default_rng(21)
+    p = synth.make_problem(4, overrides=dict(R=40, prefix=("fixed", 0)))
+    vals = (rng.integers(-3, 4, size=(p.R, p.B)) * 0.5).astype(np.float32)
+    vals[p.decoded.numpy() != 0] = -np.inf
+    for c in (1, 2, 3):
+        dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, c)
+        ws = F.Workspace(dims)
+        cap = F.plan_capacity(p.decoded, p.budget, c)
+        kept = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+        cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+        F.focus_topk_select(dims, torch.from_numpy(vals).cuda(), p.decoded.cuda(),
+                            p.budget.cuda(), kept, cu, ws)
+        assert F.focus_read_device_status(ws) == 0
+        okept, ocu, _ = orc.select_structured(vals.astype(np.float64), p.decoded, p.budget, c)
+        np.testing.assert_array_equal(cu.cpu().numpy(), ocu)
+        np.testing.assert_array_equal(kept[:int(ocu[-1])].cpu().numpy(), okept)
+
+
+def test_structural_full_config_sampled(orc):
+    """Constraints on a full-size workload in the benchmark's launch configuration,
+    checked on sampled requests; cu_seqlens must be consistent with the lists."""
+    from focus_testutil import check_structured
+    p = synth.make_problem(4, wide_logits=True)
+    out = run_evict(p.to("cuda"), constraints=3)
+    assert out["status"] == 0
+    req = _sample_requests(p)
+    ref = orc.evict(p.subset(req), constraints=3)
+    assert_close_delta(out["delta"][req], ref["pooled"])
+    # compare the sampled requests' retained sets
+    got_kept, got_cu = [], [0]
+    for r in req:
+        seg = out["kept"][out["cu_seqlens"][r]:out["cu_seqlens"][r + 1]]
+        got_kept.append(seg)
+        got_cu.append(got_cu[-1] + len(seg))
+    got_kept = np.concatenate(got_kept) if got_kept else np.zeros(0, np.int32)
+    dec = p.decoded.numpy()[req]
+    bud = p.budget.numpy()[req]
+    exact, n = check_structured(got_kept, np.array(got_cu), ref["kept"], ref["cu_seqlens"],
+                                ref["pooled"], dec, bud)
+    assert exact >= n // 2, (exact, n)
+    check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))

@@ -31,6 +31,12 @@ MUTATIONS = {
     "output_not_ascending": ("while (t > 0 && chosen[t - 1] > x)", "while (0)"),
     "compact_wrong_source": ("hidden + ((size_t)r * B + j) * H",
                              "hidden + ((size_t)r * B + (row - cu_seqlens[r])) * H"),
+    "successor_instead_of_predecessor": ("keep[cand[t] - 1] = 1;", "keep[cand[t] + 1 < B ? cand[t] + 1 : cand[t]] = 1;"),
+    "predecessor_only_if_masked": ("                if (cand[t] >= 1)\n                    keep[cand[t] - 1] = 1;",
+                                   "                if (cand[t] >= 1 && !decoded[(size_t)r * B + cand[t] - 1])\n                    keep[cand[t] - 1] = 1;"),
+    "rightmost_rule_keeps_decoded": ("                if (decoded[(size_t)r * B + j] == 0)\n                    keep[j] = 1;",
+                                     "                keep[j] = 1;"),
+    "rightmost_rule_uses_leftmost": ("            if (cand[t] > rightmost)", "            if (rightmost < 0 || cand[t] < rightmost)"),
 }
 
 
