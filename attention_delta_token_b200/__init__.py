@@ -46,11 +46,13 @@ class FocusDims(ctypes.Structure):
     _fields_ = [("R", ctypes.c_int32), ("B", ctypes.c_int32), ("Hq", ctypes.c_int32),
                 ("Hkv", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("hidden", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("pool_window", ctypes.c_int32),
-                ("constraints", ctypes.c_int32)]
+                ("constraints", ctypes.c_int32), ("score", ctypes.c_int32)]
 
 
 KEEP_PREDECESSOR = 1               # retain each candidate's immediate predecessor
 KEEP_MASKED_BEFORE_RIGHTMOST = 2   # retain masked tokens left of the rightmost candidate
+SCORE_DELTA = 0                    # rank by I1 - I0 (the method)
+SCORE_LAYER1 = 1                   # rank by I1 alone (Figure 13 ablation; layer 0 skipped)
 
 
 def _load() -> ctypes.CDLL:
@@ -88,11 +90,11 @@ _lib = _load()
 
 
 def make_dims(R, B, Hq, Hkv, head_dim, hidden, softmax_scale=None, pool_window=3,
-              constraints=0) -> FocusDims:
+              constraints=0, score=SCORE_DELTA) -> FocusDims:
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(head_dim)
     return FocusDims(int(R), int(B), int(Hq), int(Hkv), int(head_dim), int(hidden),
-                     float(softmax_scale), int(pool_window), int(constraints))
+                     float(softmax_scale), int(pool_window), int(constraints), int(score))
 
 
 def _ptr(t: torch.Tensor | None, dtype=None, name="tensor"):
@@ -209,13 +211,13 @@ def focus_evict(dims, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block, cu_prefi
                 decoded, budget, kept_idx, cu_seqlens, packed, ws: Workspace, delta_out=None,
                 i0_out=None, i1_out=None, stream=None):
     bf, f32 = torch.bfloat16, torch.float32
-    if k0_prefix.shape[0] != k1_prefix.shape[0]:
+    if k0_prefix is not None and k0_prefix.shape[0] != k1_prefix.shape[0]:
         raise ValueError("k0_prefix and k1_prefix must have the same number of rows")
     _ok(_lib.focus_evict(
         ctypes.byref(dims), _ptr(q0, bf, "q0"), _ptr(k0_prefix, bf, "k0_prefix"),
         _ptr(k0_block, bf, "k0_block"), _ptr(q1, bf, "q1"), _ptr(k1_prefix, bf, "k1_prefix"),
         _ptr(k1_block, bf, "k1_block"), _ptr(cu_prefix, torch.int32, "cu_prefix"),
-        int(k0_prefix.shape[0]), _ptr(hidden, bf, "hidden"),
+        int(k1_prefix.shape[0]), _ptr(hidden, bf, "hidden"),
         _ptr(decoded, torch.uint8, "decoded"), _ptr(budget, torch.int32, "budget"),
         _ptr(kept_idx, torch.int32, "kept_idx"), _ptr(cu_seqlens, torch.int32, "cu_seqlens"),
         _ptr(packed, bf, "packed"), int(packed.shape[0]),
@@ -235,13 +237,13 @@ def focus_evict_static_scratch(dims, q0, k0_prefix, k0_block, q1, k1_prefix, k1_
     `device_status` (optional int32 CUDA tensor of one element) receives the raw
     device status bits (0 = fine)."""
     bf, f32 = torch.bfloat16, torch.float32
-    if k0_prefix.shape[0] != k1_prefix.shape[0]:
+    if k0_prefix is not None and k0_prefix.shape[0] != k1_prefix.shape[0]:
         raise ValueError("k0_prefix and k1_prefix must have the same number of rows")
     _ok(_lib.focus_evict_static_scratch(
         ctypes.byref(dims), _ptr(q0, bf, "q0"), _ptr(k0_prefix, bf, "k0_prefix"),
         _ptr(k0_block, bf, "k0_block"), _ptr(q1, bf, "q1"), _ptr(k1_prefix, bf, "k1_prefix"),
         _ptr(k1_block, bf, "k1_block"), _ptr(cu_prefix, torch.int32, "cu_prefix"),
-        int(k0_prefix.shape[0]), _ptr(hidden, bf, "hidden"),
+        int(k1_prefix.shape[0]), _ptr(hidden, bf, "hidden"),
         _ptr(decoded, torch.uint8, "decoded"), _ptr(budget, torch.int32, "budget"),
         _ptr(kept_idx, torch.int32, "kept_idx"), _ptr(cu_seqlens, torch.int32, "cu_seqlens"),
         _ptr(packed, bf, "packed"), int(packed.shape[0]),

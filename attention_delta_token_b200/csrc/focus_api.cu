@@ -58,6 +58,7 @@ focus_status_t check_dims(const focus_dims_t *d) {
         return FOCUS_ERR_INVALID_ARGUMENT;
     if (!isfinite(d->softmax_scale) || d->softmax_scale < 0.f) return FOCUS_ERR_INVALID_ARGUMENT;
     if (d->constraints < 0 || d->constraints > 3) return FOCUS_ERR_INVALID_ARGUMENT;
+    if (d->score < 0 || d->score > 1) return FOCUS_ERR_INVALID_ARGUMENT;
     if (d->B > 128 || (d->head_dim != 64 && d->head_dim != 128) || d->Hq % d->Hkv != 0 ||
         d->hidden % 8 != 0 || d->pool_window % 2 == 0)
         return FOCUS_ERR_UNSUPPORTED_SHAPE;
@@ -376,7 +377,8 @@ focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void 
                            size_t workspace_bytes, void *stream) {
     FOCUS_TRY(check_dims(dims));
     const focus_dims_t &d = *dims;
-    FOCUS_TRY(check_attn_inputs(d, q0, k0_prefix, cu_prefix, total_prefix, k0_block));
+    const bool layer1_only = d.score == FOCUS_SCORE_LAYER1;
+    if (!layer1_only) FOCUS_TRY(check_attn_inputs(d, q0, k0_prefix, cu_prefix, total_prefix, k0_block));
     FOCUS_TRY(check_attn_inputs(d, q1, k1_prefix, cu_prefix, total_prefix, k1_block));
     FOCUS_TRY(check_ptr(hidden, 16));
     FOCUS_TRY(check_ptr(decoded, 1));
@@ -397,9 +399,17 @@ focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void 
 
     AttnParams p;
     memset(&p, 0, sizeof p);
-    fill_common(p, d, cu_prefix, total_prefix, ws, 2);
-    FOCUS_TRY(encode_layer(p, 0, d, q0, k0_prefix, total_prefix, k0_block));
-    FOCUS_TRY(encode_layer(p, 1, d, q1, k1_prefix, total_prefix, k1_block));
+    if (layer1_only) {  // the Figure 13 ablation: rank by I1, layer 0 is not touched
+        fill_common(p, d, cu_prefix, total_prefix, ws, 1);
+        FOCUS_TRY(encode_layer(p, 0, d, q1, k1_prefix, total_prefix, k1_block));
+        p.tm_q[1] = p.tm_q[0];
+        p.tm_kp[1] = p.tm_kp[0];
+        p.tm_kb[1] = p.tm_kb[0];
+    } else {
+        fill_common(p, d, cu_prefix, total_prefix, ws, 2);
+        FOCUS_TRY(encode_layer(p, 0, d, q0, k0_prefix, total_prefix, k0_block));
+        FOCUS_TRY(encode_layer(p, 1, d, q1, k1_prefix, total_prefix, k1_block));
+    }
 
     focus::PlanParams pp;
     memset(&pp, 0, sizeof pp);
@@ -433,6 +443,7 @@ focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void 
     sp.MT = p.MT;
     sp.H = d.hidden;
     sp.pool_window = d.pool_window;
+    sp.layers = layer1_only ? 1 : 2;
     if (d.constraints) {
         const WsLayout w = ws_layout(d);
         sp.constraints = d.constraints;

@@ -87,6 +87,7 @@ struct SelectParams {
     uint32_t *status;
     long long capacity;
     int R, B, Hkv, MT, H, pool_window;
+    int layers;                // 2: score = I1 - I0; 1: only I1 was computed (score = I1)
     // Structural constraints (constraints != 0): the retained positions of request r
     // go to lists[r*B ..] and their number to counts[r]; kept_idx/cu_seqlens are
     // written later by the scan and list-driven compaction.

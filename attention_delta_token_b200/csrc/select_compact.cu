@@ -217,15 +217,21 @@ __global__ void __launch_bounds__(256) select_compact_kernel(const SelectParams 
         if (j < B) {
             const size_t lstride = static_cast<size_t>(p.R) * p.Hkv * p.MT * B;
             float i0 = 0.f, i1 = 0.f;
-            for (int g = 0; g < p.Hkv * p.MT; ++g) {
-                const size_t idx = (rb * p.Hkv * p.MT) + static_cast<size_t>(g) * B + j;
-                i0 += p.partial[idx];
-                i1 += p.partial[lstride + idx];
+            if (p.layers == 1) {  // only the layer-1 statistics exist: score = I1
+                for (int g = 0; g < p.Hkv * p.MT; ++g)
+                    i1 += p.partial[(rb * p.Hkv * p.MT) + static_cast<size_t>(g) * B + j];
+                raw_s[j] = i1;
+            } else {
+                for (int g = 0; g < p.Hkv * p.MT; ++g) {
+                    const size_t idx = (rb * p.Hkv * p.MT) + static_cast<size_t>(g) * B + j;
+                    i0 += p.partial[idx];
+                    i1 += p.partial[lstride + idx];
+                }
+                raw_s[j] = i1 - i0;
+                if (p.i0_out) p.i0_out[rb + j] = i0;
             }
-            raw_s[j] = i1 - i0;
-            if (p.i0_out) p.i0_out[rb + j] = i0;
             if (p.i1_out) p.i1_out[rb + j] = i1;
-            if (p.raw_out) p.raw_out[rb + j] = i1 - i0;
+            if (p.raw_out) p.raw_out[rb + j] = raw_s[j];
         }
         __syncthreads();
         if (j < B) {

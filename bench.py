@@ -47,24 +47,25 @@ TRACE_EVERY = 8  # timed steps between two CUDA-event measurements of the attent
 
 # ---------------------------------------------------------------- accounting
 
-def algorithmic_counts(p) -> dict:
+def algorithmic_counts(p, layers: int = 2) -> dict:
     """Work the method must do per step (not what an implementation happens to do).
 
-    attention: both layers read every prefix and block key once (Hkv x d bf16 per
-    key) and every block query once; flops 2*d per (query row, key) per layer;
-    one exp per (query row, key) per layer.  Select/compact: the mask, budget,
-    kept indices, cu_seqlens, and the kept hidden rows read once and written once.
+    attention: each of the `layers` layers (2; 1 when ranking by I1 alone) reads
+    every prefix and block key once (Hkv x d bf16 per key) and every block query
+    once; flops 2*d per (query row, key) per layer; one exp per (query row, key)
+    per layer.  Select/compact: the mask, budget, kept indices, cu_seqlens, and the
+    kept hidden rows read once and written once.
     """
     L = p.prefix_len.astype(np.int64)
     N = L + p.B
     dec = p.decoded.cpu().numpy()
     masked = (dec == 0).sum(1).astype(np.int64)
     k = np.minimum(np.clip(p.budget.cpu().numpy().astype(np.int64), 0, None), masked)
-    attn = 2 * (N * p.Hkv * p.d * 2 + p.B * p.Hq * p.d * 2)
+    attn = layers * (N * p.Hkv * p.d * 2 + p.B * p.Hq * p.d * 2)
     rest = p.B + 4 + 4 * k + 4 + k * p.H * 2 * 2
     return dict(attn_bytes=int(attn.sum()), bytes=int(attn.sum() + rest.sum() + 4),
-                flops=int((2 * 2 * p.Hq * p.B * N * p.d).sum()),
-                exps=int((2 * p.Hq * p.B * N).sum()), decisions=int(masked.sum()),
+                flops=int((layers * 2 * p.Hq * p.B * N * p.d).sum()),
+                exps=int((layers * p.Hq * p.B * N).sum()), decisions=int(masked.sum()),
                 kept_rows=int(k.sum()), blocks=int(p.R))
 
 
@@ -210,16 +211,19 @@ def run_ours(args, rank, world, local_rank):
                                    "name": f"{cfg.name}_r{args.requests}"})
     seed = rank_seed(args.config, rank)
     p = synth.make_problem(cfg, seed=seed, device=dev)
-    counts = algorithmic_counts(p)
-    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, args.constraints)
+    counts = algorithmic_counts(p, layers=1 if args.score else 2)
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, args.constraints,
+                       args.score)
     ws = F.Workspace(dims, dev)
     cap = F.plan_capacity(p.decoded, p.budget, args.constraints)
     kept, cu, packed = make_outputs(p, cap, dev)
     stream = torch.cuda.current_stream(dev)
     in_bytes = sum(t.numel() * t.element_size() for t in p.tensors().values())
 
+    layer0 = (None, None, None) if args.score else (p.q0, p.k0_prefix, p.k0_block)
+
     def step():
-        F.focus_evict(dims, p.q0, p.k0_prefix, p.k0_block, p.q1, p.k1_prefix, p.k1_block,
+        F.focus_evict(dims, *layer0, p.q1, p.k1_prefix, p.k1_block,
                       p.cu_prefix, p.hidden, p.decoded, p.budget, kept, cu, packed, ws)
 
     def barrier():
@@ -321,13 +325,13 @@ def run_ours(args, rank, world, local_rank):
                 "input_bytes_per_step": int(in_bytes),
                 "l2": f"no flush: {in_bytes / 2**30:.2f} GiB of inputs per step > 126 MB L2",
                 "accumulate": "fp32", "parallelism": f"dp{world} (request-sharded replicas)",
-                "constraints": args.constraints,
+                "constraints": args.constraints, "score": args.score,
             },
             "decisions_per_s": world * counts["decisions"] / step_s,
             "roofline": {
                 "bound": "hbm", "kernel": "attn_stats_kernel", "achieved": achieved,
                 "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": read_traffic(workload),
+                "traffic": read_traffic(workload) if not args.score else None,
                 "algorithmic_bytes_per_launch": counts["attn_bytes"],
                 "ms_per_launch": attn_s_max * 1e3, "peak_source": f"{peak_src} (hbm_gbs)",
                 "launches_timed": len(traced),
@@ -430,6 +434,8 @@ def main():
     ap.add_argument("--constraints", type=int, default=0, choices=[0, 1, 2, 3],
                     help="structural constraints on the retained set (bit 1: predecessors, "
                          "bit 2: masked tokens left of the rightmost candidate)")
+    ap.add_argument("--score", type=int, default=0, choices=[0, 1],
+                    help="0: rank by I1 - I0 (the method); 1: by I1 alone (layer 0 skipped)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

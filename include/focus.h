@@ -33,7 +33,7 @@
  *    focus_read_device_status().
  *  - Shapes: 1 <= B <= 128; head_dim in {64, 128}; Hq % Hkv == 0 and
  *    G = Hq / Hkv divides 128; hidden % 8 == 0; pool_window odd and >= 1;
- *    R >= 1; constraints in 0..3 (else FOCUS_ERR_INVALID_ARGUMENT).  Other shapes
+ *    R >= 1; constraints in 0..3 and score in 0..1 (else FOCUS_ERR_INVALID_ARGUMENT).  Other shapes
  *    return FOCUS_ERR_UNSUPPORTED_SHAPE.
  *  - Per-request budgets are clamped to [0, masked_r] on the device, so
  *    k_r = min(max(budget[r], 0), masked_r).  Without structural constraints
@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define FOCUS_ABI_VERSION 2
+#define FOCUS_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define FOCUS_API __attribute__((visibility("default")))
@@ -85,7 +85,13 @@ typedef struct {
     int32_t constraints;   /* structural constraints on the retained set, bit mask:
                               FOCUS_KEEP_PREDECESSOR | FOCUS_KEEP_MASKED_BEFORE_RIGHTMOST;
                               0 keeps exactly the top-K candidates                   */
+    int32_t score;         /* what is pooled and ranked: FOCUS_SCORE_DELTA (I1 - I0, the
+                              method) or FOCUS_SCORE_LAYER1 (I1 alone, the Figure 13
+                              ablation: layer 0 is not computed and may be NULL)     */
 } focus_dims_t;
+
+#define FOCUS_SCORE_DELTA 0
+#define FOCUS_SCORE_LAYER1 1
 
 /*
  * Structural constraints ("What carries the argument": after the top-K candidates
@@ -184,7 +190,9 @@ FOCUS_API focus_status_t focus_compact(const focus_dims_t *dims, const void *hid
  * importance, delta, MaxPool1D, mask, top-K, compaction.  Arguments as in the
  * calls above; q0/k0_* are layer 0, q1/k1_* the layer-1 Q/K projections, both
  * layers share cu_prefix/total_prefix.  delta_out (pooled and masked), i0_out
- * and i1_out ([R, B] float32) are optional (NULL skips them).
+ * and i1_out ([R, B] float32) are optional (NULL skips them).  With
+ * dims.score == FOCUS_SCORE_LAYER1 the layer-0 arguments may be NULL, I0 is not
+ * computed (i0_out is left untouched) and delta_out holds the pooled, masked I1.
  */
 FOCUS_API focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void *k0_prefix,
                            const void *k0_block, const void *q1, const void *k1_prefix,

@@ -178,14 +178,19 @@ class Oracle:
         _check(st, "compact")
         return packed[:capacity]
 
-    def evict(self, p, constraints: int = 0) -> dict:
+    def evict(self, p, constraints: int = 0, score: int = 0) -> dict:
         """The whole step on a problem object with the fields of ``synth.FocusProblem``.
 
         Returns float64 i0, i1, delta (raw), pooled (masked) [R, B]; int32 kept
-        and cu_seqlens; uint16 packed [sum k, H].
+        and cu_seqlens; uint16 packed [sum k, H].  With ``score=1`` (rank by the
+        layer-1 importance alone) the layer-0 importance is taken as zero, so the
+        pooled score is MaxPool1D(I1).
         """
-        i0 = self.importance(p.q0, p.k0_prefix, p.cu_prefix, p.k0_block, Hq=p.Hq, Hkv=p.Hkv,
-                             scale=p.scale)
+        if score:
+            i0 = np.zeros((p.R, p.B), np.float64)
+        else:
+            i0 = self.importance(p.q0, p.k0_prefix, p.cu_prefix, p.k0_block, Hq=p.Hq,
+                                 Hkv=p.Hkv, scale=p.scale)
         i1 = self.importance(p.q1, p.k1_prefix, p.cu_prefix, p.k1_block, Hq=p.Hq, Hkv=p.Hkv,
                              scale=p.scale)
         raw, pooled = self.delta_pool_mask(i0, i1, p.decoded, window=p.pool_window)
@@ -229,8 +234,8 @@ def compact(*a, **k):
     return default().compact(*a, **k)
 
 
-def evict(p, constraints: int = 0) -> dict:
-    return default().evict(p, constraints)
+def evict(p, constraints: int = 0, score: int = 0) -> dict:
+    return default().evict(p, constraints, score)
 
 
 def select_structured(*a, **k):

@@ -18,11 +18,12 @@ RTOL = 1e-2
 TIE_TOL = 2e-3
 
 
-def run_evict(p, *, outputs=True, capacity=None, stream=None, constraints=0):
+def run_evict(p, *, outputs=True, capacity=None, stream=None, constraints=0, score=0):
     """focus_evict on a problem whose tensors live on the GPU.  Returns numpy arrays."""
     import attention_delta_token_b200 as F
-    dev = p.q0.device
-    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, constraints)
+    dev = p.q1.device
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, constraints,
+                       score)
     ws = F.Workspace(dims, dev)
     cap = F.plan_capacity(p.decoded, p.budget, constraints) if capacity is None else capacity
     kept = torch.full((max(cap, 1),), -1, dtype=torch.int32, device=dev)[:cap]
@@ -30,7 +31,8 @@ def run_evict(p, *, outputs=True, capacity=None, stream=None, constraints=0):
     packed = torch.zeros((max(cap, 1), p.H), dtype=torch.bfloat16, device=dev)[:cap]
     mk = (lambda: torch.full((p.R, p.B), float("nan"), device=dev)) if outputs else (lambda: None)
     delta, i0, i1 = mk(), mk(), mk()
-    F.focus_evict(dims, p.q0, p.k0_prefix, p.k0_block, p.q1, p.k1_prefix, p.k1_block, p.cu_prefix,
+    l0 = (None, None, None) if score else (p.q0, p.k0_prefix, p.k0_block)
+    F.focus_evict(dims, *l0, p.q1, p.k1_prefix, p.k1_block, p.cu_prefix,
                   p.hidden, p.decoded, p.budget, kept, cu, packed, ws, delta_out=delta,
                   i0_out=i0, i1_out=i1, stream=stream)
     status = F.focus_read_device_status(ws, stream)

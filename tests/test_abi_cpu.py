@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol():
 def test_status_strings_and_version():
     for code, name in F.STATUS.items():
         assert F.focus_status_string(code) == name
-    assert F.focus_abi_version() == 2
+    assert F.focus_abi_version() == 3
 
 
 def dims(**kw):
@@ -68,6 +68,7 @@ BAD_DIMS = [
     (dict(softmax_scale=-1.0), INVALID), (dict(softmax_scale=math.nan), INVALID),
     (dict(softmax_scale=math.inf), INVALID), (dict(pool_window=0), INVALID),
     (dict(constraints=4), INVALID), (dict(constraints=-1), INVALID),
+    (dict(score=2), INVALID), (dict(score=-1), INVALID),
     (dict(B=129), UNSUPPORTED), (dict(head_dim=96), UNSUPPORTED), (dict(head_dim=256), UNSUPPORTED),
     (dict(Hq=30, Hkv=8), UNSUPPORTED), (dict(Hq=24, Hkv=8), UNSUPPORTED),
     (dict(Hq=256, Hkv=1), UNSUPPORTED), (dict(hidden=4092), UNSUPPORTED),

@@ -307,3 +307,20 @@ def test_structural_full_config_sampled(orc):
                                 ref["pooled"], dec, bud)
     assert exact >= n // 2, (exact, n)
     check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))
+
+
+@pytest.mark.parametrize("case", ["sdar_r8_wide", "ragged_r10_ties", "tiny"])
+def test_layer1_score_vs_oracle(case, orc):
+    """Ranking by the layer-1 importance alone (the Figure 13 ablation): layer 0 is
+    neither passed nor computed; the pooled score is MaxPool1D(I1)."""
+    cfg, ov, wide = STRUCTURED_CASES[case]
+    p = synth.make_problem(cfg, seed=400, wide_logits=wide, overrides=ov)
+    ref = orc.evict(p, score=1)
+    out = run_evict(p.to("cuda"), score=1)
+    assert out["status"] == 0
+    assert np.isnan(out["i0"]).all()  # left untouched
+    assert_close_importance(out["i1"], ref["i1"], "I1")
+    assert_close_delta(out["delta"], ref["pooled"])
+    check_selection(out["kept"], out["cu_seqlens"], ref["pooled"], p.decoded.numpy(),
+                    p.budget.numpy())
+    check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))
