@@ -78,6 +78,8 @@ def _load() -> ctypes.CDLL:
         "focus_evict_static_scratch": (ctypes.c_int, [D, P, P, P, P, P, P, P, i64, P, P, P, P, P,
                                                       P, i64, P, P, P, P, P]),
         "focus_selftest_wait_timeout": (ctypes.c_int, [P, ctypes.c_uint64, P, P]),
+        "focus_evict_with_lse0": (ctypes.c_int, [D, P, P, P, P, P, P, P, i64, P, P, P, P, P, P,
+                                                 i64, P, P, P, P, sz, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -223,6 +225,24 @@ def focus_evict(dims, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block, cu_prefi
         _ptr(packed, bf, "packed"), int(packed.shape[0]),
         _ptr(delta_out, f32, "delta_out"), _ptr(i0_out, f32, "i0_out"),
         _ptr(i1_out, f32, "i1_out"), ws.ptr, ws.nbytes, _stream(stream)), "focus_evict")
+
+
+def focus_evict_with_lse0(dims, lse0, q0, k0_block, q1, k1_prefix, k1_block, cu_prefix, hidden,
+                          decoded, budget, kept_idx, cu_seqlens, packed, ws: Workspace,
+                          delta_out=None, i0_out=None, i1_out=None, stream=None):
+    """focus_evict with layer 0's row log-sum-exps given (lse0 [R, B, Hq] float32, natural
+    log, over each row's prefix and block keys): layer 0 reads only Q0 and its block keys."""
+    bf, f32 = torch.bfloat16, torch.float32
+    _ok(_lib.focus_evict_with_lse0(
+        ctypes.byref(dims), _ptr(lse0, f32, "lse0"), _ptr(q0, bf, "q0"),
+        _ptr(k0_block, bf, "k0_block"), _ptr(q1, bf, "q1"), _ptr(k1_prefix, bf, "k1_prefix"),
+        _ptr(k1_block, bf, "k1_block"), _ptr(cu_prefix, torch.int32, "cu_prefix"),
+        int(k1_prefix.shape[0]), _ptr(hidden, bf, "hidden"),
+        _ptr(decoded, torch.uint8, "decoded"), _ptr(budget, torch.int32, "budget"),
+        _ptr(kept_idx, torch.int32, "kept_idx"), _ptr(cu_seqlens, torch.int32, "cu_seqlens"),
+        _ptr(packed, bf, "packed"), int(packed.shape[0]),
+        _ptr(delta_out, f32, "delta_out"), _ptr(i0_out, f32, "i0_out"),
+        _ptr(i1_out, f32, "i1_out"), ws.ptr, ws.nbytes, _stream(stream)), "focus_evict_with_lse0")
 
 
 STATIC_SCRATCH_BYTES = 8 << 20

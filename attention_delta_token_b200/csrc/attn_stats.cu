@@ -74,6 +74,11 @@ __device__ __forceinline__ Item decode_item(const AttnParams &p, int it) {
     w.pstart = p.cu_prefix[w.r];
     w.L = p.cu_prefix[w.r + 1] - w.pstart;
     w.bad = w.pstart < 0 || w.L < 0 || static_cast<long long>(w.pstart) + w.L > p.total_prefix;
+    if (p.lse0 && w.layer == 0) {  // the row normalisers are given: only the block keys matter
+        w.bad = false;
+        w.L = 0;
+        w.pstart = 0;
+    }
     if (w.bad) {
         w.L = 0;
         w.pstart = 0;
@@ -396,8 +401,16 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
                         break;
                     }
                     const float2 s0 = stat[row], s1 = stat[128 + row];
-                    const float M = fmaxf(s0.x, s1.x);  // finite: half 0 always has a column
-                    const float Ltot = s0.y * ex2(s0.x - M) + s1.y * ex2(s1.x - M);
+                    float M = fmaxf(s0.x, s1.x);  // finite: half 0 always has a column
+                    float Ltot = s0.y * ex2(s0.x - M) + s1.y * ex2(s1.x - M);
+                    if (p.lse0 && w.layer == 0 && row < rows_valid) {
+                        // Given normaliser: p_ij = exp(s_ij - lse_i) = 2^(x_ij - lse_i log2 e).
+                        const int tok = w.mt * p.tok_per_tile + row / p.G;
+                        const int h = w.kvh * p.G + row % p.G;
+                        M = p.lse0[(static_cast<size_t>(w.r) * p.B + tok) * p.Hq + h] *
+                            1.4426950408889634f;
+                        Ltot = 1.f;
+                    }
                     if (nh > 0) {
                         const float scale = (row < rows_valid) ? ex2(m - M) / Ltot : 0.f;
 #pragma unroll

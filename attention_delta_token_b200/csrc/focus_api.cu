@@ -368,17 +368,29 @@ focus_status_t focus_compact(const focus_dims_t *dims, const void *hidden, const
     return FOCUS_OK;
 }
 
-focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void *k0_prefix,
-                           const void *k0_block, const void *q1, const void *k1_prefix,
-                           const void *k1_block, const int32_t *cu_prefix, int64_t total_prefix,
-                           const void *hidden, const uint8_t *decoded, const int32_t *budget,
-                           int32_t *kept_idx, int32_t *cu_seqlens, void *packed, int64_t capacity,
-                           float *delta_out, float *i0_out, float *i1_out, void *workspace,
-                           size_t workspace_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// The fused step; `lse0` (nullable) supplies layer 0's row log-sum-exps, in which
+// case layer 0 reads only Q0 and its block keys (k0_prefix is not used).
+focus_status_t evict_impl(const focus_dims_t *dims, const float *lse0, const void *q0,
+                          const void *k0_prefix, const void *k0_block, const void *q1,
+                          const void *k1_prefix, const void *k1_block, const int32_t *cu_prefix,
+                          int64_t total_prefix, const void *hidden, const uint8_t *decoded,
+                          const int32_t *budget, int32_t *kept_idx, int32_t *cu_seqlens,
+                          void *packed, int64_t capacity, float *delta_out, float *i0_out,
+                          float *i1_out, void *workspace, size_t workspace_bytes, void *stream) {
     FOCUS_TRY(check_dims(dims));
     const focus_dims_t &d = *dims;
     const bool layer1_only = d.score == FOCUS_SCORE_LAYER1;
-    if (!layer1_only) FOCUS_TRY(check_attn_inputs(d, q0, k0_prefix, cu_prefix, total_prefix, k0_block));
+    if (lse0) {
+        if (layer1_only) return FOCUS_ERR_INVALID_ARGUMENT;
+        FOCUS_TRY(check_ptr(lse0, 4));
+        FOCUS_TRY(check_attn_inputs(d, q0, nullptr, cu_prefix, 0, k0_block));
+    } else if (!layer1_only) {
+        FOCUS_TRY(check_attn_inputs(d, q0, k0_prefix, cu_prefix, total_prefix, k0_block));
+    }
     FOCUS_TRY(check_attn_inputs(d, q1, k1_prefix, cu_prefix, total_prefix, k1_block));
     FOCUS_TRY(check_ptr(hidden, 16));
     FOCUS_TRY(check_ptr(decoded, 1));
@@ -407,8 +419,12 @@ focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void 
         p.tm_kb[1] = p.tm_kb[0];
     } else {
         fill_common(p, d, cu_prefix, total_prefix, ws, 2);
-        FOCUS_TRY(encode_layer(p, 0, d, q0, k0_prefix, total_prefix, k0_block));
+        if (lse0)  // layer 0 streams no prefix: its prefix map is never read
+            FOCUS_TRY(encode_layer(p, 0, d, q0, nullptr, 0, k0_block));
+        else
+            FOCUS_TRY(encode_layer(p, 0, d, q0, k0_prefix, total_prefix, k0_block));
         FOCUS_TRY(encode_layer(p, 1, d, q1, k1_prefix, total_prefix, k1_block));
+        p.lse0 = lse0;
     }
 
     focus::PlanParams pp;
@@ -465,6 +481,37 @@ focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void 
                             d.hidden, nullptr, nullptr};
     FOCUS_CUDA(focus::launch_compact(cp, s, /*pdl=*/true));
     return FOCUS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void *k0_prefix,
+                           const void *k0_block, const void *q1, const void *k1_prefix,
+                           const void *k1_block, const int32_t *cu_prefix, int64_t total_prefix,
+                           const void *hidden, const uint8_t *decoded, const int32_t *budget,
+                           int32_t *kept_idx, int32_t *cu_seqlens, void *packed, int64_t capacity,
+                           float *delta_out, float *i0_out, float *i1_out, void *workspace,
+                           size_t workspace_bytes, void *stream) {
+    return evict_impl(dims, nullptr, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block, cu_prefix,
+                      total_prefix, hidden, decoded, budget, kept_idx, cu_seqlens, packed,
+                      capacity, delta_out, i0_out, i1_out, workspace, workspace_bytes, stream);
+}
+
+focus_status_t focus_evict_with_lse0(const focus_dims_t *dims, const float *lse0, const void *q0,
+                                     const void *k0_block, const void *q1, const void *k1_prefix,
+                                     const void *k1_block, const int32_t *cu_prefix,
+                                     int64_t total_prefix, const void *hidden,
+                                     const uint8_t *decoded, const int32_t *budget,
+                                     int32_t *kept_idx, int32_t *cu_seqlens, void *packed,
+                                     int64_t capacity, float *delta_out, float *i0_out,
+                                     float *i1_out, void *workspace, size_t workspace_bytes,
+                                     void *stream) {
+    if (!lse0) return FOCUS_ERR_INVALID_ARGUMENT;
+    return evict_impl(dims, lse0, q0, nullptr, k0_block, q1, k1_prefix, k1_block, cu_prefix,
+                      total_prefix, hidden, decoded, budget, kept_idx, cu_seqlens, packed,
+                      capacity, delta_out, i0_out, i1_out, workspace, workspace_bytes, stream);
 }
 
 const char *focus_status_string(focus_status_t st) {

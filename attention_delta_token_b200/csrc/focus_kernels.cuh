@@ -55,6 +55,8 @@ struct AttnParams {
     int tok_per_tile;          // 128 / G block tokens per row tile
     int n_blk;                 // keys in the block tile: B rounded up to 16
     float scale_log2;          // softmax_scale * log2(e)
+    const float *lse0;         // [R, B, Hq] layer-0 row log-sum-exps (natural log) or null:
+                               // given, layer-0 items read only the block keys
 };
 
 size_t attn_smem_bytes(int head_dim);

@@ -47,25 +47,32 @@ TRACE_EVERY = 8  # timed steps between two CUDA-event measurements of the attent
 
 # ---------------------------------------------------------------- accounting
 
-def algorithmic_counts(p, layers: int = 2) -> dict:
+def algorithmic_counts(p, layers: int = 2, lse0: bool = False) -> dict:
     """Work the method must do per step (not what an implementation happens to do).
 
     attention: each of the `layers` layers (2; 1 when ranking by I1 alone) reads
     every prefix and block key once (Hkv x d bf16 per key) and every block query
     once; flops 2*d per (query row, key) per layer; one exp per (query row, key)
-    per layer.  Select/compact: the mask, budget, kept indices, cu_seqlens, and the
-    kept hidden rows read once and written once.
+    per layer.  With `lse0` (layer 0's row log-sum-exps given) layer 0 reads only its
+    B block keys, Q0 and the LSEs.  Select/compact: the mask, budget, kept indices,
+    cu_seqlens, and the kept hidden rows read once and written once.
     """
     L = p.prefix_len.astype(np.int64)
     N = L + p.B
     dec = p.decoded.cpu().numpy()
     masked = (dec == 0).sum(1).astype(np.int64)
     k = np.minimum(np.clip(p.budget.cpu().numpy().astype(np.int64), 0, None), masked)
-    attn = layers * (N * p.Hkv * p.d * 2 + p.B * p.Hq * p.d * 2)
+    n0 = np.full_like(N, p.B) if lse0 else N  # keys layer 0 streams
+    attn = layers * (p.B * p.Hq * p.d * 2) + N * p.Hkv * p.d * 2
+    flops = 2 * p.Hq * p.B * N * p.d
+    exps = p.Hq * p.B * N
+    if layers == 2:
+        attn = attn + n0 * p.Hkv * p.d * 2 + (p.B * p.Hq * 4 if lse0 else 0)
+        flops = flops + 2 * p.Hq * p.B * n0 * p.d
+        exps = exps + p.Hq * p.B * n0
     rest = p.B + 4 + 4 * k + 4 + k * p.H * 2 * 2
     return dict(attn_bytes=int(attn.sum()), bytes=int(attn.sum() + rest.sum() + 4),
-                flops=int((layers * 2 * p.Hq * p.B * N * p.d).sum()),
-                exps=int((layers * p.Hq * p.B * N).sum()), decisions=int(masked.sum()),
+                flops=int(flops.sum()), exps=int(exps.sum()), decisions=int(masked.sum()),
                 kept_rows=int(k.sum()), blocks=int(p.R))
 
 
@@ -173,6 +180,23 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- our arm
 
+def layer0_row_lse(p) -> torch.Tensor:
+    """Layer-0 row log-sum-exps [R, B, Hq] over each row's prefix and block keys, in
+    float32 on the device: the input an engine's layer-0 attention forward hands over
+    (computed here with torch as setup, outside the timed region)."""
+    G = p.Hq // p.Hkv
+    cu = p.cu_prefix.cpu().numpy()
+    out = torch.empty(p.R, p.B, p.Hq, dtype=torch.float32, device=p.q0.device)
+    for r in range(p.R):
+        keys = torch.cat([p.k0_prefix[int(cu[r]):int(cu[r + 1])], p.k0_block[r]], 0).float()
+        q = p.q0[r].float()  # [B, Hq, d]
+        for g in range(p.Hkv):
+            qs = q[:, g * G:(g + 1) * G].reshape(-1, p.d)
+            s = p.scale * (qs @ keys[:, g].T)
+            out[r, :, g * G:(g + 1) * G] = torch.logsumexp(s, dim=-1).view(p.B, G)
+    return out
+
+
 def make_outputs(p, cap, dev):
     kept = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)[:cap]
     cu = torch.empty(p.R + 1, dtype=torch.int32, device=dev)
@@ -211,7 +235,7 @@ def run_ours(args, rank, world, local_rank):
                                    "name": f"{cfg.name}_r{args.requests}"})
     seed = rank_seed(args.config, rank)
     p = synth.make_problem(cfg, seed=seed, device=dev)
-    counts = algorithmic_counts(p, layers=1 if args.score else 2)
+    counts = algorithmic_counts(p, layers=1 if args.score else 2, lse0=args.lse0)
     dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, args.constraints,
                        args.score)
     ws = F.Workspace(dims, dev)
@@ -221,10 +245,18 @@ def run_ours(args, rank, world, local_rank):
     in_bytes = sum(t.numel() * t.element_size() for t in p.tensors().values())
 
     layer0 = (None, None, None) if args.score else (p.q0, p.k0_prefix, p.k0_block)
+    if args.lse0:
+        torch.backends.cuda.matmul.allow_tf32 = False
+        lse0 = layer0_row_lse(p)
 
-    def step():
-        F.focus_evict(dims, *layer0, p.q1, p.k1_prefix, p.k1_block,
-                      p.cu_prefix, p.hidden, p.decoded, p.budget, kept, cu, packed, ws)
+        def step():
+            F.focus_evict_with_lse0(dims, lse0, p.q0, p.k0_block, p.q1, p.k1_prefix, p.k1_block,
+                                    p.cu_prefix, p.hidden, p.decoded, p.budget, kept, cu,
+                                    packed, ws)
+    else:
+        def step():
+            F.focus_evict(dims, *layer0, p.q1, p.k1_prefix, p.k1_block,
+                          p.cu_prefix, p.hidden, p.decoded, p.budget, kept, cu, packed, ws)
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -267,7 +299,7 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- end to end: pinned host inputs -> device, the C-ABI call, result -> host
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not (args.score or args.lse0):  # the end-to-end path is the method's
         host = {k: v.to("cpu").pin_memory() for k, v in p.tensors().items()}
         dev_t = p.tensors()
         out_kept = torch.empty(kept.shape, dtype=kept.dtype).pin_memory()
@@ -325,13 +357,13 @@ def run_ours(args, rank, world, local_rank):
                 "input_bytes_per_step": int(in_bytes),
                 "l2": f"no flush: {in_bytes / 2**30:.2f} GiB of inputs per step > 126 MB L2",
                 "accumulate": "fp32", "parallelism": f"dp{world} (request-sharded replicas)",
-                "constraints": args.constraints, "score": args.score,
+                "constraints": args.constraints, "score": args.score, "lse0": args.lse0,
             },
             "decisions_per_s": world * counts["decisions"] / step_s,
             "roofline": {
                 "bound": "hbm", "kernel": "attn_stats_kernel", "achieved": achieved,
                 "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": read_traffic(workload) if not args.score else None,
+                "traffic": read_traffic(workload) if not (args.score or args.lse0) else None,
                 "algorithmic_bytes_per_launch": counts["attn_bytes"],
                 "ms_per_launch": attn_s_max * 1e3, "peak_source": f"{peak_src} (hbm_gbs)",
                 "launches_timed": len(traced),
@@ -436,6 +468,8 @@ def main():
                          "bit 2: masked tokens left of the rightmost candidate)")
     ap.add_argument("--score", type=int, default=0, choices=[0, 1],
                     help="0: rank by I1 - I0 (the method); 1: by I1 alone (layer 0 skipped)")
+    ap.add_argument("--lse0", action="store_true",
+                    help="layer 0's row log-sum-exps are given (focus_evict_with_lse0)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -213,6 +213,24 @@ FOCUS_API focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, c
 FOCUS_API void focus_set_trace_events(void *start_event, void *stop_event);
 
 /*
+ * The fused step when the engine already ran layer 0's attention (as FOCUS does:
+ * layer 0 runs on the whole block) and kept its row log-sum-exps:
+ *   lse0 [R, B, Hq] float32, lse0[r][i][h] = ln sum_j exp(softmax_scale * q0[r,i,h,:] . k0_j)
+ *        over request r's prefix keys and its B block keys (what an attention
+ *        forward returns alongside its output).
+ * I0[r][j] = sum over h, i of exp(softmax_scale * q0[r,i,h,:] . k0_block[r,j,h/G,:] - lse0[r][i][h]),
+ * so layer 0 reads only Q0 and its block keys: no layer-0 prefix K argument.
+ * Everything else is focus_evict's (layer 1 is computed in full).  dims.score
+ * must be FOCUS_SCORE_DELTA.
+ */
+FOCUS_API focus_status_t focus_evict_with_lse0(
+    const focus_dims_t *dims, const float *lse0, const void *q0, const void *k0_block,
+    const void *q1, const void *k1_prefix, const void *k1_block, const int32_t *cu_prefix,
+    int64_t total_prefix, const void *hidden, const uint8_t *decoded, const int32_t *budget,
+    int32_t *kept_idx, int32_t *cu_seqlens, void *packed, int64_t capacity, float *delta_out,
+    float *i0_out, float *i1_out, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * The fused step for callers that cannot allocate device memory.  (The FOCUS
  * pages have no counterpart: this is a deployment variant of focus_evict.)
  *

@@ -92,10 +92,11 @@ class Oracle:
         lib.focus_oracle_select.argtypes = [i32, i32, P, P, P, P, P, i64]
         lib.focus_oracle_compact.argtypes = [i32, i32, i32, P, P, P, P, i64]
         lib.focus_oracle_select_structured.argtypes = [i32, i32, P, P, P, i32, P, P, i64]
+        lib.focus_oracle_importance_lse.argtypes = [i32, i32, i32, i32, i32, f64, P, P, P, P]
         lib.focus_oracle_num_threads.argtypes = []
         for fn in (lib.focus_oracle_importance, lib.focus_oracle_delta, lib.focus_oracle_select,
                    lib.focus_oracle_compact, lib.focus_oracle_num_threads,
-                   lib.focus_oracle_select_structured):
+                   lib.focus_oracle_select_structured, lib.focus_oracle_importance_lse):
             fn.restype = ctypes.c_int
         self.lib = lib
 
@@ -116,6 +117,18 @@ class Oracle:
         st = self.lib.focus_oracle_importance(R, B, Hq, Hkv, d, float(scale), _p(qa), _p(kp),
                                               _p(cu), _p(kb), _p(out))
         _check(st, "importance")
+        return out
+
+    def importance_lse(self, q, k_block, lse, *, Hq: int, Hkv: int, scale: float) -> np.ndarray:
+        """I[r, j] from given row log-sum-exps lse [R, B, Hq]: only the block keys are read."""
+        qa, kb = _u16(q), _u16(k_block)
+        ls = _arr(lse, np.float64)
+        R, B, hq, d = qa.shape
+        assert hq == Hq and kb.shape == (R, B, Hkv, d) and ls.shape == (R, B, Hq)
+        out = np.zeros((R, B), np.float64)
+        st = self.lib.focus_oracle_importance_lse(R, B, Hq, Hkv, d, float(scale), _p(qa), _p(kb),
+                                                  _p(ls), _p(out))
+        _check(st, "importance_lse")
         return out
 
     def delta_pool_mask(self, i0, i1, decoded, *, window: int = 3):
@@ -178,16 +191,19 @@ class Oracle:
         _check(st, "compact")
         return packed[:capacity]
 
-    def evict(self, p, constraints: int = 0, score: int = 0) -> dict:
+    def evict(self, p, constraints: int = 0, score: int = 0, lse0=None) -> dict:
         """The whole step on a problem object with the fields of ``synth.FocusProblem``.
 
         Returns float64 i0, i1, delta (raw), pooled (masked) [R, B]; int32 kept
         and cu_seqlens; uint16 packed [sum k, H].  With ``score=1`` (rank by the
         layer-1 importance alone) the layer-0 importance is taken as zero, so the
-        pooled score is MaxPool1D(I1).
+        pooled score is MaxPool1D(I1).  With ``lse0`` ([R, B, Hq] row log-sum-exps of
+        layer 0) the layer-0 importance is taken from it (``importance_lse``).
         """
         if score:
             i0 = np.zeros((p.R, p.B), np.float64)
+        elif lse0 is not None:
+            i0 = self.importance_lse(p.q0, p.k0_block, lse0, Hq=p.Hq, Hkv=p.Hkv, scale=p.scale)
         else:
             i0 = self.importance(p.q0, p.k0_prefix, p.cu_prefix, p.k0_block, Hq=p.Hq,
                                  Hkv=p.Hkv, scale=p.scale)
@@ -234,8 +250,12 @@ def compact(*a, **k):
     return default().compact(*a, **k)
 
 
-def evict(p, constraints: int = 0, score: int = 0) -> dict:
-    return default().evict(p, constraints, score)
+def evict(p, constraints: int = 0, score: int = 0, lse0=None) -> dict:
+    return default().evict(p, constraints, score, lse0)
+
+
+def importance_lse(*a, **k):
+    return default().importance_lse(*a, **k)
 
 
 def select_structured(*a, **k):

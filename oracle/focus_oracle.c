@@ -170,6 +170,45 @@ int focus_oracle_importance(int R, int B, int Hq, int Hkv, int d, double scale,
 }
 
 /*
+ * Attention importance from a given row normaliser (the log-sum-exp an
+ * attention forward already produced for the same rows):
+ *
+ *   out[r][j] = sum over h, i of exp(scale * q[r,i,h,:] . k_block[r,j,h/G,:] - lse[r][i][h])
+ *
+ *   lse [R, B, Hq] float64, lse[r][i][h] = ln sum_j exp(s_j) over the row's keys.
+ * With the true log-sum-exp this equals focus_oracle_importance; only the B block
+ * keys are read.
+ */
+int focus_oracle_importance_lse(int R, int B, int Hq, int Hkv, int d, double scale,
+                                const uint16_t *q, const uint16_t *k_block, const double *lse,
+                                double *out)
+{
+    if (R < 0 || B <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0)
+        return ORACLE_BAD_ARGUMENT;
+    const int G = Hq / Hkv;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < R; ++r) {
+        for (int j = 0; j < B; ++j) {
+            double acc = 0.0;
+            for (int h = 0; h < Hq; ++h) {
+                const int g = h / G;
+                const uint16_t *kj = k_block + (((size_t)r * B + j) * Hkv + g) * d;
+                for (int i = 0; i < B; ++i) {
+                    const size_t row = ((size_t)r * B + i) * Hq + h;  /* query (r, i, h) */
+                    const uint16_t *qi = q + row * d;
+                    double dot = 0.0;
+                    for (int c = 0; c < d; ++c)
+                        dot += bf16_bits_to_double(qi[c]) * bf16_bits_to_double(kj[c]);
+                    acc += exp(scale * dot - lse[row]);
+                }
+            }
+            out[(size_t)r * B + j] = acc;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/*
  * Importance delta, MaxPool1D smoothing and decoded mask.
  *
  *   delta[r][j]  = i1[r][j] - i0[r][j]                          (Eq. 3)

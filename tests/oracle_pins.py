@@ -199,6 +199,42 @@ def pin_library_softmax_columns(orc):
     np.testing.assert_allclose(I, want, rtol=1e-12, atol=1e-15)
 
 
+def _true_lse(q, kp, cu, kb, Hkv, scale):
+    """Row log-sum-exps over prefix + block keys with torch float64 logsumexp."""
+    R, B, Hq, _ = q.shape
+    G = Hq // Hkv
+    out = np.zeros((R, B, Hq))
+    for r in range(R):
+        keys = torch.cat([kp[int(cu[r]):int(cu[r + 1])], kb[r]], 0).double()
+        for h in range(Hq):
+            s = scale * q[r, :, h].double() @ keys[:, h // G].T
+            out[r, :, h] = torch.logsumexp(s, dim=-1).numpy()
+    return out
+
+
+def pin_importance_lse_matches_full(orc):
+    """Given the true row log-sum-exps (torch logsumexp over prefix and block keys),
+    the block-keys-only importance equals the full one."""
+    q, kp, cu, kb = small_problem(17, R=3, B=5, Hq=4, Hkv=2, d=6, L=(0, 4, 9), std=1.0)
+    lse = _true_lse(q, kp, cu, kb, 2, 0.7)
+    full = orc.importance(q, kp, cu, kb, Hq=4, Hkv=2, scale=0.7)
+    via = orc.importance_lse(q, kb, lse, Hq=4, Hkv=2, scale=0.7)
+    np.testing.assert_allclose(via, full, rtol=1e-12, atol=1e-15)
+
+
+def pin_importance_lse_closed_form(orc):
+    """One head, one query, lse = c: I_j = exp(s_j - c), and a shift of c scales I by e^-shift."""
+    q = bf16(np.array([1.0, 2.0]).reshape(1, 2, 1, 1))
+    k = bf16(np.array([0.5, -1.0]).reshape(1, 2, 1, 1))
+    lse = np.zeros((1, 2, 1))
+    got = orc.importance_lse(q, k, lse, Hq=1, Hkv=1, scale=1.0)
+    # column j sums over the two queries i: exp(q_i * k_j)
+    want = [math.exp(0.5) + math.exp(1.0), math.exp(-1.0) + math.exp(-2.0)]
+    np.testing.assert_allclose(got[0], want, rtol=1e-14)
+    got2 = orc.importance_lse(q, k, lse + 0.75, Hq=1, Hkv=1, scale=1.0)
+    np.testing.assert_allclose(got2, got * math.exp(-0.75), rtol=1e-14)
+
+
 # --------------------------------------------------------------------------- delta / pool / mask
 
 def pin_delta_sign_and_pool(orc):
@@ -381,5 +417,6 @@ PINS = [
     pin_heads_sum, pin_requests_independent, pin_library_softmax_columns,
     pin_delta_sign_and_pool, pin_pool_spreads_decoded_neighbour, pin_topk_lexsort,
     pin_topk_bruteforce, pin_capacity_status, pin_compact_fancy_indexing, pin_hand_evict,
-    pin_hand_structural, pin_structural_properties,
+    pin_hand_structural, pin_structural_properties, pin_importance_lse_matches_full,
+    pin_importance_lse_closed_form,
 ]

@@ -141,6 +141,20 @@ def test_other_entry_points_check_pointers():
     assert L.focus_clear_device_status(None, 1024, None) == WORKSPACE
 
 
+def test_lse0_entry_point_validation():
+    d = dims()
+    ws = F.focus_workspace_size(d)
+    L = F._lib
+    args = lambda lse, dd: (ctypes.byref(dd), lse, A, A, A, A, A, A, 100, A, A, A, A, A, A, 16,
+                            None, None, None, A, ws, None)
+    assert L.focus_evict_with_lse0(*args(None, d)) == INVALID         # lse0 required
+    assert L.focus_evict_with_lse0(*args(A + 2, d)) == INVALID        # misaligned
+    d1 = dims(score=1)
+    assert L.focus_evict_with_lse0(*args(A, d1)) == INVALID           # I1-only ranking has no layer 0
+    assert L.focus_evict_with_lse0(ctypes.byref(d), A, None, A, A, A, A, A, 100, A, A, A, A, A, A,
+                                   16, None, None, None, A, ws, None) == INVALID  # q0 missing
+
+
 def test_plan_capacity_bounds_structured_counts():
     """With structural constraints plan_capacity is an upper bound of the retained rows."""
     import oracle

@@ -324,3 +324,53 @@ def test_layer1_score_vs_oracle(case, orc):
     check_selection(out["kept"], out["cu_seqlens"], ref["pooled"], p.decoded.numpy(),
                     p.budget.numpy())
     check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))
+
+
+def _row_lse(p, device="cpu"):
+    """Layer-0 row log-sum-exps over each row's prefix and block keys (torch float64):
+    the input an engine's layer-0 attention forward would hand over."""
+    G = p.Hq // p.Hkv
+    cu = p.cu_prefix.cpu().numpy()
+    out = torch.zeros(p.R, p.B, p.Hq, dtype=torch.float64)
+    for r in range(p.R):
+        keys = torch.cat([p.k0_prefix[int(cu[r]):int(cu[r + 1])].cpu(), p.k0_block[r].cpu()], 0)
+        for h in range(p.Hq):
+            s = p.scale * p.q0[r, :, h].cpu().double() @ keys[:, h // G].double().T
+            out[r, :, h] = torch.logsumexp(s, dim=-1)
+    return out
+
+
+@pytest.mark.parametrize("case", ["sdar_r8_wide", "ragged_r10_ties", "block128_r3", "tiny"])
+def test_evict_with_lse0_vs_oracle(case, orc):
+    """Layer 0 from the engine's row log-sum-exps: only Q0 and the block keys are read;
+    the result matches the oracle's importance-from-LSE and, the LSE being the true one,
+    the full computation."""
+    import attention_delta_token_b200 as F
+    cfg, ov, wide = STRUCTURED_CASES[case]
+    p = synth.make_problem(cfg, seed=500, wide_logits=wide, overrides=ov)
+    lse = _row_lse(p).float()
+    g = p.to("cuda")
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+    ws = F.Workspace(dims)
+    cap = F.plan_capacity(p.decoded, p.budget)
+    kept = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+    packed = torch.zeros(cap, p.H, dtype=torch.bfloat16, device="cuda")
+    delta = torch.empty(p.R, p.B, device="cuda")
+    i0 = torch.empty_like(delta)
+    i1 = torch.empty_like(delta)
+    F.focus_evict_with_lse0(dims, lse.cuda(), g.q0, g.k0_block, g.q1, g.k1_prefix, g.k1_block,
+                            g.cu_prefix, g.hidden, g.decoded, g.budget, kept, cu, packed, ws,
+                            delta_out=delta, i0_out=i0, i1_out=i1)
+    assert F.focus_read_device_status(ws) == 0
+    ref = orc.evict(p, lse0=lse.double().numpy())
+    full = orc.evict(p)
+    assert_close_importance(i0.cpu().numpy(), ref["i0"], "I0 from lse")
+    assert_close_importance(i0.cpu().numpy(), full["i0"], "I0 vs full")
+    assert_close_importance(i1.cpu().numpy(), ref["i1"], "I1")
+    assert_close_delta(delta.cpu().numpy(), ref["pooled"])
+    np.testing.assert_array_equal(cu.cpu().numpy(), ref["cu_seqlens"])
+    check_selection(kept.cpu().numpy(), cu.cpu().numpy(), ref["pooled"], p.decoded.numpy(),
+                    p.budget.numpy())
+    check_packed(packed.view(torch.int16).cpu().numpy().view(np.uint16), kept.cpu().numpy(),
+                 cu.cpu().numpy(), hidden_bits(p))

@@ -37,6 +37,9 @@ MUTATIONS = {
     "rightmost_rule_keeps_decoded": ("                if (decoded[(size_t)r * B + j] == 0)\n                    keep[j] = 1;",
                                      "                keep[j] = 1;"),
     "rightmost_rule_uses_leftmost": ("            if (cand[t] > rightmost)", "            if (rightmost < 0 || cand[t] < rightmost)"),
+    "lse_sign": ("acc += exp(scale * dot - lse[row]);", "acc += exp(scale * dot + lse[row]);"),
+    "lse_wrong_head_index": ("const size_t row = ((size_t)r * B + i) * Hq + h;",
+                             "const size_t row = ((size_t)r * B + i) * Hq + g;"),
 }
 
 
