@@ -80,6 +80,9 @@ def _load() -> ctypes.CDLL:
         "focus_selftest_wait_timeout": (ctypes.c_int, [P, ctypes.c_uint64, P, P]),
         "focus_evict_with_lse0": (ctypes.c_int, [D, P, P, P, P, P, P, P, i64, P, P, P, P, P, P,
                                                  i64, P, P, P, P, sz, P]),
+        "focus_evict_paged": (ctypes.c_int, [D, P, P, P, P, P, P, P, ctypes.c_int32, P,
+                                             ctypes.c_int32, ctypes.c_int32, P, P, P, P, P, P, i64,
+                                             P, P, P, P, sz, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -243,6 +246,27 @@ def focus_evict_with_lse0(dims, lse0, q0, k0_block, q1, k1_prefix, k1_block, cu_
         _ptr(packed, bf, "packed"), int(packed.shape[0]),
         _ptr(delta_out, f32, "delta_out"), _ptr(i0_out, f32, "i0_out"),
         _ptr(i1_out, f32, "i1_out"), ws.ptr, ws.nbytes, _stream(stream)), "focus_evict_with_lse0")
+
+
+def focus_evict_paged(dims, q0, k0_pages, k0_block, q1, k1_pages, k1_block, page_table,
+                      prefix_len, hidden, decoded, budget, kept_idx, cu_seqlens, packed,
+                      ws: Workspace, delta_out=None, i0_out=None, i1_out=None, stream=None):
+    """focus_evict with the prefix keys in page pools k*_pages [num_pages, page_size, Hkv, d]
+    addressed through page_table [R, max_pages] int32 and prefix_len [R] int32."""
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    if k0_pages.shape != k1_pages.shape:
+        raise ValueError("both layers' page pools must have the same shape")
+    _ok(_lib.focus_evict_paged(
+        ctypes.byref(dims), _ptr(q0, bf, "q0"), _ptr(k0_pages, bf, "k0_pages"),
+        _ptr(k0_block, bf, "k0_block"), _ptr(q1, bf, "q1"), _ptr(k1_pages, bf, "k1_pages"),
+        _ptr(k1_block, bf, "k1_block"), _ptr(page_table, i32, "page_table"),
+        int(page_table.shape[1]), _ptr(prefix_len, i32, "prefix_len"), int(k0_pages.shape[0]),
+        int(k0_pages.shape[1]), _ptr(hidden, bf, "hidden"),
+        _ptr(decoded, torch.uint8, "decoded"), _ptr(budget, i32, "budget"),
+        _ptr(kept_idx, i32, "kept_idx"), _ptr(cu_seqlens, i32, "cu_seqlens"),
+        _ptr(packed, bf, "packed"), int(packed.shape[0]),
+        _ptr(delta_out, f32, "delta_out"), _ptr(i0_out, f32, "i0_out"),
+        _ptr(i1_out, f32, "i1_out"), ws.ptr, ws.nbytes, _stream(stream)), "focus_evict_paged")
 
 
 STATIC_SCRATCH_BYTES = 8 << 20

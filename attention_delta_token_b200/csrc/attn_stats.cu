@@ -71,9 +71,15 @@ __device__ __forceinline__ Item decode_item(const AttnParams &p, int it) {
     w.kvh = rem / p.MT;
     w.mt = rem - w.kvh * p.MT;
     w.r = p.order ? p.order[rank] : rank;
-    w.pstart = p.cu_prefix[w.r];
-    w.L = p.cu_prefix[w.r + 1] - w.pstart;
-    w.bad = w.pstart < 0 || w.L < 0 || static_cast<long long>(w.pstart) + w.L > p.total_prefix;
+    if (p.page_table) {
+        w.pstart = 0;
+        w.L = p.prefix_len[w.r];
+        w.bad = w.L < 0 || static_cast<long long>(w.L) > static_cast<long long>(p.max_pages) * p.page_size;
+    } else {
+        w.pstart = p.cu_prefix[w.r];
+        w.L = p.cu_prefix[w.r + 1] - w.pstart;
+        w.bad = w.pstart < 0 || w.L < 0 || static_cast<long long>(w.pstart) + w.L > p.total_prefix;
+    }
     if (p.lse0 && w.layer == 0) {  // the row normalisers are given: only the block keys matter
         w.bad = false;
         w.L = 0;
@@ -220,7 +226,27 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
                         break;
                     }
                     uint8_t *dst = sK + s * S::kTileBytes;
-                    if (t < w.n_pre) {
+                    if (t < w.n_pre && p.page_table) {
+                        // The tile's keys come from page_rows-row boxes of consecutive pages;
+                        // boxes past the prefix are not loaded (their columns are masked).
+                        const int first = t * kTileKeys;
+                        const int nbox = min(kTileKeys, w.L - first + p.page_rows - 1) / p.page_rows;
+                        mbar_arrive_expect_tx(&full[s], nbox * p.page_rows * 128 * S::kChunks);
+                        for (int u = 0; u < nbox; ++u) {
+                            const int key = first + u * p.page_rows;
+                            int page = p.page_table[static_cast<size_t>(w.r) * p.max_pages +
+                                                    key / p.page_size];
+                            if (page < 0 || page >= p.num_pages) {
+                                atomicOr(p.status, FOCUS_DEV_BAD_INPUT);
+                                page = 0;  // keep the copy in bounds; the result is flagged
+                            }
+                            const int row = page * p.page_size + key % p.page_size;
+#pragma unroll
+                            for (int c = 0; c < S::kChunks; ++c)
+                                tma_load_3d(dst + c * kChunkBytes + u * p.page_rows * 128,
+                                            &p.tm_kp[w.layer], &full[s], c * 64, w.kvh, row, pol);
+                        }
+                    } else if (t < w.n_pre) {
                         mbar_arrive_expect_tx(&full[s], S::kTileBytes);
 #pragma unroll
                         for (int c = 0; c < S::kChunks; ++c)

@@ -142,16 +142,18 @@ focus_status_t encode_rows_heads_d(CUtensorMap *tm, const void *base, long long 
     return r == CUDA_SUCCESS ? FOCUS_OK : FOCUS_ERR_CUDA;
 }
 
-// Fills the tensor maps of one layer.
+// Fills the tensor maps of one layer.  The prefix map views `total_prefix` rows of
+// k_prefix (a packed prefix buffer or a page pool) in boxes of `prefix_box_rows`.
 focus_status_t encode_layer(AttnParams &p, int layer, const focus_dims_t &d, const void *q,
-                            const void *k_prefix, long long total_prefix, const void *k_block) {
+                            const void *k_prefix, long long total_prefix, const void *k_block,
+                            int prefix_box_rows = focus::kTileKeys) {
     const int G = d.Hq / d.Hkv;
     const long long rb = static_cast<long long>(d.R) * d.B;
     FOCUS_TRY(encode_rows_heads_d(&p.tm_q[layer], q, rb, d.Hq, d.head_dim, G, focus::kTileRows / G));
     // With no prefix rows anywhere the prefix map is never read; point it at the block keys.
     if (total_prefix > 0)
         FOCUS_TRY(encode_rows_heads_d(&p.tm_kp[layer], k_prefix, total_prefix, d.Hkv, d.head_dim, 1,
-                                      focus::kTileKeys));
+                                      prefix_box_rows));
     else
         FOCUS_TRY(encode_rows_heads_d(&p.tm_kp[layer], k_block, rb, d.Hkv, d.head_dim, 1,
                                       focus::kTileKeys));
@@ -374,16 +376,42 @@ namespace {
 
 // The fused step; `lse0` (nullable) supplies layer 0's row log-sum-exps, in which
 // case layer 0 reads only Q0 and its block keys (k0_prefix is not used).
-focus_status_t evict_impl(const focus_dims_t *dims, const float *lse0, const void *q0,
-                          const void *k0_prefix, const void *k0_block, const void *q1,
-                          const void *k1_prefix, const void *k1_block, const int32_t *cu_prefix,
-                          int64_t total_prefix, const void *hidden, const uint8_t *decoded,
-                          const int32_t *budget, int32_t *kept_idx, int32_t *cu_seqlens,
-                          void *packed, int64_t capacity, float *delta_out, float *i0_out,
-                          float *i1_out, void *workspace, size_t workspace_bytes, void *stream) {
+// Paged prefix keys: k*_prefix point at page pools [num_pages, page_size, Hkv, d].
+struct Paging {
+    const int32_t *page_table;  // [R, max_pages]
+    const int32_t *prefix_len;  // [R]
+    int max_pages, num_pages, page_size;
+};
+
+focus_status_t check_paging(const Paging &pg) {
+    FOCUS_TRY(check_ptr(pg.page_table, 4));
+    FOCUS_TRY(check_ptr(pg.prefix_len, 4));
+    if (pg.max_pages < 1 || pg.num_pages < 1) return FOCUS_ERR_INVALID_ARGUMENT;
+    if (pg.page_size < 8 || pg.page_size > (1 << 16) || (pg.page_size & (pg.page_size - 1)))
+        return FOCUS_ERR_UNSUPPORTED_SHAPE;
+    if (static_cast<long long>(pg.num_pages) * pg.page_size > 0x7fffffffll)
+        return FOCUS_ERR_UNSUPPORTED_SHAPE;
+    return FOCUS_OK;
+}
+
+focus_status_t evict_impl(const focus_dims_t *dims, const float *lse0, const Paging *paging,
+                          const void *q0, const void *k0_prefix, const void *k0_block,
+                          const void *q1, const void *k1_prefix, const void *k1_block,
+                          const int32_t *cu_prefix, int64_t total_prefix, const void *hidden,
+                          const uint8_t *decoded, const int32_t *budget, int32_t *kept_idx,
+                          int32_t *cu_seqlens, void *packed, int64_t capacity, float *delta_out,
+                          float *i0_out, float *i1_out, void *workspace, size_t workspace_bytes,
+                          void *stream) {
     FOCUS_TRY(check_dims(dims));
     const focus_dims_t &d = *dims;
     const bool layer1_only = d.score == FOCUS_SCORE_LAYER1;
+    int prefix_box = focus::kTileKeys;
+    if (paging) {  // the page pools stand in for the packed prefix buffers
+        FOCUS_TRY(check_paging(*paging));
+        total_prefix = static_cast<long long>(paging->num_pages) * paging->page_size;
+        prefix_box = paging->page_size < focus::kTileKeys ? paging->page_size : focus::kTileKeys;
+        cu_prefix = paging->prefix_len;  // only checked for presence below; lengths come from here
+    }
     if (lse0) {
         if (layer1_only) return FOCUS_ERR_INVALID_ARGUMENT;
         FOCUS_TRY(check_ptr(lse0, 4));
@@ -413,7 +441,7 @@ focus_status_t evict_impl(const focus_dims_t *dims, const float *lse0, const voi
     memset(&p, 0, sizeof p);
     if (layer1_only) {  // the Figure 13 ablation: rank by I1, layer 0 is not touched
         fill_common(p, d, cu_prefix, total_prefix, ws, 1);
-        FOCUS_TRY(encode_layer(p, 0, d, q1, k1_prefix, total_prefix, k1_block));
+        FOCUS_TRY(encode_layer(p, 0, d, q1, k1_prefix, total_prefix, k1_block, prefix_box));
         p.tm_q[1] = p.tm_q[0];
         p.tm_kp[1] = p.tm_kp[0];
         p.tm_kb[1] = p.tm_kb[0];
@@ -422,14 +450,24 @@ focus_status_t evict_impl(const focus_dims_t *dims, const float *lse0, const voi
         if (lse0)  // layer 0 streams no prefix: its prefix map is never read
             FOCUS_TRY(encode_layer(p, 0, d, q0, nullptr, 0, k0_block));
         else
-            FOCUS_TRY(encode_layer(p, 0, d, q0, k0_prefix, total_prefix, k0_block));
-        FOCUS_TRY(encode_layer(p, 1, d, q1, k1_prefix, total_prefix, k1_block));
+            FOCUS_TRY(encode_layer(p, 0, d, q0, k0_prefix, total_prefix, k0_block, prefix_box));
+        FOCUS_TRY(encode_layer(p, 1, d, q1, k1_prefix, total_prefix, k1_block, prefix_box));
         p.lse0 = lse0;
+    }
+    if (paging) {
+        p.cu_prefix = nullptr;
+        p.page_table = paging->page_table;
+        p.prefix_len = paging->prefix_len;
+        p.page_size = paging->page_size;
+        p.max_pages = paging->max_pages;
+        p.num_pages = paging->num_pages;
+        p.page_rows = prefix_box;
     }
 
     focus::PlanParams pp;
     memset(&pp, 0, sizeof pp);
-    pp.cu_prefix = cu_prefix;
+    pp.cu_prefix = paging ? nullptr : cu_prefix;
+    pp.prefix_len = paging ? paging->prefix_len : nullptr;
     pp.decoded = decoded;
     pp.budget = budget;
     pp.order = const_cast<int32_t *>(p.order);
@@ -494,7 +532,8 @@ focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void 
                            int32_t *kept_idx, int32_t *cu_seqlens, void *packed, int64_t capacity,
                            float *delta_out, float *i0_out, float *i1_out, void *workspace,
                            size_t workspace_bytes, void *stream) {
-    return evict_impl(dims, nullptr, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block, cu_prefix,
+    return evict_impl(dims, nullptr, nullptr, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block,
+                      cu_prefix,
                       total_prefix, hidden, decoded, budget, kept_idx, cu_seqlens, packed,
                       capacity, delta_out, i0_out, i1_out, workspace, workspace_bytes, stream);
 }
@@ -509,9 +548,25 @@ focus_status_t focus_evict_with_lse0(const focus_dims_t *dims, const float *lse0
                                      float *i1_out, void *workspace, size_t workspace_bytes,
                                      void *stream) {
     if (!lse0) return FOCUS_ERR_INVALID_ARGUMENT;
-    return evict_impl(dims, lse0, q0, nullptr, k0_block, q1, k1_prefix, k1_block, cu_prefix,
+    return evict_impl(dims, lse0, nullptr, q0, nullptr, k0_block, q1, k1_prefix, k1_block,
+                      cu_prefix,
                       total_prefix, hidden, decoded, budget, kept_idx, cu_seqlens, packed,
                       capacity, delta_out, i0_out, i1_out, workspace, workspace_bytes, stream);
+}
+
+focus_status_t focus_evict_paged(const focus_dims_t *dims, const void *q0, const void *k0_pages,
+                                 const void *k0_block, const void *q1, const void *k1_pages,
+                                 const void *k1_block, const int32_t *page_table, int32_t max_pages,
+                                 const int32_t *prefix_len, int32_t num_pages, int32_t page_size,
+                                 const void *hidden, const uint8_t *decoded,
+                                 const int32_t *budget, int32_t *kept_idx, int32_t *cu_seqlens,
+                                 void *packed, int64_t capacity, float *delta_out, float *i0_out,
+                                 float *i1_out, void *workspace, size_t workspace_bytes,
+                                 void *stream) {
+    const Paging pg{page_table, prefix_len, max_pages, num_pages, page_size};
+    return evict_impl(dims, nullptr, &pg, q0, k0_pages, k0_block, q1, k1_pages, k1_block, nullptr,
+                      0, hidden, decoded, budget, kept_idx, cu_seqlens, packed, capacity,
+                      delta_out, i0_out, i1_out, workspace, workspace_bytes, stream);
 }
 
 const char *focus_status_string(focus_status_t st) {

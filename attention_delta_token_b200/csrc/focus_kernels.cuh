@@ -57,6 +57,12 @@ struct AttnParams {
     float scale_log2;          // softmax_scale * log2(e)
     const float *lse0;         // [R, B, Hq] layer-0 row log-sum-exps (natural log) or null:
                                // given, layer-0 items read only the block keys
+    // Paged prefix keys (page_table != null): prefix key t of request r is row
+    // page_table[r * max_pages + t / page_size] * page_size + t % page_size of the
+    // page pool that tm_kp views ([num_pages * page_size, Hkv, d], box rows page_rows).
+    const int32_t *page_table;  // [R, max_pages]
+    const int32_t *prefix_len;  // [R]
+    int page_size, max_pages, num_pages, page_rows;
 };
 
 size_t attn_smem_bytes(int head_dim);
@@ -65,7 +71,8 @@ cudaError_t launch_attn_stats(const AttnParams &p, int head_dim, cudaStream_t st
 
 // ---------------------------------------------------------------- planning
 struct PlanParams {
-    const int32_t *cu_prefix;  // [R+1]
+    const int32_t *cu_prefix;  // [R+1] (packed prefix) or null
+    const int32_t *prefix_len; // [R] (paged prefix) or null
     const uint8_t *decoded;    // [R,B] or null (no counts)
     const int32_t *budget;     // [R]   or null
     int32_t *order;            // [R]   or null (no ordering)

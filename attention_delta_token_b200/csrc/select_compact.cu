@@ -47,6 +47,11 @@ __device__ __forceinline__ int kept_count(const uint8_t *decoded, const int32_t 
     return min(max(budget[r], 0), masked_count(decoded, r, B));
 }
 
+// Prefix length of request r: from the paged lengths or the packed offsets.
+__device__ __forceinline__ int prefix_length(const PlanParams &p, int r) {
+    return p.prefix_len ? p.prefix_len[r] : p.cu_prefix[r + 1] - p.cu_prefix[r];
+}
+
 // Exclusive block-wide scan of one int per thread (kPlanThreads threads).
 __device__ __forceinline__ int block_exclusive_scan(int x, int *warp_tot, int &total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -89,7 +94,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
     if (p.order && R <= kRankSortR) {
         // Rank of each request under (L desc, r asc): a plain count, no sort passes.
         for (int i = threadIdx.x; i < R; i += blockDim.x) {
-            const int L = max(p.cu_prefix[i + 1] - p.cu_prefix[i], 0);
+            const int L = max(prefix_length(p, i), 0);
             keys[i] = (static_cast<unsigned long long>(0x7fffffffu - static_cast<uint32_t>(L)) << 32) |
                       static_cast<uint32_t>(i);
         }
@@ -107,8 +112,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
             for (int i = threadIdx.x; i < n; i += blockDim.x) {
                 unsigned long long key = ~0ull;
                 if (i < R) {
-                    int L = p.cu_prefix[i + 1] - p.cu_prefix[i];
-                    L = max(L, 0);
+                    const int L = max(prefix_length(p, i), 0);
                     key = (static_cast<unsigned long long>(0x7fffffffu - static_cast<uint32_t>(L)) << 32) |
                           static_cast<uint32_t>(i);
                 }

@@ -245,7 +245,14 @@ def run_ours(args, rank, world, local_rank):
     in_bytes = sum(t.numel() * t.element_size() for t in p.tensors().values())
 
     layer0 = (None, None, None) if args.score else (p.q0, p.k0_prefix, p.k0_block)
-    if args.lse0:
+    if args.page_size:
+        pg = synth.to_paged(p, args.page_size, seed=seed)
+
+        def step():
+            F.focus_evict_paged(dims, p.q0, pg.k0_pages, p.k0_block, p.q1, pg.k1_pages, p.k1_block,
+                                pg.page_table, pg.prefix_len, p.hidden, p.decoded, p.budget, kept,
+                                cu, packed, ws)
+    elif args.lse0:
         torch.backends.cuda.matmul.allow_tf32 = False
         lse0 = layer0_row_lse(p)
 
@@ -299,7 +306,7 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- end to end: pinned host inputs -> device, the C-ABI call, result -> host
     e2e = None
-    if not args.no_e2e and not (args.score or args.lse0):  # the end-to-end path is the method's
+    if not args.no_e2e and not (args.score or args.lse0 or args.page_size):  # the default path
         host = {k: v.to("cpu").pin_memory() for k, v in p.tensors().items()}
         dev_t = p.tensors()
         out_kept = torch.empty(kept.shape, dtype=kept.dtype).pin_memory()
@@ -358,12 +365,14 @@ def run_ours(args, rank, world, local_rank):
                 "l2": f"no flush: {in_bytes / 2**30:.2f} GiB of inputs per step > 126 MB L2",
                 "accumulate": "fp32", "parallelism": f"dp{world} (request-sharded replicas)",
                 "constraints": args.constraints, "score": args.score, "lse0": args.lse0,
+                "page_size": args.page_size,
             },
             "decisions_per_s": world * counts["decisions"] / step_s,
             "roofline": {
                 "bound": "hbm", "kernel": "attn_stats_kernel", "achieved": achieved,
                 "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": read_traffic(workload) if not (args.score or args.lse0) else None,
+                "traffic": (read_traffic(workload)
+                            if not (args.score or args.lse0 or args.page_size) else None),
                 "algorithmic_bytes_per_launch": counts["attn_bytes"],
                 "ms_per_launch": attn_s_max * 1e3, "peak_source": f"{peak_src} (hbm_gbs)",
                 "launches_timed": len(traced),
@@ -470,6 +479,9 @@ def main():
                     help="0: rank by I1 - I0 (the method); 1: by I1 alone (layer 0 skipped)")
     ap.add_argument("--lse0", action="store_true",
                     help="layer 0's row log-sum-exps are given (focus_evict_with_lse0)")
+    ap.add_argument("--page-size", type=int, default=0,
+                    help="read the prefix keys from a paged pool with pages of this many tokens "
+                         "(focus_evict_paged)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

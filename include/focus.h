@@ -213,6 +213,27 @@ FOCUS_API focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, c
 FOCUS_API void focus_set_trace_events(void *start_event, void *stop_event);
 
 /*
+ * The fused step with the prefix keys in a paged KV cache (pages of page_size
+ * tokens, each request owning an ordered list of pages, the same list for both
+ * layers), read in place:
+ *   k0_pages, k1_pages [num_pages, page_size, Hkv, d] bf16 (16-byte aligned)
+ *   page_table [R, max_pages] int32: request r's prefix key t is row
+ *              t % page_size of page page_table[r][t / page_size]
+ *   prefix_len [R] int32: prefix length of each request (0 <= L_r <= max_pages * page_size)
+ *   page_size: a power of two, 8 .. 65536.  Pages shorter than 128 tokens are
+ *              gathered several per 128-key tile.
+ * Everything else is focus_evict's.  A page index outside [0, num_pages) sets
+ * FOCUS_ERR_DEVICE_CHECK in the device status (page 0 is read instead).
+ */
+FOCUS_API focus_status_t focus_evict_paged(
+    const focus_dims_t *dims, const void *q0, const void *k0_pages, const void *k0_block,
+    const void *q1, const void *k1_pages, const void *k1_block, const int32_t *page_table,
+    int32_t max_pages, const int32_t *prefix_len, int32_t num_pages, int32_t page_size,
+    const void *hidden, const uint8_t *decoded, const int32_t *budget, int32_t *kept_idx,
+    int32_t *cu_seqlens, void *packed, int64_t capacity, float *delta_out, float *i0_out,
+    float *i1_out, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * The fused step when the engine already ran layer 0's attention (as FOCUS does:
  * layer 0 runs on the whole block) and kept its row log-sum-exps:
  *   lse0 [R, B, Hq] float32, lse0[r][i][h] = ln sum_j exp(softmax_scale * q0[r,i,h,:] . k0_j)

@@ -93,10 +93,13 @@ class Oracle:
         lib.focus_oracle_compact.argtypes = [i32, i32, i32, P, P, P, P, i64]
         lib.focus_oracle_select_structured.argtypes = [i32, i32, P, P, P, i32, P, P, i64]
         lib.focus_oracle_importance_lse.argtypes = [i32, i32, i32, i32, i32, f64, P, P, P, P]
+        lib.focus_oracle_importance_paged.argtypes = [i32, i32, i32, i32, i32, f64, P, P, P, i32,
+                                                      P, i32, i32, P, P]
         lib.focus_oracle_num_threads.argtypes = []
         for fn in (lib.focus_oracle_importance, lib.focus_oracle_delta, lib.focus_oracle_select,
                    lib.focus_oracle_compact, lib.focus_oracle_num_threads,
-                   lib.focus_oracle_select_structured, lib.focus_oracle_importance_lse):
+                   lib.focus_oracle_select_structured, lib.focus_oracle_importance_lse,
+                   lib.focus_oracle_importance_paged):
             fn.restype = ctypes.c_int
         self.lib = lib
 
@@ -117,6 +120,23 @@ class Oracle:
         st = self.lib.focus_oracle_importance(R, B, Hq, Hkv, d, float(scale), _p(qa), _p(kp),
                                               _p(cu), _p(kb), _p(out))
         _check(st, "importance")
+        return out
+
+    def importance_paged(self, q, k_pages, page_table, prefix_len, k_block, *, Hq: int, Hkv: int,
+                         scale: float) -> np.ndarray:
+        """I[r, j] with the prefix keys in a page pool k_pages [num_pages, page_size, Hkv, d]
+        addressed through page_table [R, max_pages] and prefix_len [R]."""
+        qa, kp, kb = _u16(q), _u16(k_pages), _u16(k_block)
+        pt = _arr(page_table, np.int32)
+        pl = _arr(prefix_len, np.int32)
+        R, B, hq, d = qa.shape
+        num_pages, page_size = kp.shape[0], kp.shape[1]
+        assert hq == Hq and kb.shape == (R, B, Hkv, d) and pt.shape[0] == R and pl.shape == (R,)
+        out = np.zeros((R, B), np.float64)
+        st = self.lib.focus_oracle_importance_paged(R, B, Hq, Hkv, d, float(scale), _p(qa), _p(kp),
+                                                    _p(pt), pt.shape[1], _p(pl), page_size,
+                                                    num_pages, _p(kb), _p(out))
+        _check(st, "importance_paged")
         return out
 
     def importance_lse(self, q, k_block, lse, *, Hq: int, Hkv: int, scale: float) -> np.ndarray:
@@ -256,6 +276,10 @@ def evict(p, constraints: int = 0, score: int = 0, lse0=None) -> dict:
 
 def importance_lse(*a, **k):
     return default().importance_lse(*a, **k)
+
+
+def importance_paged(*a, **k):
+    return default().importance_paged(*a, **k)
 
 
 def select_structured(*a, **k):

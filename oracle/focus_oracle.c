@@ -170,6 +170,102 @@ int focus_oracle_importance(int R, int B, int Hq, int Hkv, int d, double scale,
 }
 
 /*
+ * Attention importance with the prefix keys in a paged pool (a KV cache laid out
+ * as pages of page_size tokens, each request owning an ordered list of pages):
+ *
+ *   prefix key t of request r = k_pages[page_table[r][t / page_size]][t % page_size][g][:]
+ *   k_pages    [num_pages, page_size, Hkv, d] bf16 bits
+ *   page_table [R, max_pages] int32;  prefix_len [R] int32
+ *
+ * Otherwise exactly focus_oracle_importance (prefix keys, then block keys).
+ */
+int focus_oracle_importance_paged(int R, int B, int Hq, int Hkv, int d, double scale,
+                                  const uint16_t *q, const uint16_t *k_pages,
+                                  const int32_t *page_table, int max_pages,
+                                  const int32_t *prefix_len, int page_size, int num_pages,
+                                  const uint16_t *k_block, double *out)
+{
+    if (R < 0 || B <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0 || page_size <= 0)
+        return ORACLE_BAD_ARGUMENT;
+    for (int r = 0; r < R; ++r) {
+        if (prefix_len[r] < 0 || (prefix_len[r] + page_size - 1) / page_size > max_pages)
+            return ORACLE_BAD_ARGUMENT;
+        for (int t = 0; t < (prefix_len[r] + page_size - 1) / page_size; ++t) {
+            const int pg = page_table[(size_t)r * max_pages + t];
+            if (pg < 0 || pg >= num_pages)
+                return ORACLE_BAD_ARGUMENT;
+        }
+    }
+    const int G = Hq / Hkv;
+    double *part = (double *)calloc((size_t)R * Hkv * B, sizeof(double));
+    if (!part)
+        return ORACLE_NO_MEMORY;
+    int failed = 0;
+
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long long task = 0; task < (long long)R * Hkv; ++task) {
+        const int r = (int)(task / Hkv);
+        const int g = (int)(task % Hkv);
+        const int L = prefix_len[r];
+        const int N = L + B;
+        double *acc = part + ((size_t)r * Hkv + g) * B;
+        double *s = (double *)malloc(sizeof(double) * (size_t)N);
+        double *qrow = (double *)malloc(sizeof(double) * (size_t)d);
+        double *keys = (double *)malloc(sizeof(double) * (size_t)N * (size_t)d);
+        if (!s || !qrow || !keys) {
+            free(s); free(qrow); free(keys);
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
+        for (int j = 0; j < N; ++j) {
+            const uint16_t *src;
+            if (j < L) {
+                const size_t page = (size_t)page_table[(size_t)r * max_pages + j / page_size];
+                src = k_pages + ((page * page_size + (size_t)(j % page_size)) * Hkv + g) * d;
+            } else {
+                src = k_block + (((size_t)r * B + (j - L)) * Hkv + g) * d;
+            }
+            for (int c = 0; c < d; ++c)
+                keys[(size_t)j * d + c] = bf16_bits_to_double(src[c]);
+        }
+        for (int h = g * G; h < (g + 1) * G; ++h) {
+            for (int i = 0; i < B; ++i) {
+                const uint16_t *qs = q + ((((size_t)r * B) + i) * Hq + h) * d;
+                for (int c = 0; c < d; ++c)
+                    qrow[c] = bf16_bits_to_double(qs[c]);
+                double m = -INFINITY;
+                for (int j = 0; j < N; ++j) {
+                    double dot = 0.0;
+                    for (int c = 0; c < d; ++c)
+                        dot += qrow[c] * keys[(size_t)j * d + c];
+                    s[j] = scale * dot;
+                    if (s[j] > m)
+                        m = s[j];
+                }
+                double Z = 0.0;
+                for (int j = 0; j < N; ++j)
+                    Z += exp(s[j] - m);
+                for (int j = 0; j < B; ++j)
+                    acc[j] += exp(s[L + j] - m) / Z;
+            }
+        }
+        free(s);
+        free(qrow);
+        free(keys);
+    }
+    for (int r = 0; r < R; ++r)
+        for (int j = 0; j < B; ++j) {
+            double sum = 0.0;
+            for (int g = 0; g < Hkv; ++g)
+                sum += part[((size_t)r * Hkv + g) * B + j];
+            out[(size_t)r * B + j] = sum;
+        }
+    free(part);
+    return failed ? ORACLE_NO_MEMORY : ORACLE_OK;
+}
+
+/*
  * Attention importance from a given row normaliser (the log-sum-exp an
  * attention forward already produced for the same rows):
  *

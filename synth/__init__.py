@@ -276,3 +276,54 @@ def make_problem(cfg: FocusConfig | int, seed: int | None = None, *, device="cpu
         budget=torch.from_numpy(budget).to(device), lifted=lifted, tie_pairs=tie_pairs,
         name=cfg.name + ("_wide" if wide_logits else ""))
 
+
+
+@dataclass
+class PagedPrefix:
+    """The prefix keys of a FocusProblem laid out as a paged KV pool.
+
+    k0_pages, k1_pages [num_pages, page_size, Hkv, d] bf16: the pools of the two
+    layers (same page table).  page_table [R, max_pages] int32 (entries past a
+    request's pages are -1); prefix_len [R] int32.  Pages are handed out in a
+    seeded random order and the unused tail of each request's last page holds
+    unrelated random keys, so reading past a prefix shows up in the results.
+    """
+    k0_pages: torch.Tensor
+    k1_pages: torch.Tensor
+    page_table: torch.Tensor
+    prefix_len: torch.Tensor
+    page_size: int
+
+    def to(self, device) -> "PagedPrefix":
+        return PagedPrefix(self.k0_pages.to(device), self.k1_pages.to(device),
+                           self.page_table.to(device), self.prefix_len.to(device), self.page_size)
+
+
+def to_paged(p: FocusProblem, page_size: int, seed: int = 0, spare_pages: int = 3) -> PagedPrefix:
+    L = p.prefix_len.astype(np.int64)
+    pages = (L + page_size - 1) // page_size
+    num_pages = int(pages.sum()) + spare_pages
+    max_pages = max(1, int(pages.max()) if p.R else 1)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    perm = rng.permutation(num_pages)
+    table = np.full((p.R, max_pages), -1, np.int32)
+    cu = p.cu_prefix.cpu().numpy().astype(np.int64)
+    dev = p.k0_prefix.device
+    gen = torch.Generator(device=dev).manual_seed(seed + 1)
+    pools = []
+    for kp in (p.k0_prefix, p.k1_prefix):
+        pool = (torch.randn(num_pages, page_size, p.Hkv, p.d, generator=gen, device=dev) /
+                math.sqrt(p.d)).to(torch.bfloat16)
+        pools.append(pool)
+    nxt = 0
+    for r in range(p.R):
+        for t in range(int(pages[r])):
+            pg = int(perm[nxt])
+            nxt += 1
+            table[r, t] = pg
+            a = int(cu[r]) + t * page_size
+            b = min(int(cu[r + 1]), a + page_size)
+            for pool, kp in zip(pools, (p.k0_prefix, p.k1_prefix)):
+                pool[pg, :b - a] = kp[a:b]
+    return PagedPrefix(pools[0], pools[1], torch.from_numpy(table).to(dev),
+                       torch.from_numpy(L.astype(np.int32)).to(dev), page_size)

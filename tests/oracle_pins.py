@@ -212,6 +212,24 @@ def _true_lse(q, kp, cu, kb, Hkv, scale):
     return out
 
 
+def pin_paged_prefix_matches_packed(orc):
+    """The same prefix keys read through a page table (shuffled pages, junk in the
+    unused tail of each last page) give the same importance as the packed layout,
+    for pages shorter and longer than the prefixes."""
+    import synth
+    for page_size in (1, 3, 4, 16):
+        p = synth.make_problem(0, overrides=dict(R=4, B=5, Hq=4, Hkv=2, d=8, H=8,
+                                                 prefix=("uniform", 0, 11), decoded=("exact", 1),
+                                                 lift=("count", 1), budget=("fixed", 2)),
+                               seed=page_size)
+        pg = synth.to_paged(p, page_size, seed=page_size)
+        packed = orc.importance(p.q0, p.k0_prefix, p.cu_prefix, p.k0_block, Hq=4, Hkv=2,
+                                scale=p.scale)
+        paged = orc.importance_paged(p.q0, pg.k0_pages, pg.page_table, pg.prefix_len, p.k0_block,
+                                     Hq=4, Hkv=2, scale=p.scale)
+        np.testing.assert_allclose(paged, packed, rtol=1e-13, atol=1e-16)
+
+
 def pin_importance_lse_matches_full(orc):
     """Given the true row log-sum-exps (torch logsumexp over prefix and block keys),
     the block-keys-only importance equals the full one."""
@@ -418,5 +436,5 @@ PINS = [
     pin_delta_sign_and_pool, pin_pool_spreads_decoded_neighbour, pin_topk_lexsort,
     pin_topk_bruteforce, pin_capacity_status, pin_compact_fancy_indexing, pin_hand_evict,
     pin_hand_structural, pin_structural_properties, pin_importance_lse_matches_full,
-    pin_importance_lse_closed_form,
+    pin_importance_lse_closed_form, pin_paged_prefix_matches_packed,
 ]

@@ -155,6 +155,25 @@ def test_lse0_entry_point_validation():
                                    16, None, None, None, A, ws, None) == INVALID  # q0 missing
 
 
+def test_paged_entry_point_validation():
+    d = dims()
+    ws = F.focus_workspace_size(d)
+    L = F._lib
+
+    def call(page_table=A, max_pages=4, prefix_len=A, num_pages=8, page_size=64, pool=A):
+        return L.focus_evict_paged(ctypes.byref(d), A, pool, A, A, pool, A, page_table, max_pages,
+                                   prefix_len, num_pages, page_size, A, A, A, A, A, A, 16, None,
+                                   None, None, A, ws, None)
+    assert call(page_table=None) == INVALID
+    assert call(prefix_len=A + 2) == INVALID
+    assert call(max_pages=0) == INVALID
+    assert call(num_pages=0) == INVALID
+    assert call(page_size=48) == UNSUPPORTED     # not a power of two
+    assert call(page_size=4) == UNSUPPORTED      # below 8
+    assert call(pool=A + 8) == INVALID           # pools must be 16-byte aligned
+    assert call(num_pages=1 << 30, page_size=1 << 12) == UNSUPPORTED
+
+
 def test_plan_capacity_bounds_structured_counts():
     """With structural constraints plan_capacity is an upper bound of the retained rows."""
     import oracle

@@ -374,3 +374,65 @@ def test_evict_with_lse0_vs_oracle(case, orc):
                     p.budget.numpy())
     check_packed(packed.view(torch.int16).cpu().numpy().view(np.uint16), kept.cpu().numpy(),
                  cu.cpu().numpy(), hidden_bits(p))
+
+
+@pytest.mark.parametrize("page_size", [8, 16, 64, 128, 256])
+def test_evict_paged_vs_oracle(page_size, orc):
+    """Prefix keys read in place from a paged pool (shuffled pages, junk after each
+    prefix's end) give the oracle's results, for pages shorter and longer than a
+    128-key tile."""
+    import attention_delta_token_b200 as F
+    p = synth.make_problem(4, seed=600 + page_size, wide_logits=True,
+                           overrides=dict(R=10, prefix=("loguniform", 700)))
+    pg = synth.to_paged(p, page_size, seed=page_size)
+    ref = orc.evict(p)
+    paged_ref = orc.importance_paged(p.q0, pg.k0_pages, pg.page_table, pg.prefix_len,
+                                     p.k0_block, Hq=p.Hq, Hkv=p.Hkv, scale=p.scale)
+    np.testing.assert_allclose(paged_ref, ref["i0"], rtol=1e-12)
+    g, gp = p.to("cuda"), pg.to("cuda")
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+    ws = F.Workspace(dims)
+    cap = F.plan_capacity(p.decoded, p.budget)
+    kept = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+    packed = torch.zeros(cap, p.H, dtype=torch.bfloat16, device="cuda")
+    delta = torch.empty(p.R, p.B, device="cuda")
+    i0, i1 = torch.empty_like(delta), torch.empty_like(delta)
+    F.focus_evict_paged(dims, g.q0, gp.k0_pages, g.k0_block, g.q1, gp.k1_pages, g.k1_block,
+                        gp.page_table, gp.prefix_len, g.hidden, g.decoded, g.budget, kept, cu,
+                        packed, ws, delta_out=delta, i0_out=i0, i1_out=i1)
+    assert F.focus_read_device_status(ws) == 0
+    assert_close_importance(i0.cpu().numpy(), ref["i0"], "I0")
+    assert_close_importance(i1.cpu().numpy(), ref["i1"], "I1")
+    assert_close_delta(delta.cpu().numpy(), ref["pooled"])
+    np.testing.assert_array_equal(cu.cpu().numpy(), ref["cu_seqlens"])
+    check_selection(kept.cpu().numpy(), cu.cpu().numpy(), ref["pooled"], p.decoded.numpy(),
+                    p.budget.numpy())
+    check_packed(packed.view(torch.int16).cpu().numpy().view(np.uint16), kept.cpu().numpy(),
+                 cu.cpu().numpy(), hidden_bits(p))
+
+
+def test_evict_paged_matches_packed_bitwise():
+    """With pages of >= 128 keys each tile is one box, so the paged call reproduces the
+    packed call bit for bit; with 64-key pages too (same keys, same order)."""
+    import attention_delta_token_b200 as F
+    p = synth.make_problem(1, seed=7, wide_logits=True, overrides=dict(R=12))
+    want = run_evict(p.to("cuda"))
+    for page_size in (64, 128, 512):
+        pg = synth.to_paged(p, page_size, seed=1).to("cuda")
+        g = p.to("cuda")
+        dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+        ws = F.Workspace(dims)
+        cap = F.plan_capacity(p.decoded, p.budget)
+        kept = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+        cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+        packed = torch.zeros(cap, p.H, dtype=torch.bfloat16, device="cuda")
+        i0 = torch.empty(p.R, p.B, device="cuda")
+        i1 = torch.empty_like(i0)
+        F.focus_evict_paged(dims, g.q0, pg.k0_pages, g.k0_block, g.q1, pg.k1_pages, g.k1_block,
+                            pg.page_table, pg.prefix_len, g.hidden, g.decoded, g.budget, kept, cu,
+                            packed, ws, i0_out=i0, i1_out=i1)
+        assert F.focus_read_device_status(ws) == 0
+        np.testing.assert_array_equal(i0.cpu().numpy(), want["i0"].astype(np.float32))
+        np.testing.assert_array_equal(i1.cpu().numpy(), want["i1"].astype(np.float32))
+        np.testing.assert_array_equal(kept.cpu().numpy(), want["kept"])

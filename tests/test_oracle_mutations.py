@@ -1,5 +1,5 @@
 """Each plausible mistake planted in a copy of the oracle (on the CPU) must fail at
-least one pin.  This shows the pins constrain every step the oracle takes:
+least one pin.  A mistake is planted at every place the same expression occurs.  This shows the pins constrain every step the oracle takes:
 scale, softmax denominator, column index, head mapping, query indexing, the
 delta's sign, the pooling window, the mask, the tie-break, the budget clamp,
 the output order and the compaction source row."""
@@ -40,6 +40,10 @@ MUTATIONS = {
     "lse_sign": ("acc += exp(scale * dot - lse[row]);", "acc += exp(scale * dot + lse[row]);"),
     "lse_wrong_head_index": ("const size_t row = ((size_t)r * B + i) * Hq + h;",
                              "const size_t row = ((size_t)r * B + i) * Hq + g;"),
+    "paged_slot_ignored": ("src = k_pages + ((page * page_size + (size_t)(j % page_size)) * Hkv + g) * d;",
+                           "src = k_pages + ((page * page_size) * Hkv + g) * d;"),
+    "paged_wrong_page": ("page_table[(size_t)r * max_pages + j / page_size]",
+                         "page_table[(size_t)r * max_pages + j % page_size]"),
 }
 
 
@@ -47,9 +51,9 @@ MUTATIONS = {
 def test_mutation_is_caught(name, tmp_path):
     old, new = MUTATIONS[name]
     src = open(SRC).read()
-    assert src.count(old) == 1, f"mutation anchor for {name} not unique"
+    assert src.count(old) >= 1, f"mutation anchor for {name} not found"
     mut = tmp_path / "mutant.c"
-    mut.write_text(src.replace(old, new))
+    mut.write_text(src.replace(old, new))  # every occurrence: the same slip everywhere
     lib = oracle.build(force=True, src=str(mut), out=str(tmp_path / "libmutant.so"))
     orc = oracle.Oracle(lib)
     failed = []
