@@ -55,6 +55,25 @@ SCORE_DELTA = 0                    # rank by I1 - I0 (the method)
 SCORE_LAYER1 = 1                   # rank by I1 alone (Figure 13 ablation; layer 0 skipped)
 
 
+class FocusEvictArgs(ctypes.Structure):
+    """Mirror of focus_evict_args_t (include/focus.h)."""
+    _fields_ = [("q0", ctypes.c_void_p), ("k0_prefix", ctypes.c_void_p),
+                ("k0_block", ctypes.c_void_p), ("lse0", ctypes.c_void_p),
+                ("q1", ctypes.c_void_p), ("k1_prefix", ctypes.c_void_p),
+                ("k1_block", ctypes.c_void_p), ("cu_prefix", ctypes.c_void_p),
+                ("total_prefix", ctypes.c_int64), ("page_table", ctypes.c_void_p),
+                ("prefix_len", ctypes.c_void_p), ("max_pages", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("hidden", ctypes.c_void_p), ("decoded", ctypes.c_void_p),
+                ("budget", ctypes.c_void_p), ("decode_avg", ctypes.c_void_p),
+                ("budget_alpha", ctypes.c_float), ("budget_out", ctypes.c_void_p),
+                ("kept_idx", ctypes.c_void_p), ("cu_seqlens", ctypes.c_void_p),
+                ("packed", ctypes.c_void_p), ("capacity", ctypes.c_int64),
+                ("delta_out", ctypes.c_void_p), ("i0_out", ctypes.c_void_p),
+                ("i1_out", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t), ("stream", ctypes.c_void_p)]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
@@ -80,6 +99,7 @@ def _load() -> ctypes.CDLL:
         "focus_selftest_wait_timeout": (ctypes.c_int, [P, ctypes.c_uint64, P, P]),
         "focus_evict_with_lse0": (ctypes.c_int, [D, P, P, P, P, P, P, P, i64, P, P, P, P, P, P,
                                                  i64, P, P, P, P, sz, P]),
+        "focus_evict_ex": (ctypes.c_int, [D, ctypes.POINTER(FocusEvictArgs)]),
         "focus_evict_paged": (ctypes.c_int, [D, P, P, P, P, P, P, P, ctypes.c_int32, P,
                                              ctypes.c_int32, ctypes.c_int32, P, P, P, P, P, P, i64,
                                              P, P, P, P, sz, P]),
@@ -269,6 +289,46 @@ def focus_evict_paged(dims, q0, k0_pages, k0_block, q1, k1_pages, k1_block, page
         _ptr(i1_out, f32, "i1_out"), ws.ptr, ws.nbytes, _stream(stream)), "focus_evict_paged")
 
 
+def focus_evict_ex(dims, *, q1, k1_prefix, k1_block, hidden, decoded, kept_idx, cu_seqlens,
+                   packed, ws: Workspace, q0=None, k0_prefix=None, k0_block=None, lse0=None,
+                   cu_prefix=None, page_table=None, prefix_len=None, budget=None,
+                   decode_avg=None, budget_alpha=1.5, budget_out=None, delta_out=None,
+                   i0_out=None, i1_out=None, stream=None):
+    """The fused step with every option (focus_evict_ex).  Packed prefix: pass cu_prefix;
+    paged prefix: pass page_table and prefix_len (k*_prefix are then page pools);
+    lse0: layer-0 row log-sum-exps; decode_avg: dynamic budget (budget then unused)."""
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    a = FocusEvictArgs()
+    a.q0, a.k0_prefix, a.k0_block = _ptr(q0, bf, "q0"), _ptr(k0_prefix, bf, "k0_prefix"), \
+        _ptr(k0_block, bf, "k0_block")
+    a.lse0 = _ptr(lse0, f32, "lse0")
+    a.q1, a.k1_prefix, a.k1_block = _ptr(q1, bf, "q1"), _ptr(k1_prefix, bf, "k1_prefix"), \
+        _ptr(k1_block, bf, "k1_block")
+    if page_table is not None:
+        a.page_table = _ptr(page_table, i32, "page_table")
+        a.prefix_len = _ptr(prefix_len, i32, "prefix_len")
+        a.max_pages = int(page_table.shape[1])
+        a.num_pages, a.page_size = int(k1_prefix.shape[0]), int(k1_prefix.shape[1])
+    else:
+        a.cu_prefix = _ptr(cu_prefix, i32, "cu_prefix")
+        a.total_prefix = int(k1_prefix.shape[0])
+    a.hidden = _ptr(hidden, bf, "hidden")
+    a.decoded = _ptr(decoded, torch.uint8, "decoded")
+    a.budget = _ptr(budget, i32, "budget")
+    a.decode_avg = _ptr(decode_avg, f32, "decode_avg")
+    a.budget_alpha = float(budget_alpha)
+    a.budget_out = _ptr(budget_out, i32, "budget_out")
+    a.kept_idx = _ptr(kept_idx, i32, "kept_idx")
+    a.cu_seqlens = _ptr(cu_seqlens, i32, "cu_seqlens")
+    a.packed = _ptr(packed, bf, "packed")
+    a.capacity = int(packed.shape[0])
+    a.delta_out, a.i0_out, a.i1_out = _ptr(delta_out, f32, "delta_out"), \
+        _ptr(i0_out, f32, "i0_out"), _ptr(i1_out, f32, "i1_out")
+    a.workspace, a.workspace_bytes = ws.ptr, ws.nbytes
+    a.stream = _stream(stream)
+    _ok(_lib.focus_evict_ex(ctypes.byref(dims), ctypes.byref(a)), "focus_evict_ex")
+
+
 STATIC_SCRATCH_BYTES = 8 << 20
 
 
@@ -304,8 +364,9 @@ def focus_selftest_wait_timeout(status, elapsed_ns, limit_ns: int, stream=None):
                                          _stream(stream)), "focus_selftest_wait_timeout")
 
 
-def plan_capacity(decoded, budget, constraints: int = 0) -> int:
-    """Rows the packed batch needs: sum_r k_r with k_r = min(max(budget_r, 0), masked_r).
+def plan_capacity(decoded, budget, constraints: int = 0, dynamic: bool = False) -> int:
+    """Rows the packed batch needs: sum_r k_r with k_r = min(max(budget_r, 0), masked_r)
+    (with `dynamic`, k_r = masked_r: the dynamic budget never exceeds it).
 
     Host-side planning helper for the scheduler that owns `decoded` and
     `budget`: without structural constraints the kept-row counts never depend on
@@ -313,9 +374,12 @@ def plan_capacity(decoded, budget, constraints: int = 0) -> int:
     sum_r min(B, masked_r + k_r) over requests with k_r > 0 (candidates, their
     predecessors and the other masked tokens)."""
     dec = decoded.detach().cpu()
-    bud = budget.detach().cpu().to(torch.int64)
     masked = (dec == 0).sum(dim=1).to(torch.int64)
-    k = torch.minimum(bud.clamp(min=0), masked)
+    if dynamic:  # a dynamic budget is at most the number of masked positions
+        k = masked
+    else:
+        bud = budget.detach().cpu().to(torch.int64)
+        k = torch.minimum(bud.clamp(min=0), masked)
     if not constraints:
         return int(k.sum())
     B = dec.shape[1]

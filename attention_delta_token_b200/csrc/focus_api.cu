@@ -394,65 +394,70 @@ focus_status_t check_paging(const Paging &pg) {
     return FOCUS_OK;
 }
 
-focus_status_t evict_impl(const focus_dims_t *dims, const float *lse0, const Paging *paging,
-                          const void *q0, const void *k0_prefix, const void *k0_block,
-                          const void *q1, const void *k1_prefix, const void *k1_block,
-                          const int32_t *cu_prefix, int64_t total_prefix, const void *hidden,
-                          const uint8_t *decoded, const int32_t *budget, int32_t *kept_idx,
-                          int32_t *cu_seqlens, void *packed, int64_t capacity, float *delta_out,
-                          float *i0_out, float *i1_out, void *workspace, size_t workspace_bytes,
-                          void *stream) {
+focus_status_t evict_impl(const focus_dims_t *dims, const focus_evict_args_t &x) {
     FOCUS_TRY(check_dims(dims));
     const focus_dims_t &d = *dims;
     const bool layer1_only = d.score == FOCUS_SCORE_LAYER1;
+    const bool dynamic = x.decode_avg != nullptr;
+    const int32_t *cu_prefix = x.cu_prefix;
+    long long total_prefix = x.total_prefix;
     int prefix_box = focus::kTileKeys;
+    const Paging pg{x.page_table, x.prefix_len, x.max_pages, x.num_pages, x.page_size};
+    const Paging *paging = x.page_table ? &pg : nullptr;
     if (paging) {  // the page pools stand in for the packed prefix buffers
         FOCUS_TRY(check_paging(*paging));
         total_prefix = static_cast<long long>(paging->num_pages) * paging->page_size;
         prefix_box = paging->page_size < focus::kTileKeys ? paging->page_size : focus::kTileKeys;
         cu_prefix = paging->prefix_len;  // only checked for presence below; lengths come from here
     }
-    if (lse0) {
+    if (x.lse0) {
         if (layer1_only) return FOCUS_ERR_INVALID_ARGUMENT;
-        FOCUS_TRY(check_ptr(lse0, 4));
-        FOCUS_TRY(check_attn_inputs(d, q0, nullptr, cu_prefix, 0, k0_block));
+        FOCUS_TRY(check_ptr(x.lse0, 4));
+        FOCUS_TRY(check_attn_inputs(d, x.q0, nullptr, cu_prefix, 0, x.k0_block));
     } else if (!layer1_only) {
-        FOCUS_TRY(check_attn_inputs(d, q0, k0_prefix, cu_prefix, total_prefix, k0_block));
+        FOCUS_TRY(check_attn_inputs(d, x.q0, x.k0_prefix, cu_prefix, total_prefix, x.k0_block));
     }
-    FOCUS_TRY(check_attn_inputs(d, q1, k1_prefix, cu_prefix, total_prefix, k1_block));
-    FOCUS_TRY(check_ptr(hidden, 16));
-    FOCUS_TRY(check_ptr(decoded, 1));
-    FOCUS_TRY(check_ptr(budget, 4));
-    FOCUS_TRY(check_ptr(cu_seqlens, 4));
-    if (capacity < 0) return FOCUS_ERR_INVALID_ARGUMENT;
-    if (capacity > 0) {
-        FOCUS_TRY(check_ptr(kept_idx, 4));
-        FOCUS_TRY(check_ptr(packed, 16));
+    FOCUS_TRY(check_attn_inputs(d, x.q1, x.k1_prefix, cu_prefix, total_prefix, x.k1_block));
+    FOCUS_TRY(check_ptr(x.hidden, 16));
+    FOCUS_TRY(check_ptr(x.decoded, 1));
+    if (dynamic) {
+        FOCUS_TRY(check_ptr(x.decode_avg, 4));
+        if (!isfinite(x.budget_alpha) || x.budget_alpha < 0.f) return FOCUS_ERR_INVALID_ARGUMENT;
+        if (x.budget_out) FOCUS_TRY(check_ptr(x.budget_out, 4));
+    } else {
+        FOCUS_TRY(check_ptr(x.budget, 4));
     }
-    if (delta_out) FOCUS_TRY(check_ptr(delta_out, 4));
-    if (i0_out) FOCUS_TRY(check_ptr(i0_out, 4));
-    if (i1_out) FOCUS_TRY(check_ptr(i1_out, 4));
-    FOCUS_TRY(check_ws(d, workspace, workspace_bytes));
+    FOCUS_TRY(check_ptr(x.cu_seqlens, 4));
+    if (x.capacity < 0) return FOCUS_ERR_INVALID_ARGUMENT;
+    if (x.capacity > 0) {
+        FOCUS_TRY(check_ptr(x.kept_idx, 4));
+        FOCUS_TRY(check_ptr(x.packed, 16));
+    }
+    if (x.delta_out) FOCUS_TRY(check_ptr(x.delta_out, 4));
+    if (x.i0_out) FOCUS_TRY(check_ptr(x.i0_out, 4));
+    if (x.i1_out) FOCUS_TRY(check_ptr(x.i1_out, 4));
+    FOCUS_TRY(check_ws(d, x.workspace, x.workspace_bytes));
     FOCUS_TRY(get_encoder());
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    cudaStream_t s = static_cast<cudaStream_t>(x.stream);
+    uint8_t *ws = static_cast<uint8_t *>(x.workspace);
 
     AttnParams p;
     memset(&p, 0, sizeof p);
     if (layer1_only) {  // the Figure 13 ablation: rank by I1, layer 0 is not touched
         fill_common(p, d, cu_prefix, total_prefix, ws, 1);
-        FOCUS_TRY(encode_layer(p, 0, d, q1, k1_prefix, total_prefix, k1_block, prefix_box));
+        FOCUS_TRY(encode_layer(p, 0, d, x.q1, x.k1_prefix, total_prefix, x.k1_block, prefix_box));
         p.tm_q[1] = p.tm_q[0];
         p.tm_kp[1] = p.tm_kp[0];
         p.tm_kb[1] = p.tm_kb[0];
     } else {
         fill_common(p, d, cu_prefix, total_prefix, ws, 2);
-        if (lse0)  // layer 0 streams no prefix: its prefix map is never read
-            FOCUS_TRY(encode_layer(p, 0, d, q0, nullptr, 0, k0_block));
+        if (x.lse0)  // layer 0 streams no prefix: its prefix map is never read
+            FOCUS_TRY(encode_layer(p, 0, d, x.q0, nullptr, 0, x.k0_block));
         else
-            FOCUS_TRY(encode_layer(p, 0, d, q0, k0_prefix, total_prefix, k0_block, prefix_box));
-        FOCUS_TRY(encode_layer(p, 1, d, q1, k1_prefix, total_prefix, k1_block, prefix_box));
-        p.lse0 = lse0;
+            FOCUS_TRY(encode_layer(p, 0, d, x.q0, x.k0_prefix, total_prefix, x.k0_block,
+                                   prefix_box));
+        FOCUS_TRY(encode_layer(p, 1, d, x.q1, x.k1_prefix, total_prefix, x.k1_block, prefix_box));
+        p.lse0 = x.lse0;
     }
     if (paging) {
         p.cu_prefix = nullptr;
@@ -463,17 +468,20 @@ focus_status_t evict_impl(const focus_dims_t *dims, const float *lse0, const Pag
         p.num_pages = paging->num_pages;
         p.page_rows = prefix_box;
     }
+    // With constraints or a dynamic budget the kept counts depend on the data, so the
+    // selection writes per-request lists and cu_seqlens is scanned afterwards.
+    const bool lists = d.constraints != 0 || dynamic;
 
     focus::PlanParams pp;
     memset(&pp, 0, sizeof pp);
     pp.cu_prefix = paging ? nullptr : cu_prefix;
     pp.prefix_len = paging ? paging->prefix_len : nullptr;
-    pp.decoded = decoded;
-    pp.budget = budget;
+    pp.decoded = x.decoded;
+    pp.budget = x.budget;
     pp.order = const_cast<int32_t *>(p.order);
-    pp.cu_seqlens = d.constraints ? nullptr : cu_seqlens;  // with constraints: after selection
+    pp.cu_seqlens = lists ? nullptr : x.cu_seqlens;
     pp.status = p.status;
-    pp.capacity = capacity;
+    pp.capacity = x.capacity;
     pp.R = d.R;
     pp.B = d.B;
     FOCUS_CUDA(focus::launch_plan(pp, s));
@@ -483,14 +491,14 @@ focus_status_t evict_impl(const focus_dims_t *dims, const float *lse0, const Pag
     focus::SelectParams sp;
     memset(&sp, 0, sizeof sp);
     sp.partial = p.partial;
-    sp.decoded = decoded;
-    sp.cu_seqlens = cu_seqlens;
-    sp.kept_idx = kept_idx;
-    sp.delta_out = delta_out;
-    sp.i0_out = i0_out;
-    sp.i1_out = i1_out;
+    sp.decoded = x.decoded;
+    sp.cu_seqlens = x.cu_seqlens;
+    sp.kept_idx = x.kept_idx;
+    sp.delta_out = x.delta_out;
+    sp.i0_out = x.i0_out;
+    sp.i1_out = x.i1_out;
     sp.status = p.status;
-    sp.capacity = capacity;
+    sp.capacity = x.capacity;
     sp.R = d.R;
     sp.B = d.B;
     sp.Hkv = d.Hkv;
@@ -498,24 +506,27 @@ focus_status_t evict_impl(const focus_dims_t *dims, const float *lse0, const Pag
     sp.H = d.hidden;
     sp.pool_window = d.pool_window;
     sp.layers = layer1_only ? 1 : 2;
-    if (d.constraints) {
+    if (lists) {
         const WsLayout w = ws_layout(d);
         sp.constraints = d.constraints;
-        sp.budget = budget;
+        sp.budget = x.budget;
+        sp.decode_avg = x.decode_avg;
+        sp.budget_alpha = x.budget_alpha;
+        sp.budget_out = x.budget_out;
         sp.lists = reinterpret_cast<int32_t *>(ws + w.lists);
         sp.counts = reinterpret_cast<int32_t *>(ws + w.counts);
         FOCUS_CUDA(focus::launch_select_compact(sp, s, /*pdl=*/true));
-        focus::ScanParams sc{sp.counts, cu_seqlens, p.status, capacity, d.R};
+        focus::ScanParams sc{sp.counts, x.cu_seqlens, p.status, x.capacity, d.R};
         FOCUS_CUDA(focus::launch_scan(sc, s, /*pdl=*/true));
-        focus::CompactParams cp{static_cast<const uint16_t *>(hidden), nullptr, cu_seqlens,
-                                static_cast<uint16_t *>(packed), p.status, capacity, d.R, d.B,
-                                d.hidden, sp.lists, kept_idx};
+        focus::CompactParams cp{static_cast<const uint16_t *>(x.hidden), nullptr, x.cu_seqlens,
+                                static_cast<uint16_t *>(x.packed), p.status, x.capacity, d.R, d.B,
+                                d.hidden, sp.lists, x.kept_idx};
         FOCUS_CUDA(focus::launch_compact(cp, s, /*pdl=*/true));
         return FOCUS_OK;
     }
     FOCUS_CUDA(focus::launch_select_compact(sp, s, /*pdl=*/true));
-    focus::CompactParams cp{static_cast<const uint16_t *>(hidden), kept_idx, cu_seqlens,
-                            static_cast<uint16_t *>(packed), p.status, capacity, d.R, d.B,
+    focus::CompactParams cp{static_cast<const uint16_t *>(x.hidden), x.kept_idx, x.cu_seqlens,
+                            static_cast<uint16_t *>(x.packed), p.status, x.capacity, d.R, d.B,
                             d.hidden, nullptr, nullptr};
     FOCUS_CUDA(focus::launch_compact(cp, s, /*pdl=*/true));
     return FOCUS_OK;
@@ -525,6 +536,11 @@ focus_status_t evict_impl(const focus_dims_t *dims, const float *lse0, const Pag
 
 extern "C" {
 
+focus_status_t focus_evict_ex(const focus_dims_t *dims, const focus_evict_args_t *args) {
+    if (!args) return FOCUS_ERR_INVALID_ARGUMENT;
+    return evict_impl(dims, *args);
+}
+
 focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void *k0_prefix,
                            const void *k0_block, const void *q1, const void *k1_prefix,
                            const void *k1_block, const int32_t *cu_prefix, int64_t total_prefix,
@@ -532,10 +548,30 @@ focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void 
                            int32_t *kept_idx, int32_t *cu_seqlens, void *packed, int64_t capacity,
                            float *delta_out, float *i0_out, float *i1_out, void *workspace,
                            size_t workspace_bytes, void *stream) {
-    return evict_impl(dims, nullptr, nullptr, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block,
-                      cu_prefix,
-                      total_prefix, hidden, decoded, budget, kept_idx, cu_seqlens, packed,
-                      capacity, delta_out, i0_out, i1_out, workspace, workspace_bytes, stream);
+    focus_evict_args_t x;
+    memset(&x, 0, sizeof x);
+    x.q0 = q0;
+    x.k0_prefix = k0_prefix;
+    x.k0_block = k0_block;
+    x.q1 = q1;
+    x.k1_prefix = k1_prefix;
+    x.k1_block = k1_block;
+    x.cu_prefix = cu_prefix;
+    x.total_prefix = total_prefix;
+    x.hidden = hidden;
+    x.decoded = decoded;
+    x.budget = budget;
+    x.kept_idx = kept_idx;
+    x.cu_seqlens = cu_seqlens;
+    x.packed = packed;
+    x.capacity = capacity;
+    x.delta_out = delta_out;
+    x.i0_out = i0_out;
+    x.i1_out = i1_out;
+    x.workspace = workspace;
+    x.workspace_bytes = workspace_bytes;
+    x.stream = stream;
+    return evict_impl(dims, x);
 }
 
 focus_status_t focus_evict_with_lse0(const focus_dims_t *dims, const float *lse0, const void *q0,
@@ -548,10 +584,30 @@ focus_status_t focus_evict_with_lse0(const focus_dims_t *dims, const float *lse0
                                      float *i1_out, void *workspace, size_t workspace_bytes,
                                      void *stream) {
     if (!lse0) return FOCUS_ERR_INVALID_ARGUMENT;
-    return evict_impl(dims, lse0, nullptr, q0, nullptr, k0_block, q1, k1_prefix, k1_block,
-                      cu_prefix,
-                      total_prefix, hidden, decoded, budget, kept_idx, cu_seqlens, packed,
-                      capacity, delta_out, i0_out, i1_out, workspace, workspace_bytes, stream);
+    focus_evict_args_t x;
+    memset(&x, 0, sizeof x);
+    x.q0 = q0;
+    x.k0_block = k0_block;
+    x.lse0 = lse0;
+    x.q1 = q1;
+    x.k1_prefix = k1_prefix;
+    x.k1_block = k1_block;
+    x.cu_prefix = cu_prefix;
+    x.total_prefix = total_prefix;
+    x.hidden = hidden;
+    x.decoded = decoded;
+    x.budget = budget;
+    x.kept_idx = kept_idx;
+    x.cu_seqlens = cu_seqlens;
+    x.packed = packed;
+    x.capacity = capacity;
+    x.delta_out = delta_out;
+    x.i0_out = i0_out;
+    x.i1_out = i1_out;
+    x.workspace = workspace;
+    x.workspace_bytes = workspace_bytes;
+    x.stream = stream;
+    return evict_impl(dims, x);
 }
 
 focus_status_t focus_evict_paged(const focus_dims_t *dims, const void *q0, const void *k0_pages,
@@ -563,10 +619,34 @@ focus_status_t focus_evict_paged(const focus_dims_t *dims, const void *q0, const
                                  void *packed, int64_t capacity, float *delta_out, float *i0_out,
                                  float *i1_out, void *workspace, size_t workspace_bytes,
                                  void *stream) {
-    const Paging pg{page_table, prefix_len, max_pages, num_pages, page_size};
-    return evict_impl(dims, nullptr, &pg, q0, k0_pages, k0_block, q1, k1_pages, k1_block, nullptr,
-                      0, hidden, decoded, budget, kept_idx, cu_seqlens, packed, capacity,
-                      delta_out, i0_out, i1_out, workspace, workspace_bytes, stream);
+    if (!page_table) return FOCUS_ERR_INVALID_ARGUMENT;
+    focus_evict_args_t x;
+    memset(&x, 0, sizeof x);
+    x.q0 = q0;
+    x.k0_prefix = k0_pages;
+    x.k0_block = k0_block;
+    x.q1 = q1;
+    x.k1_prefix = k1_pages;
+    x.k1_block = k1_block;
+    x.page_table = page_table;
+    x.prefix_len = prefix_len;
+    x.max_pages = max_pages;
+    x.num_pages = num_pages;
+    x.page_size = page_size;
+    x.hidden = hidden;
+    x.decoded = decoded;
+    x.budget = budget;
+    x.kept_idx = kept_idx;
+    x.cu_seqlens = cu_seqlens;
+    x.packed = packed;
+    x.capacity = capacity;
+    x.delta_out = delta_out;
+    x.i0_out = i0_out;
+    x.i1_out = i1_out;
+    x.workspace = workspace;
+    x.workspace_bytes = workspace_bytes;
+    x.stream = stream;
+    return evict_impl(dims, x);
 }
 
 const char *focus_status_string(focus_status_t st) {

@@ -104,6 +104,11 @@ struct SelectParams {
     const int32_t *budget;     // [R]
     int32_t *lists;            // [R*B]
     int32_t *counts;           // [R]
+    // Dynamic budget (decode_avg != null): K_r from the historical yield and the
+    // masked delta's mean + std, written to budget_out (nullable).
+    const float *decode_avg;   // [R]
+    float budget_alpha;
+    int32_t *budget_out;       // [R]
 };
 
 struct ScanParams {

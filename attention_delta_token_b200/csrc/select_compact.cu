@@ -248,12 +248,37 @@ __global__ void __launch_bounds__(256) select_compact_kernel(const SelectParams 
     }
     __syncthreads();
 
-    if (p.constraints) {
-        // Candidates, then the structural constraints; the retained positions go to a
-        // per-request list (their count depends on the data: cu_seqlens comes later).
+    if (p.constraints || p.decode_avg) {
+        // Candidates (under the given or the dynamic budget), then the structural
+        // constraints; the retained positions go to a per-request list (their count
+        // depends on the data: cu_seqlens comes later).
         __shared__ int rightmost;
+        __shared__ int k_dyn;
         const int masked = __syncthreads_count(j < B && dec_s[j] == 0);
-        const int k = min(max(p.budget[r], 0), masked);
+        if (p.decode_avg && j == 0) {
+            // K = min(max(ceil(alpha * yield), #{masked D > mean + std}, 1), masked),
+            // statistics over the masked positions in position order.
+            int K = 0;
+            if (masked > 0) {
+                float sum = 0.f;
+                for (int t = 0; t < B; ++t)
+                    if (!dec_s[t]) sum += val_s[t];
+                const float mu = sum / masked;
+                float ss = 0.f;
+                for (int t = 0; t < B; ++t)
+                    if (!dec_s[t]) ss += (val_s[t] - mu) * (val_s[t] - mu);
+                const float thr = mu + sqrtf(ss / masked);
+                int n = 0;
+                for (int t = 0; t < B; ++t) n += !dec_s[t] && val_s[t] > thr;
+                const float want = ceilf(p.budget_alpha * fmaxf(p.decode_avg[r], 0.f));
+                K = want >= static_cast<float>(masked) ? masked : max(static_cast<int>(want), n);
+                K = min(max(K, 1), masked);
+            }
+            k_dyn = K;
+            if (p.budget_out) p.budget_out[r] = K;
+        }
+        __syncthreads();
+        const int k = p.decode_avg ? k_dyn : min(max(p.budget[r], 0), masked);
         if (j == 0) rightmost = -1;
         if (j < B) {
             const float v = val_s[j];

@@ -245,7 +245,22 @@ def run_ours(args, rank, world, local_rank):
     in_bytes = sum(t.numel() * t.element_size() for t in p.tensors().values())
 
     layer0 = (None, None, None) if args.score else (p.q0, p.k0_prefix, p.k0_block)
-    if args.page_size:
+    if args.dynamic_budget:
+        # historical decoded-per-step averages: ~10% of a 32-token block per step
+        # (Figure 2), drawn uniformly in [0, 0.2 B] per request
+        gen = torch.Generator().manual_seed(seed)
+        decode_avg = (torch.rand(p.R, generator=gen) * 0.2 * p.B).to(dev)
+        budget_out = torch.empty(p.R, dtype=torch.int32, device=dev)
+        cap = F.plan_capacity(p.decoded, None, args.constraints, dynamic=True)
+        kept, cu, packed = make_outputs(p, cap, dev)
+
+        def step():
+            F.focus_evict_ex(dims, q0=p.q0, k0_prefix=p.k0_prefix, k0_block=p.k0_block, q1=p.q1,
+                             k1_prefix=p.k1_prefix, k1_block=p.k1_block, cu_prefix=p.cu_prefix,
+                             hidden=p.hidden, decoded=p.decoded, decode_avg=decode_avg,
+                             budget_alpha=1.5, budget_out=budget_out, kept_idx=kept,
+                             cu_seqlens=cu, packed=packed, ws=ws)
+    elif args.page_size:
         pg = synth.to_paged(p, args.page_size, seed=seed)
 
         def step():
@@ -306,7 +321,7 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- end to end: pinned host inputs -> device, the C-ABI call, result -> host
     e2e = None
-    if not args.no_e2e and not (args.score or args.lse0 or args.page_size):  # the default path
+    if not args.no_e2e and not (args.score or args.lse0 or args.page_size or args.dynamic_budget):
         host = {k: v.to("cpu").pin_memory() for k, v in p.tensors().items()}
         dev_t = p.tensors()
         out_kept = torch.empty(kept.shape, dtype=kept.dtype).pin_memory()
@@ -365,14 +380,15 @@ def run_ours(args, rank, world, local_rank):
                 "l2": f"no flush: {in_bytes / 2**30:.2f} GiB of inputs per step > 126 MB L2",
                 "accumulate": "fp32", "parallelism": f"dp{world} (request-sharded replicas)",
                 "constraints": args.constraints, "score": args.score, "lse0": args.lse0,
-                "page_size": args.page_size,
+                "page_size": args.page_size, "dynamic_budget": args.dynamic_budget,
             },
             "decisions_per_s": world * counts["decisions"] / step_s,
             "roofline": {
                 "bound": "hbm", "kernel": "attn_stats_kernel", "achieved": achieved,
                 "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "traffic": (read_traffic(workload)
-                            if not (args.score or args.lse0 or args.page_size) else None),
+                            if not (args.score or args.lse0 or args.page_size
+                                    or args.dynamic_budget) else None),
                 "algorithmic_bytes_per_launch": counts["attn_bytes"],
                 "ms_per_launch": attn_s_max * 1e3, "peak_source": f"{peak_src} (hbm_gbs)",
                 "launches_timed": len(traced),
@@ -482,6 +498,8 @@ def main():
     ap.add_argument("--page-size", type=int, default=0,
                     help="read the prefix keys from a paged pool with pages of this many tokens "
                          "(focus_evict_paged)")
+    ap.add_argument("--dynamic-budget", action="store_true",
+                    help="dynamic retention budget (focus_evict_ex with decode_avg)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -213,6 +213,58 @@ FOCUS_API focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, c
 FOCUS_API void focus_set_trace_events(void *start_event, void *stop_event);
 
 /*
+ * All arguments of the fused step, for focus_evict_ex.  Optional features are
+ * switched on by their pointers:
+ *  - lse0 != NULL: layer 0's row log-sum-exps are given (see focus_evict_with_lse0);
+ *    k0_prefix is then not read.
+ *  - page_table != NULL: the prefix keys are in page pools (see focus_evict_paged);
+ *    cu_prefix/total_prefix are then not used.
+ *  - decode_avg != NULL: dynamic retention budget (below); `budget` is then not read.
+ *
+ * Dynamic budget.  Eq. 4 is not printed on the FOCUS pages; the Referee Report
+ * summary says the budget comes "from historical decoding yield and within-block
+ * delta statistics", the Free-Parameter Ledger gives the expansion factor
+ * alpha = 1.5 of Eq. 4, and Figure 14 marks the "+Std" sigma threshold used for
+ * it.  This library's reading, per request r, over its masked positions M_r and
+ * the pooled, masked delta D:
+ *   mu_r = mean D_j, sigma_r = population std of D_j (j in M_r),
+ *   n_r  = #{j in M_r : D_j > mu_r + sigma_r},
+ *   K_r  = min(max(ceil(budget_alpha * max(decode_avg[r], 0)), n_r, 1), |M_r|)  (0 if M_r is empty)
+ * decode_avg [R] float32 is the request's historical mean number of tokens
+ * decoded per step.  budget_out [R] int32 (nullable) receives K_r.  The retained
+ * counts then depend on the data: `capacity` must be an upper bound (the number
+ * of masked positions, or min(B, 2 x masked) with structural constraints) and
+ * cu_seqlens is computed on the device.
+ */
+typedef struct {
+    const void *q0, *k0_prefix, *k0_block;  /* layer 0 */
+    const float *lse0;                      /* optional [R, B, Hq] */
+    const void *q1, *k1_prefix, *k1_block;  /* layer 1 */
+    const int32_t *cu_prefix;               /* packed prefix layout */
+    int64_t total_prefix;
+    const int32_t *page_table;              /* paged prefix layout (optional) */
+    const int32_t *prefix_len;
+    int32_t max_pages, num_pages, page_size;
+    const void *hidden;                     /* [R, B, H] bf16 */
+    const uint8_t *decoded;                 /* [R, B] */
+    const int32_t *budget;                  /* [R]; unused with decode_avg */
+    const float *decode_avg;                /* optional [R]: dynamic budget */
+    float budget_alpha;                     /* Eq. 4 expansion factor (1.5) */
+    int32_t *budget_out;                    /* optional [R] */
+    int32_t *kept_idx;                      /* outputs */
+    int32_t *cu_seqlens;
+    void *packed;
+    int64_t capacity;
+    float *delta_out, *i0_out, *i1_out;     /* optional [R, B] */
+    void *workspace;
+    size_t workspace_bytes;
+    void *stream;
+} focus_evict_args_t;
+
+/* The fused step with every option (focus_evict and its variants call this). */
+FOCUS_API focus_status_t focus_evict_ex(const focus_dims_t *dims, const focus_evict_args_t *args);
+
+/*
  * The fused step with the prefix keys in a paged KV cache (pages of page_size
  * tokens, each request owning an ordered list of pages, the same list for both
  * layers), read in place:

@@ -95,11 +95,12 @@ class Oracle:
         lib.focus_oracle_importance_lse.argtypes = [i32, i32, i32, i32, i32, f64, P, P, P, P]
         lib.focus_oracle_importance_paged.argtypes = [i32, i32, i32, i32, i32, f64, P, P, P, i32,
                                                       P, i32, i32, P, P]
+        lib.focus_oracle_dynamic_budget.argtypes = [i32, i32, P, P, P, f64, P]
         lib.focus_oracle_num_threads.argtypes = []
         for fn in (lib.focus_oracle_importance, lib.focus_oracle_delta, lib.focus_oracle_select,
                    lib.focus_oracle_compact, lib.focus_oracle_num_threads,
                    lib.focus_oracle_select_structured, lib.focus_oracle_importance_lse,
-                   lib.focus_oracle_importance_paged):
+                   lib.focus_oracle_importance_paged, lib.focus_oracle_dynamic_budget):
             fn.restype = ctypes.c_int
         self.lib = lib
 
@@ -197,6 +198,18 @@ class Oracle:
         _check(st, "select_structured", allow_capacity=True)
         return kept[:min(cap, int(cu[-1]))], cu, st
 
+    def dynamic_budget(self, pooled, decoded, decode_avg, alpha: float = 1.5) -> np.ndarray:
+        """K_r from the historical yield and the masked-delta mean + std (see the C source)."""
+        pv = _arr(pooled, np.float64)
+        dec = _arr(decoded, np.uint8)
+        avg = _arr(decode_avg, np.float64)
+        R, B = pv.shape
+        out = np.zeros((R,), np.int32)
+        st = self.lib.focus_oracle_dynamic_budget(R, B, _p(pv), _p(dec), _p(avg), float(alpha),
+                                                  _p(out))
+        _check(st, "dynamic_budget")
+        return out
+
     def compact(self, hidden, kept, cu_seqlens, *, capacity: int | None = None) -> np.ndarray:
         """packed [capacity, H] uint16 (bf16 bits) of the kept hidden rows."""
         hid = _u16(hidden)
@@ -211,7 +224,8 @@ class Oracle:
         _check(st, "compact")
         return packed[:capacity]
 
-    def evict(self, p, constraints: int = 0, score: int = 0, lse0=None) -> dict:
+    def evict(self, p, constraints: int = 0, score: int = 0, lse0=None, decode_avg=None,
+              alpha: float = 1.5) -> dict:
         """The whole step on a problem object with the fields of ``synth.FocusProblem``.
 
         Returns float64 i0, i1, delta (raw), pooled (masked) [R, B]; int32 kept
@@ -230,13 +244,16 @@ class Oracle:
         i1 = self.importance(p.q1, p.k1_prefix, p.cu_prefix, p.k1_block, Hq=p.Hq, Hkv=p.Hkv,
                              scale=p.scale)
         raw, pooled = self.delta_pool_mask(i0, i1, p.decoded, window=p.pool_window)
+        budget = p.budget
+        if decode_avg is not None:  # dynamic budget (Eq. 4 as read)
+            budget = self.dynamic_budget(pooled, p.decoded, decode_avg, alpha)
         if constraints:
-            kept, cu, st = self.select_structured(pooled, p.decoded, p.budget, constraints)
+            kept, cu, st = self.select_structured(pooled, p.decoded, budget, constraints)
         else:
-            kept, cu, st = self.select(pooled, p.decoded, p.budget)
+            kept, cu, st = self.select(pooled, p.decoded, budget)
         packed = self.compact(p.hidden, kept, cu)
         return dict(i0=i0, i1=i1, delta=raw, pooled=pooled, kept=kept, cu_seqlens=cu,
-                    packed=packed)
+                    packed=packed, budget=np.asarray(_arr(budget, np.int32)))
 
 
 _default = None
@@ -270,8 +287,13 @@ def compact(*a, **k):
     return default().compact(*a, **k)
 
 
-def evict(p, constraints: int = 0, score: int = 0, lse0=None) -> dict:
-    return default().evict(p, constraints, score, lse0)
+def evict(p, constraints: int = 0, score: int = 0, lse0=None, decode_avg=None,
+          alpha: float = 1.5) -> dict:
+    return default().evict(p, constraints, score, lse0, decode_avg, alpha)
+
+
+def dynamic_budget(*a, **k):
+    return default().dynamic_budget(*a, **k)
 
 
 def importance_lse(*a, **k):

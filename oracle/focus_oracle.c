@@ -492,6 +492,58 @@ int focus_oracle_select_structured(int R, int B, const double *pooled, const uin
 }
 
 /*
+ * Dynamic retention budget (a reading of Eq. 4, which the pages do not print:
+ * "Dynamic Budgeting" sets K from the request's historical decoding yield scaled
+ * by the expansion factor alpha (default 1.5, Free-Parameter Ledger) and from the
+ * within-block delta statistics -- the "+Std" sigma threshold of Figure 14):
+ *
+ *   over the masked positions M_r of block r (D = pooled, masked delta):
+ *     mu_r = mean_{j in M_r} D_j,  sigma_r = sqrt(mean_{j in M_r} (D_j - mu_r)^2)
+ *     n_r  = #{j in M_r : D_j > mu_r + sigma_r}
+ *   K_r = min(max(ceil(alpha * decode_avg[r]), n_r, 1), |M_r|);  K_r = 0 when M_r is empty.
+ */
+int focus_oracle_dynamic_budget(int R, int B, const double *pooled, const uint8_t *decoded,
+                                const double *decode_avg, double alpha, int32_t *budget_out)
+{
+    if (R < 0 || B <= 0 || !(alpha >= 0.0))
+        return ORACLE_BAD_ARGUMENT;
+    for (int r = 0; r < R; ++r) {
+        const double *D = pooled + (size_t)r * B;
+        const uint8_t *dec = decoded + (size_t)r * B;
+        int m = 0;
+        double sum = 0.0;
+        for (int j = 0; j < B; ++j)
+            if (!dec[j]) {
+                ++m;
+                sum += D[j];
+            }
+        if (m == 0) {
+            budget_out[r] = 0;
+            continue;
+        }
+        const double mu = sum / m;
+        double ss = 0.0;
+        for (int j = 0; j < B; ++j)
+            if (!dec[j])
+                ss += (D[j] - mu) * (D[j] - mu);
+        const double sigma = sqrt(ss / m);
+        int n = 0;
+        for (int j = 0; j < B; ++j)
+            if (!dec[j] && D[j] > mu + sigma)
+                ++n;
+        double want = ceil(alpha * (decode_avg[r] > 0.0 ? decode_avg[r] : 0.0));
+        if (want < n)
+            want = n;
+        if (want < 1)
+            want = 1;
+        if (want > m)
+            want = m;
+        budget_out[r] = (int32_t)want;
+    }
+    return ORACLE_OK;
+}
+
+/*
  * Compaction of the retained tokens' hidden rows into a packed varlen batch:
  *   packed[cu[r] + t][:] = hidden[r][kept[cu[r] + t]][:]   (bit copy)
  */

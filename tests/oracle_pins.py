@@ -230,6 +230,33 @@ def pin_paged_prefix_matches_packed(orc):
         np.testing.assert_allclose(paged, packed, rtol=1e-13, atol=1e-16)
 
 
+def pin_hand_dynamic_budget(orc):
+    """Dynamic budgets worked by hand (tests/golden/hand_dynamic_budget.json)."""
+    fx = json.load(open(os.path.join(GOLDEN, "hand_dynamic_budget.json")))
+    for c in fx["cases"]:
+        pooled = np.array([[_num(x) for x in c["pooled"]]])
+        dec = np.array([c["decoded"]], np.uint8)
+        got = orc.dynamic_budget(pooled, dec, np.array([c["decode_avg"]]), c["alpha"])
+        assert got.tolist() == [c["budget"]], (c["derivation"], got)
+
+
+def pin_dynamic_budget_bounds(orc):
+    """On random blocks: 1 <= K_r <= masked_r (0 when nothing is masked); K_r grows with
+    the historical yield; a large yield saturates at masked_r."""
+    rng = np.random.default_rng(22)
+    R, B = 40, 16
+    pooled = rng.normal(size=(R, B))
+    dec = (rng.random((R, B)) < 0.4).astype(np.uint8)
+    pooled[dec != 0] = -np.inf
+    masked = (dec == 0).sum(1)
+    k_lo = orc.dynamic_budget(pooled, dec, np.zeros(R))
+    k_hi = orc.dynamic_budget(pooled, dec, np.full(R, 3.0))
+    k_sat = orc.dynamic_budget(pooled, dec, np.full(R, 1e6))
+    assert ((k_lo >= np.minimum(1, masked)) & (k_lo <= masked)).all()
+    assert (k_hi >= k_lo).all() and (k_hi >= np.minimum(5, masked)).all()  # ceil(1.5 * 3) = 5
+    np.testing.assert_array_equal(k_sat, masked)
+
+
 def pin_importance_lse_matches_full(orc):
     """Given the true row log-sum-exps (torch logsumexp over prefix and block keys),
     the block-keys-only importance equals the full one."""
@@ -436,5 +463,6 @@ PINS = [
     pin_delta_sign_and_pool, pin_pool_spreads_decoded_neighbour, pin_topk_lexsort,
     pin_topk_bruteforce, pin_capacity_status, pin_compact_fancy_indexing, pin_hand_evict,
     pin_hand_structural, pin_structural_properties, pin_importance_lse_matches_full,
-    pin_importance_lse_closed_form, pin_paged_prefix_matches_packed,
+    pin_importance_lse_closed_form, pin_paged_prefix_matches_packed, pin_hand_dynamic_budget,
+    pin_dynamic_budget_bounds,
 ]

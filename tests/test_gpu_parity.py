@@ -436,3 +436,54 @@ def test_evict_paged_matches_packed_bitwise():
         np.testing.assert_array_equal(i0.cpu().numpy(), want["i0"].astype(np.float32))
         np.testing.assert_array_equal(i1.cpu().numpy(), want["i1"].astype(np.float32))
         np.testing.assert_array_equal(kept.cpu().numpy(), want["kept"])
+
+
+@pytest.mark.parametrize("case,constraints", [("sdar_r8_wide", 0), ("ragged_r10_ties", 0),
+                                              ("block128_r3", 0), ("sdar_r8_wide", 3)])
+def test_dynamic_budget_vs_oracle(case, constraints, orc):
+    """Dynamic budget (Eq. 4 as read): the GPU's K_r equals the oracle's wherever no
+    masked pooled delta lies within 1e-2 of the mean + std threshold; the selection
+    under the GPU's K_r matches the oracle's under the same K_r."""
+    import attention_delta_token_b200 as F
+    cfg, ov, wide = STRUCTURED_CASES[case]
+    p = synth.make_problem(cfg, seed=700, wide_logits=wide, overrides=ov)
+    rng = np.random.default_rng(7)
+    avg = rng.uniform(0.0, 4.0, size=p.R).astype(np.float32)
+    ref = orc.evict(p, constraints=constraints, decode_avg=avg.astype(np.float64))
+    g = p.to("cuda")
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, constraints)
+    ws = F.Workspace(dims)
+    cap = F.plan_capacity(p.decoded, None, constraints, dynamic=True)
+    kept = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+    packed = torch.zeros(cap, p.H, dtype=torch.bfloat16, device="cuda")
+    delta = torch.empty(p.R, p.B, device="cuda")
+    kout = torch.full((p.R,), -1, dtype=torch.int32, device="cuda")
+    F.focus_evict_ex(dims, q0=g.q0, k0_prefix=g.k0_prefix, k0_block=g.k0_block, q1=g.q1,
+                     k1_prefix=g.k1_prefix, k1_block=g.k1_block, cu_prefix=g.cu_prefix,
+                     hidden=g.hidden, decoded=g.decoded, decode_avg=torch.from_numpy(avg).cuda(),
+                     budget_alpha=1.5, budget_out=kout, kept_idx=kept, cu_seqlens=cu,
+                     packed=packed, ws=ws, delta_out=delta)
+    assert F.focus_read_device_status(ws) == 0
+    assert_close_delta(delta.cpu().numpy(), ref["pooled"])
+    kg = kout.cpu().numpy()
+    dec = p.decoded.numpy()
+    checked = 0
+    for r in range(p.R):
+        m = dec[r] == 0
+        assert (kg[r] == 0) if not m.any() else (1 <= kg[r] <= m.sum())
+        D = ref["pooled"][r][m]
+        if D.size == 0:
+            continue
+        thr = D.mean() + D.std()
+        if np.all(np.abs(D - thr) > 1e-2):
+            assert kg[r] == ref["budget"][r], (r, kg[r], ref["budget"][r])
+            checked += 1
+    assert checked >= p.R // 2, checked
+    # selection under the GPU's own budgets
+    cu_h = cu.cpu().numpy()
+    kept_h = kept[:int(cu_h[-1])].cpu().numpy()
+    if constraints == 0:
+        check_selection(kept_h, cu_h, ref["pooled"], dec, kg)
+    check_packed(packed[:int(cu_h[-1])].view(torch.int16).cpu().numpy().view(np.uint16), kept_h,
+                 cu_h, hidden_bits(p))

@@ -44,6 +44,9 @@ MUTATIONS = {
                            "src = k_pages + ((page * page_size) * Hkv + g) * d;"),
     "paged_wrong_page": ("page_table[(size_t)r * max_pages + j / page_size]",
                          "page_table[(size_t)r * max_pages + j % page_size]"),
+    "budget_threshold_mean_only": ("if (!dec[j] && D[j] > mu + sigma)", "if (!dec[j] && D[j] > mu)"),
+    "budget_alpha_dropped": ("double want = ceil(alpha * (decode_avg[r]", "double want = ceil(1.0 * (decode_avg[r]"),
+    "budget_sample_std": ("const double sigma = sqrt(ss / m);", "const double sigma = sqrt(ss / (m > 1 ? m - 1 : 1));"),
 }
 
 
