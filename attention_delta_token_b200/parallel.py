@@ -1,0 +1,70 @@
+"""Tensor-parallel (head-sharded) eviction.
+
+In a tensor-parallel engine each rank holds a contiguous slice of the query
+heads and of their kv heads.  I_j is a sum over heads ("What carries the
+argument": the column-wise sum of the attention the block's queries pay token
+j), so each rank computes the importance of its own heads for both layers with
+focus_attn_stats, one all-reduce (sum, fp32, 2 x R x B values) combines them,
+and every rank then runs the delta, MaxPool1D, mask, top-K and compaction on
+the same numbers, so all ranks keep the same tokens.
+
+All arithmetic runs in the library's kernels; this module only slices the work
+and issues the collective through torch.distributed (NCCL on GPUs).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (Workspace, focus_attn_stats, focus_compact, focus_importance_delta,
+               focus_topk_select, make_dims)
+
+
+def shard_heads(Hq: int, Hkv: int, rank: int, world: int) -> tuple[slice, slice]:
+    """The query-head and kv-head slices rank `rank` owns (kv heads split evenly, each
+    with its G = Hq/Hkv query heads)."""
+    if Hkv % world:
+        raise ValueError(f"Hkv = {Hkv} does not split over {world} ranks")
+    G = Hq // Hkv
+    kv = Hkv // world
+    return slice(rank * kv * G, (rank + 1) * kv * G), slice(rank * kv, (rank + 1) * kv)
+
+
+def partial_importance(R, B, Hq_local, Hkv_local, d, q0, k0_prefix, k0_block, q1, k1_prefix,
+                       k1_block, cu_prefix, softmax_scale, out=None, ws=None, stream=None):
+    """[2, R, B] float32: this rank's share of I0 and I1 (its heads only)."""
+    dims = make_dims(R, B, Hq_local, Hkv_local, d, 8, softmax_scale)
+    if ws is None:
+        ws = Workspace(dims, q1.device, stream)
+    if out is None:
+        out = torch.empty(2, R, B, dtype=torch.float32, device=q1.device)
+    focus_attn_stats(dims, q0, k0_prefix, cu_prefix, k0_block, out[0], ws, stream)
+    focus_attn_stats(dims, q1, k1_prefix, cu_prefix, k1_block, out[1], ws, stream)
+    return out
+
+
+def finish_from_importance(dims, importance, decoded, budget, hidden, kept_idx, cu_seqlens,
+                           packed, ws=None, delta_out=None, stream=None):
+    """Delta, MaxPool1D, mask, top-K and compaction from the summed [2, R, B] importance."""
+    if ws is None:
+        ws = Workspace(dims, importance.device, stream)
+    delta = delta_out if delta_out is not None else torch.empty_like(importance[0])
+    focus_importance_delta(dims, importance[0], importance[1], decoded, delta, stream=stream)
+    focus_topk_select(dims, delta, decoded, budget, kept_idx, cu_seqlens, ws, stream)
+    focus_compact(dims, hidden, kept_idx, cu_seqlens, packed, ws, stream)
+    return ws
+
+
+def evict_head_sharded(dims, rank, world, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block,
+                       cu_prefix, hidden, decoded, budget, kept_idx, cu_seqlens, packed,
+                       group=None, delta_out=None, stream=None):
+    """The fused step on one rank of a head-sharded group.  `dims` holds the full head
+    counts; q*/k* are this rank's slices (shard_heads); the other arguments are the
+    full per-request tensors, identical on every rank.  One all-reduce."""
+    world_heads = dims.Hq // world, dims.Hkv // world
+    part = partial_importance(dims.R, dims.B, world_heads[0], world_heads[1], dims.head_dim, q0,
+                              k0_prefix, k0_block, q1, k1_prefix, k1_block, cu_prefix,
+                              dims.softmax_scale, stream=stream)
+    if world > 1:
+        torch.distributed.all_reduce(part, op=torch.distributed.ReduceOp.SUM, group=group)
+    return finish_from_importance(dims, part, decoded, budget, hidden, kept_idx, cu_seqlens,
+                                  packed, delta_out=delta_out, stream=stream)

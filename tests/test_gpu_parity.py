@@ -487,3 +487,75 @@ def test_dynamic_budget_vs_oracle(case, constraints, orc):
         check_selection(kept_h, cu_h, ref["pooled"], dec, kg)
     check_packed(packed[:int(cu_h[-1])].view(torch.int16).cpu().numpy().view(np.uint16), kept_h,
                  cu_h, hidden_bits(p))
+
+
+def test_head_sharded_two_way_matches_fused(orc):
+    """Tensor-parallel head sharding, emulated on one GPU: two head shards' partial
+    importance summed (the all-reduce), then delta/select/compaction, give the fused
+    step's results within tolerance and the oracle's selection."""
+    import attention_delta_token_b200 as F
+    from attention_delta_token_b200 import parallel
+    p = synth.make_problem(1, seed=800, wide_logits=True, overrides=dict(R=10))
+    g = p.to("cuda")
+    world = 2
+    parts = []
+    for rank in range(world):
+        hq, hk = parallel.shard_heads(p.Hq, p.Hkv, rank, world)
+        parts.append(parallel.partial_importance(
+            p.R, p.B, p.Hq // world, p.Hkv // world, p.d,
+            g.q0[:, :, hq].contiguous(), g.k0_prefix[:, hk].contiguous(),
+            g.k0_block[:, :, hk].contiguous(), g.q1[:, :, hq].contiguous(),
+            g.k1_prefix[:, hk].contiguous(), g.k1_block[:, :, hk].contiguous(), g.cu_prefix,
+            p.scale))
+    total = parts[0] + parts[1]  # what the all-reduce computes
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+    cap = F.plan_capacity(p.decoded, p.budget)
+    kept = torch.empty(cap, dtype=torch.int32, device="cuda")
+    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+    packed = torch.empty(cap, p.H, dtype=torch.bfloat16, device="cuda")
+    delta = torch.empty(p.R, p.B, device="cuda")
+    ws = parallel.finish_from_importance(dims, total, g.decoded, g.budget, g.hidden, kept, cu,
+                                         packed, delta_out=delta)
+    assert F.focus_read_device_status(ws) == 0
+    fused = run_evict(g)
+    assert_close_importance(total[0].cpu().numpy(), fused["i0"], "I0 sharded vs fused")
+    assert_close_importance(total[1].cpu().numpy(), fused["i1"], "I1 sharded vs fused")
+    ref = orc.evict(p)
+    assert_close_delta(delta.cpu().numpy(), ref["pooled"])
+    check_selection(kept.cpu().numpy(), cu.cpu().numpy(), ref["pooled"], p.decoded.numpy(),
+                    p.budget.numpy())
+    check_packed(packed.view(torch.int16).cpu().numpy().view(np.uint16), kept.cpu().numpy(),
+                 cu.cpu().numpy(), hidden_bits(p))
+
+
+EDGE_CASES = {
+    # more than 1024 requests: the planner orders them with a bitonic sort
+    "r1500_tiny_heads": (0, dict(R=1500, B=8, Hq=2, Hkv=1, d=64, H=64, prefix=("uniform", 0, 200),
+                                 decoded=("uniform", 0.0, 0.5), lift=("frac", 0.2),
+                                 budget=("ceil", 0.3))),
+    # one very long prefix: 157 key tiles in one work item
+    "long_prefix_20k": (1, dict(R=2, prefix=("uniform", 19000, 20000))),
+    # multi-query attention: all 32 query heads read one kv head (4 tokens per row tile)
+    "mqa_g32": (1, dict(R=3, Hq=32, Hkv=1, prefix=("uniform", 0, 400))),
+    # d = 64 with 16 query heads per kv head
+    "d64_g16": (1, dict(R=4, d=64, Hq=32, Hkv=2, prefix=("uniform", 0, 300))),
+}
+
+
+@pytest.mark.parametrize("case", sorted(EDGE_CASES))
+def test_edge_shapes_vs_oracle(case, orc):
+    cfg, ov = EDGE_CASES[case]
+    p = synth.make_problem(cfg, seed=900 + sorted(EDGE_CASES).index(case), wide_logits=True,
+                           overrides=ov)
+    req = list(range(p.R)) if p.R <= 64 else _sample_requests(p, n=40)
+    ref = orc.evict(p.subset(req))
+    out = run_evict(p.to("cuda"))
+    assert out["status"] == 0
+    assert_close_importance(out["i0"][req], ref["i0"], "I0")
+    assert_close_importance(out["i1"][req], ref["i1"], "I1")
+    assert_close_delta(out["delta"][req], ref["pooled"])
+    _, cu_all, _ = orc.select(np.zeros((p.R, p.B)), p.decoded, p.budget)
+    np.testing.assert_array_equal(out["cu_seqlens"], cu_all)
+    check_selection(out["kept"], out["cu_seqlens"], ref["pooled"], p.decoded.numpy(),
+                    p.budget.numpy(), requests=req)
+    check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))

@@ -1,7 +1,9 @@
 """The N > 1 host logic of the benchmark, on CPU with gloo ranks (world size 2).
 
 The eviction path shards by request: every rank runs its own batch and the only
-cross-rank steps are the barrier and the max-over-ranks of the timed region.
+cross-rank steps are the barrier and the max-over-ranks of the timed region.  The
+head-sharded (tensor-parallel) variant adds one all-reduce of the partial
+importance, checked here against the oracle's importance over all heads.
 """
 import json
 import os
@@ -77,3 +79,75 @@ def test_reference_arm_under_torchrun_prints_once():
     assert d["impl"] == "reference" and d["unit"] == "blocks/s" and d["value"] > 0
     assert d["n_gpus"] == 2 and d["steps"] == 3
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_shard_heads_partitions_the_heads():
+    from attention_delta_token_b200.parallel import shard_heads
+    for Hq, Hkv, world in ((32, 8, 2), (32, 8, 4), (32, 8, 8), (32, 4, 4), (8, 8, 2)):
+        G = Hq // Hkv
+        seen_q, seen_k = [], []
+        for r in range(world):
+            hq, hk = shard_heads(Hq, Hkv, r, world)
+            q = list(range(Hq))[hq]
+            k = list(range(Hkv))[hk]
+            assert q == [h for h in range(Hq) if h // G in k]  # each query head with its kv head
+            seen_q += q
+            seen_k += k
+        assert seen_q == list(range(Hq)) and seen_k == list(range(Hkv))
+    with pytest.raises(ValueError):
+        shard_heads(32, 8, 0, 3)
+
+
+def _tp_worker(rank, world, port, out_dir):
+    """One rank of a head-sharded group on CPU: its partial importance comes from the
+    oracle on its own head slice; the library call that follows the all-reduce is
+    replaced by a recorder (no GPU here)."""
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        import synth
+        from attention_delta_token_b200 import make_dims, parallel
+        p = synth.make_problem(0, seed=77, overrides=dict(R=3, Hq=8, Hkv=4))
+        hq, hk = parallel.shard_heads(p.Hq, p.Hkv, rank, world)
+
+        def partial(R, B, Hq_l, Hkv_l, d, q0, k0p, k0b, q1, k1p, k1b, cu, scale, **kw):
+            i = [oracle.importance(q, kp, cu, kb, Hq=Hq_l, Hkv=Hkv_l, scale=scale)
+                 for q, kp, kb in ((q0, k0p, k0b), (q1, k1p, k1b))]
+            return torch.tensor(np.stack(i), dtype=torch.float32)
+
+        seen = {}
+
+        def finish(dims, importance, *a, **kw):
+            seen["importance"] = importance.clone()
+
+        parallel.partial_importance = partial
+        parallel.finish_from_importance = finish
+        dims = make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale)
+        parallel.evict_head_sharded(
+            dims, rank, world, p.q0[:, :, hq].contiguous(), p.k0_prefix[:, hk].contiguous(),
+            p.k0_block[:, :, hk].contiguous(), p.q1[:, :, hq].contiguous(),
+            p.k1_prefix[:, hk].contiguous(), p.k1_block[:, :, hk].contiguous(), p.cu_prefix,
+            p.hidden, p.decoded, p.budget, None, None, None)
+        full = [oracle.importance(q, kp, p.cu_prefix, kb, Hq=p.Hq, Hkv=p.Hkv, scale=p.scale)
+                for q, kp, kb in ((p.q0, p.k0_prefix, p.k0_block), (p.q1, p.k1_prefix, p.k1_block))]
+        np.save(os.path.join(out_dir, f"tp{rank}.npy"), seen["importance"].numpy())
+        np.save(os.path.join(out_dir, "tp_full.npy"), np.stack(full))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gloo_world2_head_sharded_importance_sums_to_the_full():
+    """I_j sums over heads, so the all-reduced per-rank importances equal the oracle's
+    importance over all heads, and every rank holds the same numbers before selecting."""
+    import tempfile
+    world = 2
+    with tempfile.TemporaryDirectory() as d:
+        mp.start_processes(_tp_worker, args=(world, _free_port(), d), nprocs=world, join=True,
+                           start_method="spawn")
+        got = [np.load(os.path.join(d, f"tp{r}.npy")) for r in range(world)]
+        full = np.load(os.path.join(d, "tp_full.npy"))
+    np.testing.assert_array_equal(got[0], got[1])
+    np.testing.assert_allclose(got[0], full, rtol=2e-6, atol=1e-6)
+    assert (full > 0).all()
