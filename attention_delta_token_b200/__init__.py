@@ -24,7 +24,7 @@ __all__ = [
     "focus_importance_delta", "focus_topk_select", "focus_compact", "focus_evict",
     "focus_status_string", "focus_abi_version", "focus_set_trace_events", "plan_capacity",
     "focus_evict_static_scratch", "STATIC_SCRATCH_BYTES", "focus_selftest_wait_timeout",
-    "LIB_PATH", "STATUS",
+    "focus_partial_importance", "focus_evict_from_importance", "LIB_PATH", "STATUS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfocus.so")
@@ -100,6 +100,8 @@ def _load() -> ctypes.CDLL:
         "focus_evict_with_lse0": (ctypes.c_int, [D, P, P, P, P, P, P, P, i64, P, P, P, P, P, P,
                                                  i64, P, P, P, P, sz, P]),
         "focus_evict_ex": (ctypes.c_int, [D, ctypes.POINTER(FocusEvictArgs)]),
+        "focus_partial_importance": (ctypes.c_int, [D, P, P, P, P, P, P, P, i64, P, P, sz, P]),
+        "focus_evict_from_importance": (ctypes.c_int, [D, P, P, P, P, P, P, P, i64, P, P, sz, P]),
         "focus_evict_paged": (ctypes.c_int, [D, P, P, P, P, P, P, P, ctypes.c_int32, P,
                                              ctypes.c_int32, ctypes.c_int32, P, P, P, P, P, P, i64,
                                              P, P, P, P, sz, P]),
@@ -248,6 +250,37 @@ def focus_evict(dims, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block, cu_prefi
         _ptr(packed, bf, "packed"), int(packed.shape[0]),
         _ptr(delta_out, f32, "delta_out"), _ptr(i0_out, f32, "i0_out"),
         _ptr(i1_out, f32, "i1_out"), ws.ptr, ws.nbytes, _stream(stream)), "focus_evict")
+
+
+def focus_partial_importance(dims, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block, cu_prefix,
+                             importance, ws: Workspace, stream=None):
+    """Both layers' importance over the heads in `dims` into importance [2, R, B] float32
+    (I0, I1); the first half of focus_evict, for head-sharded (tensor-parallel) ranks."""
+    bf = torch.bfloat16
+    if importance.shape != (2, dims.R, dims.B):
+        raise ValueError(f"importance must be [2, {dims.R}, {dims.B}]")
+    _ok(_lib.focus_partial_importance(
+        ctypes.byref(dims), _ptr(q0, bf, "q0"), _ptr(k0_prefix, bf, "k0_prefix"),
+        _ptr(k0_block, bf, "k0_block"), _ptr(q1, bf, "q1"), _ptr(k1_prefix, bf, "k1_prefix"),
+        _ptr(k1_block, bf, "k1_block"), _ptr(cu_prefix, torch.int32, "cu_prefix"),
+        int(k1_prefix.shape[0]), _ptr(importance, torch.float32, "importance"), ws.ptr,
+        ws.nbytes, _stream(stream)), "focus_partial_importance")
+
+
+def focus_evict_from_importance(dims, importance, hidden, decoded, budget, kept_idx, cu_seqlens,
+                                packed, ws: Workspace, delta_out=None, stream=None):
+    """Delta, MaxPool1D, mask, top-K and compaction from importance [2, R, B] float32; the
+    second half of focus_evict."""
+    bf = torch.bfloat16
+    if importance.shape != (2, dims.R, dims.B):
+        raise ValueError(f"importance must be [2, {dims.R}, {dims.B}]")
+    _ok(_lib.focus_evict_from_importance(
+        ctypes.byref(dims), _ptr(importance, torch.float32, "importance"),
+        _ptr(hidden, bf, "hidden"), _ptr(decoded, torch.uint8, "decoded"),
+        _ptr(budget, torch.int32, "budget"), _ptr(kept_idx, torch.int32, "kept_idx"),
+        _ptr(cu_seqlens, torch.int32, "cu_seqlens"), _ptr(packed, bf, "packed"),
+        int(packed.shape[0]), _ptr(delta_out, torch.float32, "delta_out"), ws.ptr, ws.nbytes,
+        _stream(stream)), "focus_evict_from_importance")
 
 
 def focus_evict_with_lse0(dims, lse0, q0, k0_block, q1, k1_prefix, k1_block, cu_prefix, hidden,

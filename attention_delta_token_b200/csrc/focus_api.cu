@@ -271,7 +271,7 @@ focus_status_t focus_attn_stats(const focus_dims_t *dims, const void *q, const v
     pp.B = d.B;
     FOCUS_CUDA(focus::launch_plan(pp, s));
     FOCUS_CUDA(launch_attn_traced(p, d.head_dim, s));
-    focus::ReduceParams rp{p.partial, importance, d.R, d.B, d.Hkv, p.MT};
+    focus::ReduceParams rp{p.partial, importance, d.R, d.B, d.Hkv, p.MT, 1};
     FOCUS_CUDA(focus::launch_reduce(rp, s));
     return FOCUS_OK;
 }
@@ -394,6 +394,79 @@ focus_status_t check_paging(const Paging &pg) {
     return FOCUS_OK;
 }
 
+// The selection half of the step, behind the kernel that produced the column
+// sums: selection per request, then the row copy spread over the whole GPU, each
+// launched with programmatic dependent launch.  With constraints or a dynamic
+// budget the kept counts depend on the data, so the selection writes per-request
+// lists, cu_seqlens is scanned afterwards and the copy reads the lists; otherwise
+// the planner has already written cu_seqlens.
+struct Tail {
+    const float *partial;  // [layers][R][groups][B] column sums
+    int groups;            // summed per request: Hkv x row tiles, or 1 for a given importance
+    int layers;            // 2: rank by I1 - I0; 1: by I1 alone
+    uint32_t *status;
+    const void *hidden;
+    const uint8_t *decoded;
+    const int32_t *budget;
+    const float *decode_avg;
+    float budget_alpha;
+    int32_t *budget_out;
+    int32_t *kept_idx;
+    int32_t *cu_seqlens;
+    void *packed;
+    int64_t capacity;
+    float *delta_out, *i0_out, *i1_out;
+};
+
+bool tail_uses_lists(const focus_dims_t &d, const Tail &t) {
+    return d.constraints != 0 || t.decode_avg != nullptr;
+}
+
+focus_status_t launch_tail(const focus_dims_t &d, const Tail &t, uint8_t *ws, cudaStream_t s) {
+    focus::SelectParams sp;
+    memset(&sp, 0, sizeof sp);
+    sp.partial = t.partial;
+    sp.decoded = t.decoded;
+    sp.cu_seqlens = t.cu_seqlens;
+    sp.kept_idx = t.kept_idx;
+    sp.delta_out = t.delta_out;
+    sp.i0_out = t.i0_out;
+    sp.i1_out = t.i1_out;
+    sp.status = t.status;
+    sp.capacity = t.capacity;
+    sp.R = d.R;
+    sp.B = d.B;
+    sp.Hkv = t.groups;
+    sp.MT = 1;
+    sp.H = d.hidden;
+    sp.pool_window = d.pool_window;
+    sp.layers = t.layers;
+    if (tail_uses_lists(d, t)) {
+        const WsLayout w = ws_layout(d);
+        sp.constraints = d.constraints;
+        sp.budget = t.budget;
+        sp.decode_avg = t.decode_avg;
+        sp.budget_alpha = t.budget_alpha;
+        sp.budget_out = t.budget_out;
+        sp.lists = reinterpret_cast<int32_t *>(ws + w.lists);
+        sp.counts = reinterpret_cast<int32_t *>(ws + w.counts);
+        FOCUS_CUDA(focus::launch_select_compact(sp, s, /*pdl=*/true));
+        focus::ScanParams sc{sp.counts, t.cu_seqlens, t.status, t.capacity, d.R};
+        FOCUS_CUDA(focus::launch_scan(sc, s, /*pdl=*/true));
+        focus::CompactParams cp{static_cast<const uint16_t *>(t.hidden), nullptr, t.cu_seqlens,
+                                static_cast<uint16_t *>(t.packed), t.status, t.capacity, d.R, d.B,
+                                d.hidden, sp.lists, t.kept_idx};
+        FOCUS_CUDA(focus::launch_compact(cp, s, /*pdl=*/true));
+        return FOCUS_OK;
+    }
+    FOCUS_CUDA(focus::launch_select_compact(sp, s, /*pdl=*/true));
+    focus::CompactParams cp{static_cast<const uint16_t *>(t.hidden), t.kept_idx, t.cu_seqlens,
+                            static_cast<uint16_t *>(t.packed), t.status, t.capacity, d.R, d.B,
+                            d.hidden, nullptr, nullptr};
+    FOCUS_CUDA(focus::launch_compact(cp, s, /*pdl=*/true));
+    return FOCUS_OK;
+}
+
 focus_status_t evict_impl(const focus_dims_t *dims, const focus_evict_args_t &x) {
     FOCUS_TRY(check_dims(dims));
     const focus_dims_t &d = *dims;
@@ -487,49 +560,10 @@ focus_status_t evict_impl(const focus_dims_t *dims, const focus_evict_args_t &x)
     FOCUS_CUDA(focus::launch_plan(pp, s));
     FOCUS_CUDA(launch_attn_traced(p, d.head_dim, s, /*pdl=*/true));
 
-    // Selection per request, then the row copy spread over the whole GPU.
-    focus::SelectParams sp;
-    memset(&sp, 0, sizeof sp);
-    sp.partial = p.partial;
-    sp.decoded = x.decoded;
-    sp.cu_seqlens = x.cu_seqlens;
-    sp.kept_idx = x.kept_idx;
-    sp.delta_out = x.delta_out;
-    sp.i0_out = x.i0_out;
-    sp.i1_out = x.i1_out;
-    sp.status = p.status;
-    sp.capacity = x.capacity;
-    sp.R = d.R;
-    sp.B = d.B;
-    sp.Hkv = d.Hkv;
-    sp.MT = p.MT;
-    sp.H = d.hidden;
-    sp.pool_window = d.pool_window;
-    sp.layers = layer1_only ? 1 : 2;
-    if (lists) {
-        const WsLayout w = ws_layout(d);
-        sp.constraints = d.constraints;
-        sp.budget = x.budget;
-        sp.decode_avg = x.decode_avg;
-        sp.budget_alpha = x.budget_alpha;
-        sp.budget_out = x.budget_out;
-        sp.lists = reinterpret_cast<int32_t *>(ws + w.lists);
-        sp.counts = reinterpret_cast<int32_t *>(ws + w.counts);
-        FOCUS_CUDA(focus::launch_select_compact(sp, s, /*pdl=*/true));
-        focus::ScanParams sc{sp.counts, x.cu_seqlens, p.status, x.capacity, d.R};
-        FOCUS_CUDA(focus::launch_scan(sc, s, /*pdl=*/true));
-        focus::CompactParams cp{static_cast<const uint16_t *>(x.hidden), nullptr, x.cu_seqlens,
-                                static_cast<uint16_t *>(x.packed), p.status, x.capacity, d.R, d.B,
-                                d.hidden, sp.lists, x.kept_idx};
-        FOCUS_CUDA(focus::launch_compact(cp, s, /*pdl=*/true));
-        return FOCUS_OK;
-    }
-    FOCUS_CUDA(focus::launch_select_compact(sp, s, /*pdl=*/true));
-    focus::CompactParams cp{static_cast<const uint16_t *>(x.hidden), x.kept_idx, x.cu_seqlens,
-                            static_cast<uint16_t *>(x.packed), p.status, x.capacity, d.R, d.B,
-                            d.hidden, nullptr, nullptr};
-    FOCUS_CUDA(focus::launch_compact(cp, s, /*pdl=*/true));
-    return FOCUS_OK;
+    Tail t{p.partial, d.Hkv * p.MT, layer1_only ? 1 : 2, p.status, x.hidden, x.decoded,
+           x.budget, x.decode_avg, x.budget_alpha, x.budget_out, x.kept_idx, x.cu_seqlens,
+           x.packed, x.capacity, x.delta_out, x.i0_out, x.i1_out};
+    return launch_tail(d, t, ws, s);
 }
 
 }  // namespace
@@ -647,6 +681,93 @@ focus_status_t focus_evict_paged(const focus_dims_t *dims, const void *q0, const
     x.workspace_bytes = workspace_bytes;
     x.stream = stream;
     return evict_impl(dims, x);
+}
+
+focus_status_t focus_partial_importance(const focus_dims_t *dims, const void *q0,
+                                        const void *k0_prefix, const void *k0_block,
+                                        const void *q1, const void *k1_prefix,
+                                        const void *k1_block, const int32_t *cu_prefix,
+                                        int64_t total_prefix, float *importance, void *workspace,
+                                        size_t workspace_bytes, void *stream) {
+    FOCUS_TRY(check_dims(dims));
+    const focus_dims_t &d = *dims;
+    const bool layer1_only = d.score == FOCUS_SCORE_LAYER1;
+    if (!layer1_only)
+        FOCUS_TRY(check_attn_inputs(d, q0, k0_prefix, cu_prefix, total_prefix, k0_block));
+    FOCUS_TRY(check_attn_inputs(d, q1, k1_prefix, cu_prefix, total_prefix, k1_block));
+    FOCUS_TRY(check_ptr(importance, 4));
+    FOCUS_TRY(check_ws(d, workspace, workspace_bytes));
+    FOCUS_TRY(get_encoder());
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+
+    AttnParams p;
+    memset(&p, 0, sizeof p);
+    const int layers = layer1_only ? 1 : 2;
+    fill_common(p, d, cu_prefix, total_prefix, ws, layers);
+    if (layer1_only) {
+        FOCUS_TRY(encode_layer(p, 0, d, q1, k1_prefix, total_prefix, k1_block));
+        p.tm_q[1] = p.tm_q[0];
+        p.tm_kp[1] = p.tm_kp[0];
+        p.tm_kb[1] = p.tm_kb[0];
+    } else {
+        FOCUS_TRY(encode_layer(p, 0, d, q0, k0_prefix, total_prefix, k0_block));
+        FOCUS_TRY(encode_layer(p, 1, d, q1, k1_prefix, total_prefix, k1_block));
+    }
+    focus::PlanParams pp;
+    memset(&pp, 0, sizeof pp);
+    pp.cu_prefix = cu_prefix;
+    pp.order = const_cast<int32_t *>(p.order);
+    pp.status = p.status;
+    pp.R = d.R;
+    pp.B = d.B;
+    FOCUS_CUDA(focus::launch_plan(pp, s));
+    FOCUS_CUDA(launch_attn_traced(p, d.head_dim, s, /*pdl=*/true));
+    float *out = layer1_only ? importance + static_cast<size_t>(d.R) * d.B : importance;
+    focus::ReduceParams rp{p.partial, out, d.R, d.B, d.Hkv, p.MT, layers};
+    FOCUS_CUDA(focus::launch_reduce(rp, s, /*pdl=*/true));
+    return FOCUS_OK;
+}
+
+focus_status_t focus_evict_from_importance(const focus_dims_t *dims, const float *importance,
+                                           const void *hidden, const uint8_t *decoded,
+                                           const int32_t *budget, int32_t *kept_idx,
+                                           int32_t *cu_seqlens, void *packed, int64_t capacity,
+                                           float *delta_out, void *workspace,
+                                           size_t workspace_bytes, void *stream) {
+    FOCUS_TRY(check_dims(dims));
+    const focus_dims_t &d = *dims;
+    FOCUS_TRY(check_ptr(importance, 4));
+    FOCUS_TRY(check_ptr(hidden, 16));
+    FOCUS_TRY(check_ptr(decoded, 1));
+    FOCUS_TRY(check_ptr(budget, 4));
+    FOCUS_TRY(check_ptr(cu_seqlens, 4));
+    if (capacity < 0) return FOCUS_ERR_INVALID_ARGUMENT;
+    if (capacity > 0) {
+        FOCUS_TRY(check_ptr(kept_idx, 4));
+        FOCUS_TRY(check_ptr(packed, 16));
+    }
+    if (delta_out) FOCUS_TRY(check_ptr(delta_out, 4));
+    FOCUS_TRY(check_ws(d, workspace, workspace_bytes));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws + ws_layout(d).status);
+
+    const bool layer1_only = d.score == FOCUS_SCORE_LAYER1;
+    Tail t{layer1_only ? importance + static_cast<size_t>(d.R) * d.B : importance, 1,
+           layer1_only ? 1 : 2, status, hidden, decoded, budget, nullptr, 0.f, nullptr,
+           kept_idx, cu_seqlens, packed, capacity, delta_out, nullptr, nullptr};
+    focus::PlanParams pp;
+    memset(&pp, 0, sizeof pp);
+    pp.decoded = decoded;
+    pp.budget = budget;
+    pp.cu_seqlens = tail_uses_lists(d, t) ? nullptr : cu_seqlens;
+    pp.status = status;
+    pp.capacity = capacity;
+    pp.R = d.R;
+    pp.B = d.B;
+    FOCUS_CUDA(focus::launch_plan(pp, s));
+    return launch_tail(d, t, ws, s);
 }
 
 const char *focus_status_string(focus_status_t st) {

@@ -130,11 +130,11 @@ struct DeltaParams {
 cudaError_t launch_delta(const DeltaParams &p, cudaStream_t stream);
 
 struct ReduceParams {
-    const float *partial;  // [R][Hkv][MT][B]
-    float *importance;     // [R,B]
-    int R, B, Hkv, MT;
+    const float *partial;  // [layers][R][Hkv][MT][B]
+    float *importance;     // [layers][R][B]
+    int R, B, Hkv, MT, layers;
 };
-cudaError_t launch_reduce(const ReduceParams &p, cudaStream_t stream);
+cudaError_t launch_reduce(const ReduceParams &p, cudaStream_t stream, bool pdl = false);
 
 struct CompactParams {
     const uint16_t *hidden;    // null: write kept_idx from lists only, copy nothing

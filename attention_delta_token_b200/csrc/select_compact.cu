@@ -346,14 +346,17 @@ __global__ void __launch_bounds__(128) delta_kernel(const DeltaParams p) {
     if (j < B) p.delta[rb + j] = pool_mask(raw_s, dec_s, B, p.pool_window, j);
 }
 
-// importance[r][j] = sum over kv heads and row tiles (fixed order) of the column sums.
+// importance[l][r][j] = sum over kv heads and row tiles (fixed order) of layer l's
+// column sums; one block per (request, layer).
 __global__ void __launch_bounds__(128) reduce_kernel(const ReduceParams p) {
-    const int r = blockIdx.x, j = threadIdx.x, B = p.B;
+    pdl_wait();  // the column sums come from the attention kernel
+    const int r = blockIdx.x, l = blockIdx.y, j = threadIdx.x, B = p.B;
     if (j >= B) return;
     const size_t rb = static_cast<size_t>(r) * B;
+    const float *part = p.partial + static_cast<size_t>(l) * p.R * p.Hkv * p.MT * B;
     float s = 0.f;
-    for (int g = 0; g < p.Hkv * p.MT; ++g) s += p.partial[rb * p.Hkv * p.MT + static_cast<size_t>(g) * B + j];
-    p.importance[rb + j] = s;
+    for (int g = 0; g < p.Hkv * p.MT; ++g) s += part[rb * p.Hkv * p.MT + static_cast<size_t>(g) * B + j];
+    p.importance[static_cast<size_t>(l) * p.R * B + rb + j] = s;
 }
 
 // Stand-alone compaction: one warp per packed row, request found by binary search.
@@ -442,9 +445,8 @@ cudaError_t launch_delta(const DeltaParams &p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_reduce(const ReduceParams &p, cudaStream_t stream) {
-    reduce_kernel<<<p.R, 128, 0, stream>>>(p);
-    return cudaGetLastError();
+cudaError_t launch_reduce(const ReduceParams &p, cudaStream_t stream, bool pdl) {
+    return launch_kernel(reduce_kernel, dim3(p.R, p.layers), dim3(128), 0, stream, pdl, p);
 }
 
 cudaError_t launch_compact(const CompactParams &p, cudaStream_t stream, bool pdl) {

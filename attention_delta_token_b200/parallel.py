@@ -4,9 +4,9 @@ In a tensor-parallel engine each rank holds a contiguous slice of the query
 heads and of their kv heads.  I_j is a sum over heads ("What carries the
 argument": the column-wise sum of the attention the block's queries pay token
 j), so each rank computes the importance of its own heads for both layers with
-focus_attn_stats, one all-reduce (sum, fp32, 2 x R x B values) combines them,
-and every rank then runs the delta, MaxPool1D, mask, top-K and compaction on
-the same numbers, so all ranks keep the same tokens.
+focus_partial_importance, one all-reduce (sum, fp32, 2 x R x B values) combines
+them, and every rank then runs focus_evict_from_importance (delta, MaxPool1D,
+mask, top-K, compaction) on the same numbers, so all ranks keep the same tokens.
 
 All arithmetic runs in the library's kernels; this module only slices the work
 and issues the collective through torch.distributed (NCCL on GPUs).
@@ -15,8 +15,7 @@ from __future__ import annotations
 
 import torch
 
-from . import (Workspace, focus_attn_stats, focus_compact, focus_importance_delta,
-               focus_topk_select, make_dims)
+from . import Workspace, focus_evict_from_importance, focus_partial_importance, make_dims
 
 
 def shard_heads(Hq: int, Hkv: int, rank: int, world: int) -> tuple[slice, slice]:
@@ -30,27 +29,27 @@ def shard_heads(Hq: int, Hkv: int, rank: int, world: int) -> tuple[slice, slice]
 
 
 def partial_importance(R, B, Hq_local, Hkv_local, d, q0, k0_prefix, k0_block, q1, k1_prefix,
-                       k1_block, cu_prefix, softmax_scale, out=None, ws=None, stream=None):
-    """[2, R, B] float32: this rank's share of I0 and I1 (its heads only)."""
-    dims = make_dims(R, B, Hq_local, Hkv_local, d, 8, softmax_scale)
+                       k1_block, cu_prefix, softmax_scale, out=None, ws=None, stream=None, score=0):
+    """[2, R, B] float32: this rank's share of I0 and I1 (its heads only), from one
+    focus_partial_importance call (planner, attention over both layers, reduction)."""
+    dims = make_dims(R, B, Hq_local, Hkv_local, d, 8, softmax_scale, score=score)
     if ws is None:
         ws = Workspace(dims, q1.device, stream)
     if out is None:
         out = torch.empty(2, R, B, dtype=torch.float32, device=q1.device)
-    focus_attn_stats(dims, q0, k0_prefix, cu_prefix, k0_block, out[0], ws, stream)
-    focus_attn_stats(dims, q1, k1_prefix, cu_prefix, k1_block, out[1], ws, stream)
+    focus_partial_importance(dims, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block, cu_prefix,
+                             out, ws, stream)
     return out
 
 
 def finish_from_importance(dims, importance, decoded, budget, hidden, kept_idx, cu_seqlens,
                            packed, ws=None, delta_out=None, stream=None):
-    """Delta, MaxPool1D, mask, top-K and compaction from the summed [2, R, B] importance."""
+    """Delta, MaxPool1D, mask, top-K and compaction from the summed [2, R, B] importance
+    (focus_evict_from_importance).  Returns the workspace, whose status covers the call."""
     if ws is None:
         ws = Workspace(dims, importance.device, stream)
-    delta = delta_out if delta_out is not None else torch.empty_like(importance[0])
-    focus_importance_delta(dims, importance[0], importance[1], decoded, delta, stream=stream)
-    focus_topk_select(dims, delta, decoded, budget, kept_idx, cu_seqlens, ws, stream)
-    focus_compact(dims, hidden, kept_idx, cu_seqlens, packed, ws, stream)
+    focus_evict_from_importance(dims, importance, hidden, decoded, budget, kept_idx, cu_seqlens,
+                                packed, ws, delta_out=delta_out, stream=stream)
     return ws
 
 
@@ -63,7 +62,7 @@ def evict_head_sharded(dims, rank, world, q0, k0_prefix, k0_block, q1, k1_prefix
     world_heads = dims.Hq // world, dims.Hkv // world
     part = partial_importance(dims.R, dims.B, world_heads[0], world_heads[1], dims.head_dim, q0,
                               k0_prefix, k0_block, q1, k1_prefix, k1_block, cu_prefix,
-                              dims.softmax_scale, stream=stream)
+                              dims.softmax_scale, stream=stream, score=dims.score)
     if world > 1:
         torch.distributed.all_reduce(part, op=torch.distributed.ReduceOp.SUM, group=group)
     return finish_from_importance(dims, part, decoded, budget, hidden, kept_idx, cu_seqlens,

@@ -10,7 +10,9 @@ Default workload: SDAR-8B shape, 256 requests, B = 32, prefix lengths
 U[1024, 4096], Hq = 32, Hkv = 8, d = 128, hidden = 4096 (seeded synthetic bf16).
 N > 1 runs under torchrun, one rank per GPU; every rank processes its own batch
 (independent requests: weak scaling, no collective on the data path); the
-time is the max over ranks.  Prints one JSON line on rank 0.
+time is the max over ranks.  Prints one JSON line on rank 0.  --tp-shards S
+instead splits the heads S ways (the tensor-parallel form: one all-reduce of
+the partial importance per step under torchrun with N = S).
 
 --impl reference times the float64 CPU oracle (the checker the tests use) on
 the host cores, on bounded samples of the same workload.
@@ -18,6 +20,7 @@ the host cores, on bounded samples of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -233,7 +236,9 @@ def run_ours(args, rank, world, local_rank):
     if args.requests:
         cfg = synth.FocusConfig(**{**cfg.__dict__, "R": args.requests,
                                    "name": f"{cfg.name}_r{args.requests}"})
-    seed = rank_seed(args.config, rank)
+    tp = args.tp_shards
+    # head-sharded ranks all work on the same requests; request-sharded ones on their own
+    seed = rank_seed(args.config, 0 if tp > 1 else rank)
     p = synth.make_problem(cfg, seed=seed, device=dev)
     counts = algorithmic_counts(p, layers=1 if args.score else 2, lse0=args.lse0)
     dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, args.constraints,
@@ -245,7 +250,31 @@ def run_ours(args, rank, world, local_rank):
     in_bytes = sum(t.numel() * t.element_size() for t in p.tensors().values())
 
     layer0 = (None, None, None) if args.score else (p.q0, p.k0_prefix, p.k0_block)
-    if args.dynamic_budget:
+    tp_ws = None
+    if tp > 1:
+        # This rank's head slice: focus_partial_importance, the all-reduce of the
+        # [2, R, B] sums (NCCL, only with one rank per shard), then the shared selection.
+        from attention_delta_token_b200.parallel import shard_heads
+        hq, hk = shard_heads(p.Hq, p.Hkv, rank if world > 1 else 0, tp)
+        sl = {k: (v[:, :, hq] if k.startswith("q") else v[:, :, hk] if k.endswith("block")
+                  else v[:, hk]).contiguous()
+              for k, v in p.tensors().items() if k[:2] in ("q0", "q1", "k0", "k1")}
+        sdims = F.make_dims(p.R, p.B, p.Hq // tp, p.Hkv // tp, p.d, 8, p.scale, p.pool_window,
+                            0, args.score)
+        tp_ws = F.Workspace(sdims, dev)
+        imp = torch.empty(2, p.R, p.B, dtype=torch.float32, device=dev)
+        s_l0 = (None, None, None) if args.score else (sl["q0"], sl["k0_prefix"], sl["k0_block"])
+        counts = algorithmic_counts(dataclasses.replace(p, Hq=p.Hq // tp, Hkv=p.Hkv // tp),
+                                    layers=1 if args.score else 2)
+
+        def step():
+            F.focus_partial_importance(sdims, *s_l0, sl["q1"], sl["k1_prefix"], sl["k1_block"],
+                                       p.cu_prefix, imp, tp_ws)
+            if world > 1:
+                dist.all_reduce(imp)
+            F.focus_evict_from_importance(dims, imp, p.hidden, p.decoded, p.budget, kept, cu,
+                                          packed, ws)
+    elif args.dynamic_budget:
         # historical decoded-per-step averages: ~10% of a 32-token block per step
         # (Figure 2), drawn uniformly in [0, 0.2 B] per request
         gen = torch.Generator().manual_seed(seed)
@@ -310,9 +339,10 @@ def run_ours(args, rank, world, local_rank):
                 F.focus_set_trace_events(None, None)
         stop.record(stream)
         barrier()
-    status = F.focus_read_device_status(ws)
-    if status != 0:
-        raise RuntimeError(f"device status {F.focus_status_string(status)}")
+    for w in (ws, tp_ws) if tp_ws is not None else (ws,):
+        status = F.focus_read_device_status(w)
+        if status != 0:
+            raise RuntimeError(f"device status {F.focus_status_string(status)}")
     elapsed = start.elapsed_time(stop) / 1e3
     attn_s = sum(a.elapsed_time(b) for a, b in zip(ev_a, ev_b)) / 1e3 / len(traced)
     elapsed_max = max_over_ranks(elapsed, dev)
@@ -321,7 +351,8 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- end to end: pinned host inputs -> device, the C-ABI call, result -> host
     e2e = None
-    if not args.no_e2e and not (args.score or args.lse0 or args.page_size or args.dynamic_budget):
+    variant = args.score or args.lse0 or args.page_size or args.dynamic_budget or tp > 1
+    if not args.no_e2e and not variant:
         host = {k: v.to("cpu").pin_memory() for k, v in p.tensors().items()}
         dev_t = p.tensors()
         out_kept = torch.empty(kept.shape, dtype=kept.dtype).pin_memory()
@@ -367,10 +398,12 @@ def run_ours(args, rank, world, local_rank):
         clocks = sampler.summary()
         sm_hz = (clocks["sm_mhz"] or 1965.0) * 1e6
         result = {
-            "metric": METRIC, "value": job_throughput(world, p.R, step_s), "unit": UNIT,
+            "metric": METRIC,
+            "value": p.R / step_s if tp > 1 else job_throughput(world, p.R, step_s), "unit": UNIT,
             "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True, "scaling": "strong" if tp > 1 else "weak",
+            "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {
                 "workload": workload, "R": p.R, "B": p.B, "Hq": p.Hq, "Hkv": p.Hkv, "d": p.d,
@@ -378,7 +411,12 @@ def run_ours(args, rank, world, local_rank):
                 "seed": seed, "kept_rows": counts["kept_rows"],
                 "input_bytes_per_step": int(in_bytes),
                 "l2": f"no flush: {in_bytes / 2**30:.2f} GiB of inputs per step > 126 MB L2",
-                "accumulate": "fp32", "parallelism": f"dp{world} (request-sharded replicas)",
+                "accumulate": "fp32",
+                "parallelism": (f"dp{world} (request-sharded replicas)" if tp <= 1 else
+                                f"tp{tp} (head-sharded, NCCL all-reduce of 2 x R x B fp32)"
+                                if world > 1 else
+                                f"tp{tp} emulated: rank 0's head shard + the shared selection "
+                                "timed on one GPU, no all-reduce"),
                 "constraints": args.constraints, "score": args.score, "lse0": args.lse0,
                 "page_size": args.page_size, "dynamic_budget": args.dynamic_budget,
             },
@@ -386,9 +424,7 @@ def run_ours(args, rank, world, local_rank):
             "roofline": {
                 "bound": "hbm", "kernel": "attn_stats_kernel", "achieved": achieved,
                 "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": (read_traffic(workload)
-                            if not (args.score or args.lse0 or args.page_size
-                                    or args.dynamic_budget) else None),
+                "traffic": read_traffic(workload) if not variant else None,
                 "algorithmic_bytes_per_launch": counts["attn_bytes"],
                 "ms_per_launch": attn_s_max * 1e3, "peak_source": f"{peak_src} (hbm_gbs)",
                 "launches_timed": len(traced),
@@ -402,8 +438,9 @@ def run_ours(args, rank, world, local_rank):
                 "peaks": f"{peak_src}: hbm {hbm} GB/s, bf16 {tc} TFLOP/s",
             },
             "clocks": clocks,
-            # plan, attention statistics, select, (scan,) compact
-            "gpu_launches": (5 if args.constraints else 4) * args.steps,
+            # plan, attention statistics, select, (scan,) compact; split into two calls
+            # (tp): plan, attention, reduce + plan, select, (scan,) compact
+            "gpu_launches": ((5 if args.constraints else 4) + (2 if tp > 1 else 0)) * args.steps,
             "e2e": e2e,
             "impl": "ours",
         }
@@ -500,16 +537,25 @@ def main():
                          "(focus_evict_paged)")
     ap.add_argument("--dynamic-budget", action="store_true",
                     help="dynamic retention budget (focus_evict_ex with decode_avg)")
+    ap.add_argument("--tp-shards", type=int, default=1,
+                    help="head-sharded (tensor-parallel) step over this many head shards: under "
+                         "torchrun one rank per shard with an NCCL all-reduce; on one GPU rank "
+                         "0's share is timed")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.tp_shards > 1 and (args.lse0 or args.page_size or args.dynamic_budget):
+        ap.error("--tp-shards combines with --constraints and --score only")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if world > 1 and args.tp_shards > 1 and args.tp_shards != world:
+        ap.error("--tp-shards under torchrun needs one rank per shard (N = S)")
 
     if args.impl == "reference":
         if rank == 0:

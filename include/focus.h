@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define FOCUS_ABI_VERSION 3
+#define FOCUS_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define FOCUS_API __attribute__((visibility("default")))
@@ -302,6 +302,46 @@ FOCUS_API focus_status_t focus_evict_with_lse0(
     int64_t total_prefix, const void *hidden, const uint8_t *decoded, const int32_t *budget,
     int32_t *kept_idx, int32_t *cu_seqlens, void *packed, int64_t capacity, float *delta_out,
     float *i0_out, float *i1_out, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The two halves of the fused step, for tensor-parallel engines whose ranks each
+ * hold a slice of the heads.  I_j is a sum over query heads ("What carries the
+ * argument"), so each rank computes the importance of its own heads with
+ * focus_partial_importance, the ranks sum the [2, R, B] results (one all-reduce),
+ * and every rank runs focus_evict_from_importance on the same sums, so all ranks
+ * keep the same tokens.  (The pages run on one GPU; this split is a deployment
+ * variant of focus_evict.)
+ *
+ * focus_partial_importance: both layers' importance over the heads in `dims`
+ * (dims.Hq / dims.Hkv = this rank's head counts, the same G = Hq/Hkv as the
+ * model), with the layouts of focus_evict restricted to those heads:
+ *   importance [2, R, B] float32 out: importance[0] = I0, importance[1] = I1.
+ * With dims.score == FOCUS_SCORE_LAYER1 the layer-0 arguments may be NULL and
+ * importance[0] is left untouched.  dims.hidden is not used (any multiple of 8).
+ * The per-(request, kv head, row tile) column sums are reduced in a fixed
+ * order, so the result is deterministic and equals what focus_attn_stats gives
+ * for each layer.
+ */
+FOCUS_API focus_status_t focus_partial_importance(
+    const focus_dims_t *dims, const void *q0, const void *k0_prefix, const void *k0_block,
+    const void *q1, const void *k1_prefix, const void *k1_block, const int32_t *cu_prefix,
+    int64_t total_prefix, float *importance, void *workspace, size_t workspace_bytes,
+    void *stream);
+
+/*
+ * focus_evict_from_importance: delta (I1 - I0, or I1 alone with
+ * dims.score == FOCUS_SCORE_LAYER1), MaxPool1D, mask, top-K (with
+ * dims.constraints applied) and compaction from a given importance
+ * [2, R, B] float32 (importance[0] is not read for the layer-1 score).
+ * Outputs and their rules as in focus_evict; delta_out (nullable) receives the
+ * pooled, masked delta.  Given the importance focus_partial_importance computes
+ * over all heads, the outputs are bit-identical to focus_evict's.
+ */
+FOCUS_API focus_status_t focus_evict_from_importance(
+    const focus_dims_t *dims, const float *importance, const void *hidden,
+    const uint8_t *decoded, const int32_t *budget, int32_t *kept_idx, int32_t *cu_seqlens,
+    void *packed, int64_t capacity, float *delta_out, void *workspace, size_t workspace_bytes,
+    void *stream);
 
 /*
  * The fused step for callers that cannot allocate device memory.  (The FOCUS

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol():
 def test_status_strings_and_version():
     for code, name in F.STATUS.items():
         assert F.focus_status_string(code) == name
-    assert F.focus_abi_version() == 3
+    assert F.focus_abi_version() == 4
 
 
 def dims(**kw):
@@ -103,6 +103,10 @@ def test_bad_dims_rejected_everywhere(over, code):
     assert F._lib.focus_importance_delta(ctypes.byref(d), A, A, A, A, None, None) == code
     assert F._lib.focus_topk_select(ctypes.byref(d), A, A, A, A, A, 16, A, 1 << 20, None) == code
     assert F._lib.focus_compact(ctypes.byref(d), A, A, A, A, 16, A, 1 << 20, None) == code
+    assert F._lib.focus_partial_importance(ctypes.byref(d), A, A, A, A, A, A, A, 100, A, A,
+                                           1 << 20, None) == code
+    assert F._lib.focus_evict_from_importance(ctypes.byref(d), A, A, A, A, A, A, A, 16, None, A,
+                                              1 << 20, None) == code
 
 
 BAD_PTRS = [
@@ -197,3 +201,34 @@ def test_plan_capacity_matches_oracle_counts():
                                                    prefix=("fixed", 0)))
         _, cu, _ = oracle.select(np.zeros((p.R, p.B)), p.decoded, p.budget)
         assert F.plan_capacity(p.decoded, p.budget) == int(cu[-1])
+
+
+def test_split_entry_points_validation():
+    """focus_partial_importance / focus_evict_from_importance reject what focus_evict
+    rejects (host checks only; nothing is launched)."""
+    d = dims()
+    ws = F.focus_workspace_size(d)
+    L = F._lib
+
+    def partial(dd=d, q0=A, k0p=A, q1=A, imp=A, w=ws):
+        return L.focus_partial_importance(ctypes.byref(dd), q0, k0p, A, q1, A, A, A, 100, imp, A,
+                                          w, None)
+
+    def from_imp(dd=d, imp=A, hidden=A, budget=A, kept=A, packed=A, cap=16, delta=None, w=ws):
+        return L.focus_evict_from_importance(ctypes.byref(dd), imp, hidden, A, budget, kept, A,
+                                             packed, cap, delta, A, w, None)
+    assert partial(q0=None) == INVALID             # layer 0 needed for the delta score
+    assert partial(q1=A + 8) == INVALID
+    assert partial(imp=None) == INVALID
+    assert partial(imp=A + 2) == INVALID
+    assert partial(w=ws - 4) == WORKSPACE
+    assert partial(dd=dims(B=129)) == UNSUPPORTED
+    assert from_imp(imp=None) == INVALID
+    assert from_imp(hidden=A + 8) == INVALID
+    assert from_imp(budget=None) == INVALID
+    assert from_imp(kept=None) == INVALID
+    assert from_imp(packed=A + 8) == INVALID
+    assert from_imp(cap=-1) == INVALID
+    assert from_imp(delta=A + 1) == INVALID
+    assert from_imp(w=8) == WORKSPACE
+    assert from_imp(dd=dims(pool_window=2)) == UNSUPPORTED

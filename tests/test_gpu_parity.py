@@ -528,6 +528,50 @@ def test_head_sharded_two_way_matches_fused(orc):
                  cu.cpu().numpy(), hidden_bits(p))
 
 
+@pytest.mark.parametrize("constraints,score", [(0, 0), (3, 0), (0, 1), (3, 1)])
+def test_split_halves_bitwise_equal_fused(constraints, score):
+    """focus_partial_importance over all heads, then focus_evict_from_importance, give
+    the fused step's importance, delta, kept set and packed rows bit for bit (the same
+    column sums reduced in the same order); the importance also equals focus_attn_stats
+    per layer."""
+    import attention_delta_token_b200 as F
+    p = synth.make_problem(4, seed=810 + 2 * constraints + score, overrides=dict(R=12))
+    g = p.to("cuda")
+    fused = run_evict(g, constraints=constraints, score=score)
+    assert fused["status"] == 0
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, constraints,
+                       score)
+    ws = F.Workspace(dims, "cuda")
+    imp = torch.full((2, p.R, p.B), float("nan"), device="cuda")
+    l0 = (None, None, None) if score else (g.q0, g.k0_prefix, g.k0_block)
+    F.focus_partial_importance(dims, *l0, g.q1, g.k1_prefix, g.k1_block, g.cu_prefix, imp, ws)
+    cap = F.plan_capacity(p.decoded, p.budget, constraints)
+    kept = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+    packed = torch.zeros(cap, p.H, dtype=torch.bfloat16, device="cuda")
+    delta = torch.empty(p.R, p.B, device="cuda")
+    F.focus_evict_from_importance(dims, imp, g.hidden, g.decoded, g.budget, kept, cu, packed,
+                                  ws, delta_out=delta)
+    assert F.focus_read_device_status(ws) == 0
+    np.testing.assert_array_equal(imp[1].cpu().numpy(), fused["i1"].astype(np.float32))
+    if score:
+        assert torch.isnan(imp[0]).all()  # layer 0 untouched
+    else:
+        np.testing.assert_array_equal(imp[0].cpu().numpy(), fused["i0"].astype(np.float32))
+        one = torch.empty(p.R, p.B, device="cuda")
+        for layer, (q, kp, kb) in enumerate(((g.q0, g.k0_prefix, g.k0_block),
+                                             (g.q1, g.k1_prefix, g.k1_block))):
+            F.focus_attn_stats(dims, q, kp, g.cu_prefix, kb, one, ws)
+            assert torch.equal(one, imp[layer])
+    np.testing.assert_array_equal(delta.cpu().numpy(), fused["delta"].astype(np.float32))
+    cu_h = cu.cpu().numpy()
+    np.testing.assert_array_equal(cu_h, fused["cu_seqlens"])
+    n = int(cu_h[-1])
+    np.testing.assert_array_equal(kept[:n].cpu().numpy(), fused["kept"][:n])
+    np.testing.assert_array_equal(packed[:n].view(torch.int16).cpu().numpy().view(np.uint16),
+                                  fused["packed"][:n])
+
+
 EDGE_CASES = {
     # more than 1024 requests: the planner orders them with a bitonic sort
     "r1500_tiny_heads": (0, dict(R=1500, B=8, Hq=2, Hkv=1, d=64, H=64, prefix=("uniform", 0, 200),
