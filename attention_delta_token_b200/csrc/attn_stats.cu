@@ -8,8 +8,8 @@
 // keys followed by its B block keys; I_j also sums over the query heads.
 //
 // Work item = one (layer, request, kv head, 128-row query tile).  The kernel is
-// persistent: two CTAs per SM, each walking the items (longest prefix first) with
-// a stride of the grid size.  Per CTA (10 warps):
+// persistent: two CTAs per SM, each taking one item per round from the list
+// (longest prefix first), in snake order across the grid.  Per CTA (10 warps):
 //   warp 0      TMA producer: the item's Q tile (once per item, as soon as the
 //               previous item's MMAs have released it), then 128-key tiles of the
 //               prefix and finally the block keys, through a 2-stage ring;
@@ -91,6 +91,17 @@ __device__ __forceinline__ Item decode_item(const AttnParams &p, int it) {
     }
     w.n_pre = (w.L + kTileKeys - 1) / kTileKeys;
     return w;
+}
+
+// The work item a CTA takes in its k-th round.  Items come longest request first;
+// the rounds alternate direction across the grid (a snake), so the CTA that took
+// the longest item of one round takes the shortest of the next and the per-CTA
+// totals even out (a plain stride hands CTA 0 the longest item of every round).
+// Increasing in k for every CTA, so the first index past the end ends the loop.
+__device__ __forceinline__ int item_of_round(int k) {
+    const int g = static_cast<int>(gridDim.x);
+    const int c = static_cast<int>(blockIdx.x);
+    return k * g + ((k & 1) ? g - 1 - c : c);
 }
 
 // Loads 32 TMEM columns of this thread's lane into v[OFF .. OFF+31].
@@ -207,7 +218,7 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
             uint32_t kt = 0;   // key tiles issued by this CTA
             int last_q = -1;   // item count of the last Q load issued
             int k = 0;
-            for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++k) {
+            for (int it = item_of_round(0); it < n_items; it = item_of_round(++k)) {
                 const Item w = decode_item(p, it);
                 if (w.bad) atomicOr(p.status, FOCUS_DEV_BAD_INPUT);
                 if (!mbar_wait(q_empty, (k & 1) ^ 1, p.status, abort_flag)) break;
@@ -277,7 +288,7 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
             uint32_t st = 0;  // S tiles produced
             int k = 0;
             bool ok = true;
-            for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++k) {
+            for (int it = item_of_round(0); ok && it < n_items; it = item_of_round(++k)) {
                 const Item w = decode_item(p, it);
                 if (!mbar_wait(q_full, k & 1, p.status, abort_flag)) break;
                 for (int t = 0; t <= w.n_pre; ++t, ++kt, ++st) {
@@ -320,7 +331,7 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
         uint32_t st = 0;
         int k = 0;
         bool ok = true;
-        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++k) {
+        for (int it = item_of_round(0); ok && it < n_items; it = item_of_round(++k)) {
             const Item w = decode_item(p, it);
             const int rows_valid = min(kTileRows, p.G * p.B - w.mt * kTileRows);
             float m = -INFINITY;  // running max of the scaled logits (log2 domain), this half
