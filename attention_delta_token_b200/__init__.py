@@ -24,7 +24,9 @@ __all__ = [
     "focus_importance_delta", "focus_topk_select", "focus_compact", "focus_evict",
     "focus_status_string", "focus_abi_version", "focus_set_trace_events", "plan_capacity",
     "focus_evict_static_scratch", "STATIC_SCRATCH_BYTES", "focus_selftest_wait_timeout",
-    "focus_partial_importance", "focus_evict_from_importance", "LIB_PATH", "STATUS",
+    "focus_partial_importance", "focus_evict_from_importance", "FocusExchange",
+    "focus_exchange_buffer_size", "focus_partial_importance_push", "focus_evict_from_exchange",
+    "focus_selftest_exchange", "LIB_PATH", "STATUS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfocus.so")
@@ -74,6 +76,12 @@ class FocusEvictArgs(ctypes.Structure):
                 ("workspace_bytes", ctypes.c_size_t), ("stream", ctypes.c_void_p)]
 
 
+class FocusExchange(ctypes.Structure):
+    """focus_exchange_t: peer_buffers is a DEVICE array of the ranks' buffer pointers."""
+    _fields_ = [("peer_buffers", ctypes.c_void_p), ("rank", ctypes.c_int32),
+                ("world", ctypes.c_int32), ("epoch", ctypes.c_uint32)]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
@@ -102,6 +110,13 @@ def _load() -> ctypes.CDLL:
         "focus_evict_ex": (ctypes.c_int, [D, ctypes.POINTER(FocusEvictArgs)]),
         "focus_partial_importance": (ctypes.c_int, [D, P, P, P, P, P, P, P, i64, P, P, sz, P]),
         "focus_evict_from_importance": (ctypes.c_int, [D, P, P, P, P, P, P, P, i64, P, P, sz, P]),
+        "focus_exchange_buffer_size": (sz, [D, ctypes.c_int32]),
+        "focus_partial_importance_push": (ctypes.c_int, [D, P, P, P, P, P, P, P, i64,
+                                                         ctypes.POINTER(FocusExchange), P, sz, P]),
+        "focus_evict_from_exchange": (ctypes.c_int, [D, P, ctypes.c_int32, ctypes.c_uint32, P, P,
+                                                     P, P, P, P, i64, P, P, sz, P]),
+        "focus_selftest_exchange": (ctypes.c_int, [P, P, P, P, ctypes.c_int32, ctypes.c_int32,
+                                                   ctypes.c_int32, ctypes.c_uint32, P]),
         "focus_evict_paged": (ctypes.c_int, [D, P, P, P, P, P, P, P, ctypes.c_int32, P,
                                              ctypes.c_int32, ctypes.c_int32, P, P, P, P, P, P, i64,
                                              P, P, P, P, sz, P]),
@@ -178,6 +193,10 @@ def focus_workspace_size(dims: FocusDims) -> int:
 
 class Workspace:
     """Device scratch for one stream of calls (status word, request order, column sums)."""
+
+    @staticmethod
+    def size(dims: FocusDims) -> int:
+        return focus_workspace_size(dims)
 
     def __init__(self, dims: FocusDims, device="cuda", stream=None):
         self.nbytes = focus_workspace_size(dims)
@@ -281,6 +300,57 @@ def focus_evict_from_importance(dims, importance, hidden, decoded, budget, kept_
         _ptr(cu_seqlens, torch.int32, "cu_seqlens"), _ptr(packed, bf, "packed"),
         int(packed.shape[0]), _ptr(delta_out, torch.float32, "delta_out"), ws.ptr, ws.nbytes,
         _stream(stream)), "focus_evict_from_importance")
+
+
+def focus_exchange_buffer_size(dims, world: int) -> int:
+    n = int(_lib.focus_exchange_buffer_size(ctypes.byref(dims), int(world)))
+    if n == 0:
+        raise FocusError(1, "focus_exchange_buffer_size (invalid dims or world)")
+    return n
+
+
+def focus_partial_importance_push(dims, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block,
+                                  cu_prefix, peer_buffers, rank: int, world: int, epoch: int,
+                                  ws: Workspace, stream=None):
+    """focus_partial_importance whose [2, R, B] sums go to slot `rank` of every rank's exchange
+    buffer; peer_buffers: int64 CUDA tensor [world] of the buffers' device addresses."""
+    bf = torch.bfloat16
+    if peer_buffers.numel() != world:
+        raise ValueError("peer_buffers must hold one address per rank")
+    ex = FocusExchange(_ptr(peer_buffers, torch.int64, "peer_buffers"), int(rank), int(world),
+                       int(epoch))
+    _ok(_lib.focus_partial_importance_push(
+        ctypes.byref(dims), _ptr(q0, bf, "q0"), _ptr(k0_prefix, bf, "k0_prefix"),
+        _ptr(k0_block, bf, "k0_block"), _ptr(q1, bf, "q1"), _ptr(k1_prefix, bf, "k1_prefix"),
+        _ptr(k1_block, bf, "k1_block"), _ptr(cu_prefix, torch.int32, "cu_prefix"),
+        int(k1_prefix.shape[0]), ctypes.byref(ex), ws.ptr, ws.nbytes, _stream(stream)),
+        "focus_partial_importance_push")
+
+
+def focus_evict_from_exchange(dims, exchange_buffer, world: int, epoch: int, hidden, decoded,
+                              budget, kept_idx, cu_seqlens, packed, ws: Workspace,
+                              delta_out=None, stream=None):
+    """focus_evict_from_importance on the rank-ordered sum of this rank's exchange buffer
+    (uint8 CUDA tensor of focus_exchange_buffer_size bytes) for `epoch`."""
+    bf = torch.bfloat16
+    _ok(_lib.focus_evict_from_exchange(
+        ctypes.byref(dims), _ptr(exchange_buffer, torch.uint8, "exchange_buffer"), int(world),
+        int(epoch), _ptr(hidden, bf, "hidden"), _ptr(decoded, torch.uint8, "decoded"),
+        _ptr(budget, torch.int32, "budget"), _ptr(kept_idx, torch.int32, "kept_idx"),
+        _ptr(cu_seqlens, torch.int32, "cu_seqlens"), _ptr(packed, bf, "packed"),
+        int(packed.shape[0]), _ptr(delta_out, torch.float32, "delta_out"), ws.ptr, ws.nbytes,
+        _stream(stream)), "focus_evict_from_exchange")
+
+
+def focus_selftest_exchange(partials, buffer_ptrs, out, scratch, epoch: int, stream=None):
+    """The exchange protocol with world = partials.shape[0] ranks emulated in one cooperative
+    launch (see focus.h).  partials/out [world, 2, R, B] float32, buffer_ptrs int64 [world],
+    scratch int32/uint32-sized zeroed [>= 1 + world] (scratch[0] = status bits)."""
+    world, _, R, B = partials.shape
+    _ok(_lib.focus_selftest_exchange(
+        _ptr(partials, torch.float32, "partials"), _ptr(buffer_ptrs, torch.int64, "buffer_ptrs"),
+        _ptr(out, torch.float32, "out"), _ptr(scratch, torch.int32, "scratch"), int(R), int(B),
+        int(world), int(epoch), _stream(stream)), "focus_selftest_exchange")
 
 
 def focus_evict_with_lse0(dims, lse0, q0, k0_block, q1, k1_prefix, k1_block, cu_prefix, hidden,

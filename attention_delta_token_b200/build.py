@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfocus.so")
 SOURCES = ["focus_api.cu", "attn_stats.cu", "select_compact.cu", "focus_static_scratch.cu",
            "focus_selftest.cu"]
-HEADERS = ["focus_device.cuh", "focus_kernels.cuh"]
+HEADERS = ["focus_device.cuh", "focus_kernels.cuh", "focus_exchange.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -204,7 +204,8 @@ size_t focus_workspace_size(const focus_dims_t *dims) {
 focus_status_t focus_clear_device_status(void *workspace, size_t workspace_bytes, void *stream) {
     if (!workspace || !aligned(workspace, kAlign) || workspace_bytes < kAlign)
         return FOCUS_ERR_WORKSPACE;
-    FOCUS_CUDA(cudaMemsetAsync(workspace, 0, sizeof(uint32_t), static_cast<cudaStream_t>(stream)));
+    // The status word and the exchange's block counter (both in the first 256 bytes).
+    FOCUS_CUDA(cudaMemsetAsync(workspace, 0, kAlign, static_cast<cudaStream_t>(stream)));
     return FOCUS_OK;
 }
 
@@ -416,6 +417,8 @@ struct Tail {
     void *packed;
     int64_t capacity;
     float *delta_out, *i0_out, *i1_out;
+    const uint32_t *ex_flags;  // peer exchange: wait for these flags to show ex_epoch
+    uint32_t ex_epoch;
 };
 
 bool tail_uses_lists(const focus_dims_t &d, const Tail &t) {
@@ -441,6 +444,8 @@ focus_status_t launch_tail(const focus_dims_t &d, const Tail &t, uint8_t *ws, cu
     sp.H = d.hidden;
     sp.pool_window = d.pool_window;
     sp.layers = t.layers;
+    sp.ex_flags = t.ex_flags;
+    sp.ex_epoch = t.ex_epoch;
     if (tail_uses_lists(d, t)) {
         const WsLayout w = ws_layout(d);
         sp.constraints = d.constraints;
@@ -562,7 +567,112 @@ focus_status_t evict_impl(const focus_dims_t *dims, const focus_evict_args_t &x)
 
     Tail t{p.partial, d.Hkv * p.MT, layer1_only ? 1 : 2, p.status, x.hidden, x.decoded,
            x.budget, x.decode_avg, x.budget_alpha, x.budget_out, x.kept_idx, x.cu_seqlens,
-           x.packed, x.capacity, x.delta_out, x.i0_out, x.i1_out};
+           x.packed, x.capacity, x.delta_out, x.i0_out, x.i1_out, nullptr, 0};
+    return launch_tail(d, t, ws, s);
+}
+
+// Both layers' importance over dims' heads: planner, attention, reduction into
+// `importance` [2, R, B] or, with `ex`, into every rank's exchange buffer.
+focus_status_t partial_importance_impl(const focus_dims_t *dims, const void *q0,
+                                       const void *k0_prefix, const void *k0_block,
+                                       const void *q1, const void *k1_prefix,
+                                       const void *k1_block, const int32_t *cu_prefix,
+                                       int64_t total_prefix, float *importance,
+                                       const focus_exchange_t *ex, void *workspace,
+                                       size_t workspace_bytes, void *stream) {
+    FOCUS_TRY(check_dims(dims));
+    const focus_dims_t &d = *dims;
+    const bool layer1_only = d.score == FOCUS_SCORE_LAYER1;
+    if (!layer1_only)
+        FOCUS_TRY(check_attn_inputs(d, q0, k0_prefix, cu_prefix, total_prefix, k0_block));
+    FOCUS_TRY(check_attn_inputs(d, q1, k1_prefix, cu_prefix, total_prefix, k1_block));
+    FOCUS_TRY(check_ws(d, workspace, workspace_bytes));
+    FOCUS_TRY(get_encoder());
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+
+    AttnParams p;
+    memset(&p, 0, sizeof p);
+    const int layers = layer1_only ? 1 : 2;
+    fill_common(p, d, cu_prefix, total_prefix, ws, layers);
+    if (layer1_only) {
+        FOCUS_TRY(encode_layer(p, 0, d, q1, k1_prefix, total_prefix, k1_block));
+        p.tm_q[1] = p.tm_q[0];
+        p.tm_kp[1] = p.tm_kp[0];
+        p.tm_kb[1] = p.tm_kb[0];
+    } else {
+        FOCUS_TRY(encode_layer(p, 0, d, q0, k0_prefix, total_prefix, k0_block));
+        FOCUS_TRY(encode_layer(p, 1, d, q1, k1_prefix, total_prefix, k1_block));
+    }
+    focus::PlanParams pp;
+    memset(&pp, 0, sizeof pp);
+    pp.cu_prefix = cu_prefix;
+    pp.order = const_cast<int32_t *>(p.order);
+    pp.status = p.status;
+    pp.R = d.R;
+    pp.B = d.B;
+    FOCUS_CUDA(focus::launch_plan(pp, s));
+    FOCUS_CUDA(launch_attn_traced(p, d.head_dim, s, /*pdl=*/true));
+    focus::ReduceParams rp;
+    memset(&rp, 0, sizeof rp);
+    rp.partial = p.partial;
+    rp.R = d.R;
+    rp.B = d.B;
+    rp.Hkv = d.Hkv;
+    rp.MT = p.MT;
+    rp.layers = layers;
+    if (ex) {
+        rp.ex_bufs = ex->peer_buffers;
+        rp.ex_rank = ex->rank;
+        rp.ex_world = ex->world;
+        rp.ex_epoch = ex->epoch;
+        rp.ex_counter = reinterpret_cast<unsigned int *>(ws + ws_layout(d).status + 64);
+    } else {
+        // With the layer-1 score the single layer goes to importance[1].
+        rp.importance = layer1_only ? importance + static_cast<size_t>(d.R) * d.B : importance;
+    }
+    FOCUS_CUDA(focus::launch_reduce(rp, s, /*pdl=*/true));
+    return FOCUS_OK;
+}
+
+// Planner, selection and compaction from per-request sums `sums` ([layers][R][groups][B],
+// summed over groups in order); with `ex_flags`, after those flags show `ex_epoch`.
+focus_status_t evict_from_sums(const focus_dims_t *dims, const float *sums, int groups,
+                               const uint32_t *ex_flags, uint32_t ex_epoch, const void *hidden,
+                               const uint8_t *decoded, const int32_t *budget, int32_t *kept_idx,
+                               int32_t *cu_seqlens, void *packed, int64_t capacity,
+                               float *delta_out, void *workspace, size_t workspace_bytes,
+                               void *stream) {
+    const focus_dims_t &d = *dims;
+    FOCUS_TRY(check_ptr(hidden, 16));
+    FOCUS_TRY(check_ptr(decoded, 1));
+    FOCUS_TRY(check_ptr(budget, 4));
+    FOCUS_TRY(check_ptr(cu_seqlens, 4));
+    if (capacity < 0) return FOCUS_ERR_INVALID_ARGUMENT;
+    if (capacity > 0) {
+        FOCUS_TRY(check_ptr(kept_idx, 4));
+        FOCUS_TRY(check_ptr(packed, 16));
+    }
+    if (delta_out) FOCUS_TRY(check_ptr(delta_out, 4));
+    FOCUS_TRY(check_ws(d, workspace, workspace_bytes));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws + ws_layout(d).status);
+
+    const bool layer1_only = d.score == FOCUS_SCORE_LAYER1;
+    Tail t{sums, groups, layer1_only ? 1 : 2, status, hidden, decoded, budget, nullptr, 0.f,
+           nullptr, kept_idx, cu_seqlens, packed, capacity, delta_out, nullptr, nullptr,
+           ex_flags, ex_epoch};
+    focus::PlanParams pp;
+    memset(&pp, 0, sizeof pp);
+    pp.decoded = decoded;
+    pp.budget = budget;
+    pp.cu_seqlens = tail_uses_lists(d, t) ? nullptr : cu_seqlens;
+    pp.status = status;
+    pp.capacity = capacity;
+    pp.R = d.R;
+    pp.B = d.B;
+    FOCUS_CUDA(focus::launch_plan(pp, s));
     return launch_tail(d, t, ws, s);
 }
 
@@ -689,44 +799,54 @@ focus_status_t focus_partial_importance(const focus_dims_t *dims, const void *q0
                                         const void *k1_block, const int32_t *cu_prefix,
                                         int64_t total_prefix, float *importance, void *workspace,
                                         size_t workspace_bytes, void *stream) {
-    FOCUS_TRY(check_dims(dims));
-    const focus_dims_t &d = *dims;
-    const bool layer1_only = d.score == FOCUS_SCORE_LAYER1;
-    if (!layer1_only)
-        FOCUS_TRY(check_attn_inputs(d, q0, k0_prefix, cu_prefix, total_prefix, k0_block));
-    FOCUS_TRY(check_attn_inputs(d, q1, k1_prefix, cu_prefix, total_prefix, k1_block));
     FOCUS_TRY(check_ptr(importance, 4));
-    FOCUS_TRY(check_ws(d, workspace, workspace_bytes));
-    FOCUS_TRY(get_encoder());
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    return partial_importance_impl(dims, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block,
+                                   cu_prefix, total_prefix, importance, nullptr, workspace,
+                                   workspace_bytes, stream);
+}
 
-    AttnParams p;
-    memset(&p, 0, sizeof p);
-    const int layers = layer1_only ? 1 : 2;
-    fill_common(p, d, cu_prefix, total_prefix, ws, layers);
-    if (layer1_only) {
-        FOCUS_TRY(encode_layer(p, 0, d, q1, k1_prefix, total_prefix, k1_block));
-        p.tm_q[1] = p.tm_q[0];
-        p.tm_kp[1] = p.tm_kp[0];
-        p.tm_kb[1] = p.tm_kb[0];
-    } else {
-        FOCUS_TRY(encode_layer(p, 0, d, q0, k0_prefix, total_prefix, k0_block));
-        FOCUS_TRY(encode_layer(p, 1, d, q1, k1_prefix, total_prefix, k1_block));
-    }
-    focus::PlanParams pp;
-    memset(&pp, 0, sizeof pp);
-    pp.cu_prefix = cu_prefix;
-    pp.order = const_cast<int32_t *>(p.order);
-    pp.status = p.status;
-    pp.R = d.R;
-    pp.B = d.B;
-    FOCUS_CUDA(focus::launch_plan(pp, s));
-    FOCUS_CUDA(launch_attn_traced(p, d.head_dim, s, /*pdl=*/true));
-    float *out = layer1_only ? importance + static_cast<size_t>(d.R) * d.B : importance;
-    focus::ReduceParams rp{p.partial, out, d.R, d.B, d.Hkv, p.MT, layers};
-    FOCUS_CUDA(focus::launch_reduce(rp, s, /*pdl=*/true));
-    return FOCUS_OK;
+size_t focus_exchange_buffer_size(const focus_dims_t *dims, int32_t world) {
+    if (check_dims(dims) != FOCUS_OK || world < 1 || world > focus::kMaxExchangeWorld) return 0;
+    return focus::ex_layout(dims->R, dims->B, world).total;
+}
+
+focus_status_t focus_partial_importance_push(const focus_dims_t *dims, const void *q0,
+                                             const void *k0_prefix, const void *k0_block,
+                                             const void *q1, const void *k1_prefix,
+                                             const void *k1_block, const int32_t *cu_prefix,
+                                             int64_t total_prefix, const focus_exchange_t *exchange,
+                                             void *workspace, size_t workspace_bytes,
+                                             void *stream) {
+    if (!exchange) return FOCUS_ERR_INVALID_ARGUMENT;
+    const focus_exchange_t &x = *exchange;
+    FOCUS_TRY(check_ptr(x.peer_buffers, 8));
+    if (x.world < 1 || x.world > focus::kMaxExchangeWorld || x.rank < 0 || x.rank >= x.world ||
+        x.epoch == 0)
+        return FOCUS_ERR_INVALID_ARGUMENT;
+    return partial_importance_impl(dims, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block,
+                                   cu_prefix, total_prefix, nullptr, &x, workspace,
+                                   workspace_bytes, stream);
+}
+
+focus_status_t focus_evict_from_exchange(const focus_dims_t *dims, const void *exchange_buffer,
+                                         int32_t world, uint32_t epoch, const void *hidden,
+                                         const uint8_t *decoded, const int32_t *budget,
+                                         int32_t *kept_idx, int32_t *cu_seqlens, void *packed,
+                                         int64_t capacity, float *delta_out, void *workspace,
+                                         size_t workspace_bytes, void *stream) {
+    FOCUS_TRY(check_dims(dims));
+    FOCUS_TRY(check_ptr(exchange_buffer, kAlign));
+    if (world < 1 || world > focus::kMaxExchangeWorld || epoch == 0)
+        return FOCUS_ERR_INVALID_ARGUMENT;
+    const focus_dims_t &d = *dims;
+    const focus::ExLayout el = focus::ex_layout(d.R, d.B, world);
+    const uint8_t *buf = static_cast<const uint8_t *>(exchange_buffer);
+    const float *slots = reinterpret_cast<const float *>(buf) +
+                         static_cast<size_t>(epoch & 1u) * 2 * d.R * world * d.B;
+    const uint32_t *flags = reinterpret_cast<const uint32_t *>(buf + el.flags);
+    return evict_from_sums(dims, slots, world, flags, epoch, hidden, decoded, budget, kept_idx,
+                           cu_seqlens, packed, capacity, delta_out, workspace, workspace_bytes,
+                           stream);
 }
 
 focus_status_t focus_evict_from_importance(const focus_dims_t *dims, const float *importance,
@@ -736,38 +856,14 @@ focus_status_t focus_evict_from_importance(const focus_dims_t *dims, const float
                                            float *delta_out, void *workspace,
                                            size_t workspace_bytes, void *stream) {
     FOCUS_TRY(check_dims(dims));
-    const focus_dims_t &d = *dims;
     FOCUS_TRY(check_ptr(importance, 4));
-    FOCUS_TRY(check_ptr(hidden, 16));
-    FOCUS_TRY(check_ptr(decoded, 1));
-    FOCUS_TRY(check_ptr(budget, 4));
-    FOCUS_TRY(check_ptr(cu_seqlens, 4));
-    if (capacity < 0) return FOCUS_ERR_INVALID_ARGUMENT;
-    if (capacity > 0) {
-        FOCUS_TRY(check_ptr(kept_idx, 4));
-        FOCUS_TRY(check_ptr(packed, 16));
-    }
-    if (delta_out) FOCUS_TRY(check_ptr(delta_out, 4));
-    FOCUS_TRY(check_ws(d, workspace, workspace_bytes));
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    uint32_t *status = reinterpret_cast<uint32_t *>(ws + ws_layout(d).status);
-
-    const bool layer1_only = d.score == FOCUS_SCORE_LAYER1;
-    Tail t{layer1_only ? importance + static_cast<size_t>(d.R) * d.B : importance, 1,
-           layer1_only ? 1 : 2, status, hidden, decoded, budget, nullptr, 0.f, nullptr,
-           kept_idx, cu_seqlens, packed, capacity, delta_out, nullptr, nullptr};
-    focus::PlanParams pp;
-    memset(&pp, 0, sizeof pp);
-    pp.decoded = decoded;
-    pp.budget = budget;
-    pp.cu_seqlens = tail_uses_lists(d, t) ? nullptr : cu_seqlens;
-    pp.status = status;
-    pp.capacity = capacity;
-    pp.R = d.R;
-    pp.B = d.B;
-    FOCUS_CUDA(focus::launch_plan(pp, s));
-    return launch_tail(d, t, ws, s);
+    // With the layer-1 score only importance[1] is read.
+    const float *sums = dims->score == FOCUS_SCORE_LAYER1
+                            ? importance + static_cast<size_t>(dims->R) * dims->B
+                            : importance;
+    return evict_from_sums(dims, sums, 1, nullptr, 0, hidden, decoded, budget, kept_idx,
+                           cu_seqlens, packed, capacity, delta_out, workspace, workspace_bytes,
+                           stream);
 }
 
 const char *focus_status_string(focus_status_t st) {

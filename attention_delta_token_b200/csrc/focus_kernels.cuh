@@ -109,6 +109,10 @@ struct SelectParams {
     const float *decode_avg;   // [R]
     float budget_alpha;
     int32_t *budget_out;       // [R]
+    // Peer exchange (ex_flags != null): `partial` is this rank's slots of the epoch
+    // ([layers][R][world = Hkv x MT][B]); wait for flags[0 .. world-1] == ex_epoch first.
+    const uint32_t *ex_flags;
+    uint32_t ex_epoch;
 };
 
 struct ScanParams {
@@ -131,9 +135,27 @@ cudaError_t launch_delta(const DeltaParams &p, cudaStream_t stream);
 
 struct ReduceParams {
     const float *partial;  // [layers][R][Hkv][MT][B]
-    float *importance;     // [layers][R][B]
+    float *importance;     // [layers][R][B] (null with the peer exchange)
     int R, B, Hkv, MT, layers;
+    // Peer exchange (ex_world > 0, focus_exchange.cuh): the sums go to slot ex_rank
+    // of every rank's exchange buffer instead of `importance`.
+    void *const *ex_bufs;       // device array [ex_world] of peer-mapped buffers
+    int ex_rank, ex_world;
+    uint32_t ex_epoch;
+    unsigned int *ex_counter;   // blocks done (in the workspace), 0 between launches
 };
+
+// Exchange buffer of one rank: slots [2 parities][2 layers][R][world][B] float32,
+// then flags [2 parities][world] uint32 at `flags` (256-byte aligned).
+constexpr int kMaxExchangeWorld = 8;
+struct ExLayout {
+    size_t flags, total;
+};
+__host__ __device__ inline ExLayout ex_layout(int R, int B, int world) {
+    const size_t slots = 2ull * 2ull * static_cast<size_t>(R) * world * B * sizeof(float);
+    const size_t flags = (slots + 255) / 256 * 256;
+    return {flags, flags + 256};
+}
 cudaError_t launch_reduce(const ReduceParams &p, cudaStream_t stream, bool pdl = false);
 
 struct CompactParams {

@@ -14,6 +14,7 @@
 
 #include "focus_device.cuh"
 #include "focus_kernels.cuh"
+#include "focus_exchange.cuh"
 
 namespace focus {
 
@@ -217,19 +218,23 @@ __global__ void __launch_bounds__(256) select_compact_kernel(const SelectParams 
     const size_t rb = static_cast<size_t>(r) * B;
 
     if (j < B) dec_s[j] = p.decoded[rb + j];
+    // With the peer exchange the sums arrive from every rank; on a timeout the
+    // status says so and the slots are read as they are.
+    if (p.ex_flags) ex_wait(p.ex_flags, p.Hkv * p.MT, p.ex_epoch, p.status);
     if (p.partial) {
+        // Loads through L2: the sums were written by another kernel (or GPU).
         if (j < B) {
             const size_t lstride = static_cast<size_t>(p.R) * p.Hkv * p.MT * B;
             float i0 = 0.f, i1 = 0.f;
             if (p.layers == 1) {  // only the layer-1 statistics exist: score = I1
                 for (int g = 0; g < p.Hkv * p.MT; ++g)
-                    i1 += p.partial[(rb * p.Hkv * p.MT) + static_cast<size_t>(g) * B + j];
+                    i1 += __ldcg(p.partial + (rb * p.Hkv * p.MT) + static_cast<size_t>(g) * B + j);
                 raw_s[j] = i1;
             } else {
                 for (int g = 0; g < p.Hkv * p.MT; ++g) {
                     const size_t idx = (rb * p.Hkv * p.MT) + static_cast<size_t>(g) * B + j;
-                    i0 += p.partial[idx];
-                    i1 += p.partial[lstride + idx];
+                    i0 += __ldcg(p.partial + idx);
+                    i1 += __ldcg(p.partial + lstride + idx);
                 }
                 raw_s[j] = i1 - i0;
                 if (p.i0_out) p.i0_out[rb + j] = i0;
@@ -347,16 +352,26 @@ __global__ void __launch_bounds__(128) delta_kernel(const DeltaParams p) {
 }
 
 // importance[l][r][j] = sum over kv heads and row tiles (fixed order) of layer l's
-// column sums; one block per (request, layer).
+// column sums; one block per (request, layer).  With the peer exchange the sum is
+// stored into every rank's exchange buffer and the last block raises this rank's
+// flags (focus_exchange.cuh).
 __global__ void __launch_bounds__(128) reduce_kernel(const ReduceParams p) {
     pdl_wait();  // the column sums come from the attention kernel
     const int r = blockIdx.x, l = blockIdx.y, j = threadIdx.x, B = p.B;
-    if (j >= B) return;
-    const size_t rb = static_cast<size_t>(r) * B;
-    const float *part = p.partial + static_cast<size_t>(l) * p.R * p.Hkv * p.MT * B;
-    float s = 0.f;
-    for (int g = 0; g < p.Hkv * p.MT; ++g) s += part[rb * p.Hkv * p.MT + static_cast<size_t>(g) * B + j];
-    p.importance[static_cast<size_t>(l) * p.R * B + rb + j] = s;
+    if (j < B) {
+        const size_t rb = static_cast<size_t>(r) * B;
+        const float *part = p.partial + static_cast<size_t>(l) * p.R * p.Hkv * p.MT * B;
+        float s = 0.f;
+        for (int g = 0; g < p.Hkv * p.MT; ++g)
+            s += __ldcg(part + rb * p.Hkv * p.MT + static_cast<size_t>(g) * B + j);
+        if (p.ex_world)
+            ex_push(p.ex_bufs, p.R, B, p.ex_world, p.ex_rank, p.ex_epoch, l, r, j, s);
+        else
+            p.importance[static_cast<size_t>(l) * p.R * B + rb + j] = s;
+    }
+    if (p.ex_world)
+        ex_signal(p.ex_bufs, ex_layout(p.R, B, p.ex_world).flags, p.ex_world, p.ex_rank,
+                  p.ex_epoch, p.ex_counter, gridDim.x * gridDim.y);
 }
 
 // Stand-alone compaction: one warp per packed row, request found by binary search.

@@ -267,13 +267,26 @@ def run_ours(args, rank, world, local_rank):
         counts = algorithmic_counts(dataclasses.replace(p, Hq=p.Hq // tp, Hkv=p.Hkv // tp),
                                     layers=1 if args.score else 2)
 
-        def step():
-            F.focus_partial_importance(sdims, *s_l0, sl["q1"], sl["k1_prefix"], sl["k1_block"],
-                                       p.cu_prefix, imp, tp_ws)
-            if world > 1:
-                dist.all_reduce(imp)
-            F.focus_evict_from_importance(dims, imp, p.hidden, p.decoded, p.budget, kept, cu,
-                                          packed, ws)
+        if args.tp_exchange == "p2p":
+            # the sums travel inside the kernels: pushed into every rank's exchange buffer
+            from attention_delta_token_b200.parallel import PeerExchange
+            ex = (PeerExchange.symmetric(dims) if world > 1 else PeerExchange.local(dims, dev))
+
+            def step():
+                epoch = ex.next_epoch()
+                F.focus_partial_importance_push(sdims, *s_l0, sl["q1"], sl["k1_prefix"],
+                                                sl["k1_block"], p.cu_prefix, ex.peer_ptrs,
+                                                ex.rank, ex.world, epoch, tp_ws)
+                F.focus_evict_from_exchange(dims, ex.buffer, ex.world, epoch, p.hidden,
+                                            p.decoded, p.budget, kept, cu, packed, ws)
+        else:
+            def step():
+                F.focus_partial_importance(sdims, *s_l0, sl["q1"], sl["k1_prefix"],
+                                           sl["k1_block"], p.cu_prefix, imp, tp_ws)
+                if world > 1:
+                    dist.all_reduce(imp)
+                F.focus_evict_from_importance(dims, imp, p.hidden, p.decoded, p.budget, kept,
+                                              cu, packed, ws)
     elif args.dynamic_budget:
         # historical decoded-per-step averages: ~10% of a 32-token block per step
         # (Figure 2), drawn uniformly in [0, 0.2 B] per request
@@ -413,10 +426,13 @@ def run_ours(args, rank, world, local_rank):
                 "l2": f"no flush: {in_bytes / 2**30:.2f} GiB of inputs per step > 126 MB L2",
                 "accumulate": "fp32",
                 "parallelism": (f"dp{world} (request-sharded replicas)" if tp <= 1 else
-                                f"tp{tp} (head-sharded, NCCL all-reduce of 2 x R x B fp32)"
+                                f"tp{tp} (head-sharded; partial importance exchanged by "
+                                f"{'peer stores inside the kernels' if args.tp_exchange == 'p2p' else 'NCCL all-reduce'})"
                                 if world > 1 else
                                 f"tp{tp} emulated: rank 0's head shard + the shared selection "
-                                "timed on one GPU, no all-reduce"),
+                                "timed on one GPU" + (", exchanging with itself through its "
+                                "exchange buffer" if args.tp_exchange == "p2p" else
+                                ", no all-reduce")),
                 "constraints": args.constraints, "score": args.score, "lse0": args.lse0,
                 "page_size": args.page_size, "dynamic_budget": args.dynamic_budget,
             },
@@ -541,6 +557,9 @@ def main():
                     help="head-sharded (tensor-parallel) step over this many head shards: under "
                          "torchrun one rank per shard with an NCCL all-reduce; on one GPU rank "
                          "0's share is timed")
+    ap.add_argument("--tp-exchange", choices=["nccl", "p2p"], default="nccl",
+                    help="with --tp-shards: NCCL all-reduce between two library calls, or the "
+                         "exchange fused into the kernels over peer memory")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -344,6 +344,69 @@ FOCUS_API focus_status_t focus_evict_from_importance(
     void *stream);
 
 /*
+ * Peer exchange of the partial importance: the head-sharded step without a
+ * separate all-reduce.  Each rank exposes one exchange buffer of
+ * focus_exchange_buffer_size(dims, world) bytes to its peers (device memory that
+ * every rank can address: CUDA IPC or symmetric-memory mappings over NVLink).
+ * focus_partial_importance_push computes the rank's [2, R, B] sums like
+ * focus_partial_importance and stores them, from the reducing kernel itself,
+ * into slot `rank` of every rank's buffer, then raises the rank's flag there;
+ * focus_evict_from_exchange waits for every rank's flag in the local buffer,
+ * sums the slots in rank order (so every rank holds bit-identical sums) and
+ * selects and compacts as focus_evict_from_importance.  (The pages run on one
+ * GPU; this is a deployment variant.)
+ *
+ * Protocol, per rank and step: push(epoch), then evict_from_exchange(epoch), on
+ * one stream, with epoch = 1, 2, 3, ... the same on every rank.  Zero every
+ * buffer once (all bytes) and synchronise the ranks on the host before the
+ * first push.  Two slot parities make it safe for a rank to run one step ahead.
+ * A flag that does not arrive within 2 s sets FOCUS_ERR_TIMEOUT in the device
+ * status (read with focus_read_device_status); the sums are then not valid.
+ * The workspace must not be shared with another stream while a push runs.
+ */
+typedef struct {
+    void *const *peer_buffers; /* DEVICE array [world] of device pointers: rank q's exchange
+                                  buffer as this process addresses it (entry `rank` = own) */
+    int32_t rank;              /* 0 <= rank < world */
+    int32_t world;             /* 1 <= world <= 8 */
+    uint32_t epoch;            /* >= 1 */
+} focus_exchange_t;
+
+/* Bytes of one rank's exchange buffer for dims.R, dims.B (0 for invalid dims or world). */
+FOCUS_API size_t focus_exchange_buffer_size(const focus_dims_t *dims, int32_t world);
+
+/* focus_partial_importance whose sums go to the peers' exchange buffers. */
+FOCUS_API focus_status_t focus_partial_importance_push(
+    const focus_dims_t *dims, const void *q0, const void *k0_prefix, const void *k0_block,
+    const void *q1, const void *k1_prefix, const void *k1_block, const int32_t *cu_prefix,
+    int64_t total_prefix, const focus_exchange_t *exchange, void *workspace,
+    size_t workspace_bytes, void *stream);
+
+/* focus_evict_from_importance on the sum over ranks of the exchange buffer's
+ * slots of `epoch` (exchange_buffer: this rank's own buffer, 256-byte aligned). */
+FOCUS_API focus_status_t focus_evict_from_exchange(
+    const focus_dims_t *dims, const void *exchange_buffer, int32_t world, uint32_t epoch,
+    const void *hidden, const uint8_t *decoded, const int32_t *budget, int32_t *kept_idx,
+    int32_t *cu_seqlens, void *packed, int64_t capacity, float *delta_out, void *workspace,
+    size_t workspace_bytes, void *stream);
+
+/*
+ * Self-test of the exchange protocol with `world` emulated ranks on ONE GPU, in one
+ * cooperative launch (all blocks resident, so blocks may wait on one another):
+ * block group q pushes partials[q] ([world][2][R][B] float32) into every buffer
+ * with the device routines the push uses, raises its flags, waits for all flags
+ * of its own buffer as the selection does, and writes the rank-ordered sum of
+ * its slots to out[q] ([world][2][R][B]).  buffers: DEVICE array [world] of
+ * exchange buffers (zeroed); scratch: DEVICE, >= 1 + world uint32, zeroed;
+ * scratch[0] receives the device status bits.  R * 2 * world <= 1024.
+ * (No counterpart on the pages: a test of this library.)
+ */
+FOCUS_API focus_status_t focus_selftest_exchange(const float *partials, void *const *buffers,
+                                                 float *out, uint32_t *scratch, int32_t R,
+                                                 int32_t B, int32_t world, uint32_t epoch,
+                                                 void *stream);
+
+/*
  * The fused step for callers that cannot allocate device memory.  (The FOCUS
  * pages have no counterpart: this is a deployment variant of focus_evict.)
  *

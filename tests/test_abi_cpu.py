@@ -232,3 +232,47 @@ def test_split_entry_points_validation():
     assert from_imp(delta=A + 1) == INVALID
     assert from_imp(w=8) == WORKSPACE
     assert from_imp(dd=dims(pool_window=2)) == UNSUPPORTED
+
+
+def test_exchange_entry_points_validation():
+    """Host checks of the peer-exchange calls (nothing is launched)."""
+    d = dims()
+    ws = F.focus_workspace_size(d)
+    L = F._lib
+    for world in (1, 2, 8):
+        slots = 2 * 2 * d.R * world * d.B * 4
+        assert F.focus_exchange_buffer_size(d, world) == (slots + 255) // 256 * 256 + 256
+    assert L.focus_exchange_buffer_size(ctypes.byref(d), 0) == 0
+    assert L.focus_exchange_buffer_size(ctypes.byref(d), 9) == 0
+
+    def push(ex):
+        return L.focus_partial_importance_push(ctypes.byref(d), A, A, A, A, A, A, A, 100,
+                                               None if ex is None else ctypes.byref(ex), A, ws,
+                                               None)
+    assert push(None) == INVALID
+    assert push(F.FocusExchange(None, 0, 2, 1)) == INVALID       # no peer array
+    assert push(F.FocusExchange(A + 4, 0, 2, 1)) == INVALID      # misaligned peer array
+    assert push(F.FocusExchange(A, 2, 2, 1)) == INVALID          # rank >= world
+    assert push(F.FocusExchange(A, -1, 2, 1)) == INVALID
+    assert push(F.FocusExchange(A, 0, 9, 1)) == INVALID          # world > 8
+    assert push(F.FocusExchange(A, 0, 2, 0)) == INVALID          # epoch 0
+    assert L.focus_partial_importance_push(ctypes.byref(dims(B=0)), A, A, A, A, A, A, A, 100,
+                                           ctypes.byref(F.FocusExchange(A, 0, 2, 1)), A, ws,
+                                           None) == INVALID
+
+    def from_ex(buf=A, world=2, epoch=1, w=ws):
+        return L.focus_evict_from_exchange(ctypes.byref(d), buf, world, epoch, A, A, A, A, A, A,
+                                           16, None, A, w, None)
+    assert from_ex(buf=None) == INVALID
+    assert from_ex(buf=A + 16) == INVALID                        # must be 256-byte aligned
+    assert from_ex(world=0) == INVALID
+    assert from_ex(epoch=0) == INVALID
+    assert from_ex(w=8) == WORKSPACE
+
+    def selftest(R=4, B=32, world=2, epoch=1, ptr=A):
+        return L.focus_selftest_exchange(A, ptr, A, A, R, B, world, epoch, None)
+    assert selftest(ptr=None) == INVALID
+    assert selftest(B=129) == INVALID
+    assert selftest(world=9) == INVALID
+    assert selftest(epoch=0) == INVALID
+    assert selftest(R=200, world=4) == INVALID                   # too many blocks to co-reside

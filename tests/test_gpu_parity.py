@@ -603,3 +603,117 @@ def test_edge_shapes_vs_oracle(case, orc):
     check_selection(out["kept"], out["cu_seqlens"], ref["pooled"], p.decoded.numpy(),
                     p.budget.numpy(), requests=req)
     check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))
+
+
+@pytest.mark.parametrize("constraints,score", [(0, 0), (3, 0), (0, 1)])
+def test_peer_exchange_single_rank_bitwise_equal_fused(constraints, score):
+    """The fused-exchange path with a group of one (the rank pushes to its own buffer and
+    its selection waits for its own flag), over three consecutive steps so both slot
+    parities are used, reproduces focus_evict bit for bit."""
+    import attention_delta_token_b200 as F
+    from attention_delta_token_b200 import parallel
+    base = dict(R=9)
+    dims = None
+    ex = None
+    for step, seed in enumerate((820, 821, 822)):
+        p = synth.make_problem(4, seed=seed + 10 * constraints + 100 * score, overrides=base)
+        g = p.to("cuda")
+        fused = run_evict(g, constraints=constraints, score=score)
+        assert fused["status"] == 0
+        if dims is None:
+            dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window,
+                               constraints, score)
+            ex = parallel.PeerExchange.local(dims, "cuda")
+        cap = F.plan_capacity(p.decoded, p.budget, constraints)
+        kept = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+        cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+        packed = torch.zeros(cap, p.H, dtype=torch.bfloat16, device="cuda")
+        delta = torch.empty(p.R, p.B, device="cuda")
+        l0 = (None, None, None) if score else (g.q0, g.k0_prefix, g.k0_block)
+        ws = parallel.evict_head_sharded(dims, 0, 1, *l0, g.q1, g.k1_prefix, g.k1_block,
+                                         g.cu_prefix, g.hidden, g.decoded, g.budget, kept, cu,
+                                         packed, delta_out=delta, exchange=ex)
+        assert F.focus_read_device_status(ws) == 0
+        assert F.focus_read_device_status(ex.push_ws) == 0
+        assert ex.epoch == step + 1
+        np.testing.assert_array_equal(delta.cpu().numpy(), fused["delta"].astype(np.float32))
+        cu_h = cu.cpu().numpy()
+        np.testing.assert_array_equal(cu_h, fused["cu_seqlens"])
+        n = int(cu_h[-1])
+        np.testing.assert_array_equal(kept[:n].cpu().numpy(), fused["kept"][:n])
+        np.testing.assert_array_equal(
+            packed[:n].view(torch.int16).cpu().numpy().view(np.uint16), fused["packed"][:n])
+    # the flags of both parities hold the last epoch that used them
+    lay = F.focus_exchange_buffer_size(dims, 1)
+    flags = ex.buffer[lay - 256:lay - 256 + 8].view(torch.int32).cpu().tolist()
+    assert flags == [2, 3]
+
+
+@pytest.mark.parametrize("world", [2, 3, 8])
+def test_peer_exchange_protocol_emulated_ranks(world):
+    """The push / flag / wait / rank-ordered sum of the exchange with `world` ranks
+    emulated by block groups of one cooperative launch on one GPU: every rank ends with
+    the same sums, equal (bitwise) to the float32 sum in rank order; three steps in a
+    row use both slot parities."""
+    import attention_delta_token_b200 as F
+    R, B = 5, 32
+    dims = F.make_dims(R, B, 4, 2, 64, 8)
+    nbytes = F.focus_exchange_buffer_size(dims, world)
+    bufs = [torch.zeros(nbytes, dtype=torch.uint8, device="cuda") for _ in range(world)]
+    ptrs = torch.tensor([b.data_ptr() for b in bufs], dtype=torch.int64, device="cuda")
+    gen = torch.Generator().manual_seed(world)
+    for epoch in (1, 2, 3):
+        scale = 10.0 ** torch.randint(-3, 3, (world, 1, 1, 1), generator=gen).float()
+        parts = torch.randn(world, 2, R, B, generator=gen) * scale
+        out = torch.full((world, 2, R, B), float("nan"), device="cuda")
+        scratch = torch.zeros(1 + world, dtype=torch.int32, device="cuda")
+        F.focus_selftest_exchange(parts.cuda(), ptrs, out, scratch, epoch)
+        torch.cuda.synchronize()
+        assert int(scratch[0]) == 0
+        assert scratch[1:].eq(0).all()  # the last block of each rank reset its counter
+        want = torch.zeros(2, R, B)
+        for q in range(world):
+            want = want + parts[q]
+        got = out.cpu()
+        for q in range(world):
+            assert torch.equal(got[q], want), (epoch, q)
+
+
+def test_peer_exchange_missing_rank_times_out():
+    """A group of two in which rank 1 never pushes: rank 0's selection gives up after its
+    bounded wait, reports FOCUS_ERR_TIMEOUT, and the context stays usable."""
+    import time
+    import attention_delta_token_b200 as F
+    p = synth.make_problem(0, seed=830)
+    g = p.to("cuda")
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+    nbytes = F.focus_exchange_buffer_size(dims, 2)
+    bufs = [torch.zeros(nbytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    ptrs = torch.tensor([b.data_ptr() for b in bufs], dtype=torch.int64, device="cuda")
+    sdims = F.make_dims(p.R, p.B, p.Hq // 2, p.Hkv // 2, p.d, 8, p.scale)
+    push_ws = F.Workspace(sdims, "cuda")
+    from attention_delta_token_b200 import parallel
+    hq, hk = parallel.shard_heads(p.Hq, p.Hkv, 0, 2)
+    F.focus_partial_importance_push(sdims, g.q0[:, :, hq].contiguous(),
+                                    g.k0_prefix[:, hk].contiguous(),
+                                    g.k0_block[:, :, hk].contiguous(), g.q1[:, :, hq].contiguous(),
+                                    g.k1_prefix[:, hk].contiguous(),
+                                    g.k1_block[:, :, hk].contiguous(), g.cu_prefix, ptrs, 0, 2, 1,
+                                    push_ws)
+    assert F.focus_read_device_status(push_ws) == 0
+    ws = F.Workspace(dims, "cuda")
+    cap = F.plan_capacity(p.decoded, p.budget)
+    kept = torch.empty(cap, dtype=torch.int32, device="cuda")
+    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+    packed = torch.empty(cap, p.H, dtype=torch.bfloat16, device="cuda")
+    t0 = time.time()
+    F.focus_evict_from_exchange(dims, bufs[0], 2, 1, g.hidden, g.decoded, g.budget, kept, cu,
+                                packed, ws)
+    st = F.focus_read_device_status(ws, timeout_ms=20000)
+    assert st == 7  # FOCUS_ERR_TIMEOUT
+    assert 1.5 < time.time() - t0 < 15
+    # rank 0's own slot arrived, rank 1's flag did not
+    flags = bufs[0][nbytes - 256:nbytes - 256 + 16].view(torch.int32).cpu().tolist()
+    assert flags == [0, 0, 1, 0]
+    out = run_evict(g)  # the context is still usable
+    assert out["status"] == 0
