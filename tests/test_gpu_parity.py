@@ -6,6 +6,8 @@ ragged tails, several 128-row query tiles, both head dims, GQA group sizes
 the launch configuration the benchmark times and are compared on sampled
 requests, which the oracle computes one by one.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -717,3 +719,21 @@ def test_peer_exchange_missing_rank_times_out():
     assert flags == [0, 0, 1, 0]
     out = run_evict(g)  # the context is still usable
     assert out["status"] == 0
+
+
+def test_peer_exchange_symmetric_memory_group_of_one():
+    """PeerExchange.symmetric (torch symmetric memory, one NCCL rank on one GPU) drives the
+    fused exchange end to end and matches focus_evict bit for bit; run in a child process
+    under a time limit."""
+    import socket
+    import subprocess
+    import sys
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    here = os.path.dirname(os.path.abspath(__file__))
+    env = dict(os.environ, MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK="0",
+               WORLD_SIZE="1", LOCAL_RANK="0", NCCL_NVLS_ENABLE="0")
+    r = subprocess.run([sys.executable, os.path.join(here, "_symm_exchange_child.py")],
+                       capture_output=True, text=True, timeout=300, env=env, cwd=here)
+    assert r.returncode == 0 and r.stdout.strip().endswith("OK"), r.stdout[-2000:] + r.stderr[-3000:]
