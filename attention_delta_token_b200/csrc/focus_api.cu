@@ -181,6 +181,37 @@ void fill_common(AttnParams &p, const focus_dims_t &d, const int32_t *cu_prefix,
     p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
 }
 
+// One layer's attention inputs.
+struct LayerIn {
+    const void *q, *k_prefix, *k_block;
+};
+
+// The attention parameters of a call over `layers` layers: with one layer `l1` is
+// it (a single-layer call, or the layer-1 score); with two, `l0` then `l1`.  With
+// `lse0` (layer 0's row log-sum-exps given) layer 0 streams no prefix, so its
+// prefix map is never read.
+focus_status_t setup_attention(AttnParams &p, const focus_dims_t &d, int layers, const LayerIn &l0,
+                               const LayerIn &l1, const int32_t *cu_prefix,
+                               long long total_prefix, uint8_t *ws,
+                               int prefix_box = focus::kTileKeys, const float *lse0 = nullptr) {
+    memset(&p, 0, sizeof p);
+    fill_common(p, d, cu_prefix, total_prefix, ws, layers);
+    if (layers == 1) {
+        FOCUS_TRY(encode_layer(p, 0, d, l1.q, l1.k_prefix, total_prefix, l1.k_block, prefix_box));
+        p.tm_q[1] = p.tm_q[0];
+        p.tm_kp[1] = p.tm_kp[0];
+        p.tm_kb[1] = p.tm_kb[0];
+        return FOCUS_OK;
+    }
+    if (lse0)
+        FOCUS_TRY(encode_layer(p, 0, d, l0.q, nullptr, 0, l0.k_block));
+    else
+        FOCUS_TRY(encode_layer(p, 0, d, l0.q, l0.k_prefix, total_prefix, l0.k_block, prefix_box));
+    FOCUS_TRY(encode_layer(p, 1, d, l1.q, l1.k_prefix, total_prefix, l1.k_block, prefix_box));
+    p.lse0 = lse0;
+    return FOCUS_OK;
+}
+
 focus_status_t check_attn_inputs(const focus_dims_t &d, const void *q, const void *k_prefix,
                                  const int32_t *cu_prefix, long long total_prefix,
                                  const void *k_block) {
@@ -256,12 +287,8 @@ focus_status_t focus_attn_stats(const focus_dims_t *dims, const void *q, const v
     uint8_t *ws = static_cast<uint8_t *>(workspace);
 
     AttnParams p;
-    memset(&p, 0, sizeof p);
-    fill_common(p, d, cu_prefix, total_prefix, ws, 1);
-    FOCUS_TRY(encode_layer(p, 0, d, q, k_prefix, total_prefix, k_block));
-    p.tm_q[1] = p.tm_q[0];
-    p.tm_kp[1] = p.tm_kp[0];
-    p.tm_kb[1] = p.tm_kb[0];
+    FOCUS_TRY(setup_attention(p, d, 1, LayerIn{}, LayerIn{q, k_prefix, k_block}, cu_prefix,
+                              total_prefix, ws));
 
     focus::PlanParams pp;
     memset(&pp, 0, sizeof pp);
@@ -519,24 +546,11 @@ focus_status_t evict_impl(const focus_dims_t *dims, const focus_evict_args_t &x)
     cudaStream_t s = static_cast<cudaStream_t>(x.stream);
     uint8_t *ws = static_cast<uint8_t *>(x.workspace);
 
+    // With the layer-1 score (the Figure 13 ablation) layer 0 is not touched.
     AttnParams p;
-    memset(&p, 0, sizeof p);
-    if (layer1_only) {  // the Figure 13 ablation: rank by I1, layer 0 is not touched
-        fill_common(p, d, cu_prefix, total_prefix, ws, 1);
-        FOCUS_TRY(encode_layer(p, 0, d, x.q1, x.k1_prefix, total_prefix, x.k1_block, prefix_box));
-        p.tm_q[1] = p.tm_q[0];
-        p.tm_kp[1] = p.tm_kp[0];
-        p.tm_kb[1] = p.tm_kb[0];
-    } else {
-        fill_common(p, d, cu_prefix, total_prefix, ws, 2);
-        if (x.lse0)  // layer 0 streams no prefix: its prefix map is never read
-            FOCUS_TRY(encode_layer(p, 0, d, x.q0, nullptr, 0, x.k0_block));
-        else
-            FOCUS_TRY(encode_layer(p, 0, d, x.q0, x.k0_prefix, total_prefix, x.k0_block,
-                                   prefix_box));
-        FOCUS_TRY(encode_layer(p, 1, d, x.q1, x.k1_prefix, total_prefix, x.k1_block, prefix_box));
-        p.lse0 = x.lse0;
-    }
+    FOCUS_TRY(setup_attention(p, d, layer1_only ? 1 : 2, LayerIn{x.q0, x.k0_prefix, x.k0_block},
+                              LayerIn{x.q1, x.k1_prefix, x.k1_block}, cu_prefix, total_prefix, ws,
+                              prefix_box, layer1_only ? nullptr : x.lse0));
     if (paging) {
         p.cu_prefix = nullptr;
         p.page_table = paging->page_table;
@@ -591,19 +605,10 @@ focus_status_t partial_importance_impl(const focus_dims_t *dims, const void *q0,
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
 
-    AttnParams p;
-    memset(&p, 0, sizeof p);
     const int layers = layer1_only ? 1 : 2;
-    fill_common(p, d, cu_prefix, total_prefix, ws, layers);
-    if (layer1_only) {
-        FOCUS_TRY(encode_layer(p, 0, d, q1, k1_prefix, total_prefix, k1_block));
-        p.tm_q[1] = p.tm_q[0];
-        p.tm_kp[1] = p.tm_kp[0];
-        p.tm_kb[1] = p.tm_kb[0];
-    } else {
-        FOCUS_TRY(encode_layer(p, 0, d, q0, k0_prefix, total_prefix, k0_block));
-        FOCUS_TRY(encode_layer(p, 1, d, q1, k1_prefix, total_prefix, k1_block));
-    }
+    AttnParams p;
+    FOCUS_TRY(setup_attention(p, d, layers, LayerIn{q0, k0_prefix, k0_block},
+                              LayerIn{q1, k1_prefix, k1_block}, cu_prefix, total_prefix, ws));
     focus::PlanParams pp;
     memset(&pp, 0, sizeof pp);
     pp.cu_prefix = cu_prefix;
