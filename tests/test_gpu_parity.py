@@ -14,7 +14,7 @@ import torch
 
 import synth
 from focus_testutil import (assert_close_delta, assert_close_importance, check_packed,
-                            check_selection, hidden_bits, run_evict)
+                            check_selection, check_structured, hidden_bits, run_evict)
 
 pytestmark = pytest.mark.gpu
 
@@ -737,3 +737,72 @@ def test_peer_exchange_symmetric_memory_group_of_one():
     r = subprocess.run([sys.executable, os.path.join(here, "_symm_exchange_child.py")],
                        capture_output=True, text=True, timeout=300, env=env, cwd=here)
     assert r.returncode == 0 and r.stdout.strip().endswith("OK"), r.stdout[-2000:] + r.stderr[-3000:]
+
+
+@pytest.mark.parametrize("constraints", [0, 3])
+def test_dynamic_budget_degenerate_blocks(constraints, orc):
+    """Dynamic budget on degenerate blocks: a fully decoded block keeps nothing (K = 0), a
+    single masked token is kept (K = 1, its sigma is 0), a fully masked block with a huge
+    historical yield is capped at the masked count, a zero yield still keeps one token; the
+    budgets, kept sets and packed rows equal the oracle's."""
+    import attention_delta_token_b200 as F
+    p = synth.make_problem(1, seed=850, wide_logits=True, overrides=dict(R=4))
+    dec = p.decoded.numpy()
+    dec[0] = 1
+    dec[1] = 1
+    dec[1, 7] = 0
+    dec[2] = 0
+    avg = np.array([3.0, 2.0, 1000.0, 0.0], np.float32)
+    ref = orc.evict(p, constraints=constraints, decode_avg=avg.astype(np.float64))
+    np.testing.assert_array_equal(ref["budget"][:3], [0, 1, p.B])
+    g = p.to("cuda")
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, constraints)
+    ws = F.Workspace(dims)
+    cap = F.plan_capacity(p.decoded, None, constraints, dynamic=True)
+    kept = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+    packed = torch.zeros(cap, p.H, dtype=torch.bfloat16, device="cuda")
+    kout = torch.full((p.R,), -1, dtype=torch.int32, device="cuda")
+    F.focus_evict_ex(dims, q0=g.q0, k0_prefix=g.k0_prefix, k0_block=g.k0_block, q1=g.q1,
+                     k1_prefix=g.k1_prefix, k1_block=g.k1_block, cu_prefix=g.cu_prefix,
+                     hidden=g.hidden, decoded=g.decoded, decode_avg=torch.from_numpy(avg).cuda(),
+                     budget_alpha=1.5, budget_out=kout, kept_idx=kept, cu_seqlens=cu,
+                     packed=packed, ws=ws)
+    assert F.focus_read_device_status(ws) == 0
+    np.testing.assert_array_equal(kout.cpu().numpy()[:3], ref["budget"][:3])
+    cu_h = cu.cpu().numpy()
+    assert cu_h[1] == 0                       # the fully decoded block keeps nothing
+    assert list(kept[cu_h[1]:cu_h[2]].cpu().numpy()) == (
+        [6, 7] if constraints & 1 else [7])   # the lone masked token (and its predecessor)
+    assert cu_h[3] - cu_h[2] == p.B           # the fully masked block is kept whole
+    n = int(cu_h[-1])
+    check_packed(packed[:n].view(torch.int16).cpu().numpy().view(np.uint16),
+                 kept[:n].cpu().numpy(), cu_h, hidden_bits(p))
+    kg = kout.cpu().numpy()
+    if kg[3] == ref["budget"][3]:  # request 3's budget is decided by a margin in the oracle
+        if constraints:
+            check_structured(kept[:n].cpu().numpy(), cu_h, ref["kept"], ref["cu_seqlens"],
+                             ref["pooled"], dec, kg)
+        else:
+            check_selection(kept[:n].cpu().numpy(), cu_h, ref["pooled"], dec, kg)
+
+
+@pytest.mark.parametrize("window", [1, 5, 7])
+def test_other_pool_windows_vs_oracle(window, orc):
+    """MaxPool1D with windows other than the pages' k = 3 (the ABI takes any odd window):
+    the fused step and the stand-alone delta call against the oracle."""
+    import attention_delta_token_b200 as F
+    p = synth.make_problem(1, seed=860 + window, wide_logits=True,
+                           overrides=dict(R=5, prefix=("uniform", 0, 500), pool_window=window))
+    assert p.pool_window == window
+    ref = orc.evict(p)
+    g = p.to("cuda")
+    _compare_full(p, run_evict(g), ref)
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, window)
+    i0 = torch.from_numpy(ref["i0"]).float().cuda()
+    i1 = torch.from_numpy(ref["i1"]).float().cuda()
+    delta = torch.empty(p.R, p.B, device="cuda")
+    F.focus_importance_delta(dims, i0, i1, g.decoded, delta)
+    _, want = orc.delta_pool_mask(i0.double().cpu().numpy(), i1.double().cpu().numpy(),
+                                  p.decoded.numpy(), window=window)
+    assert_close_delta(delta.cpu().numpy(), want)
