@@ -23,6 +23,25 @@ namespace {
 constexpr int kPlanThreads = 1024;
 constexpr int kRankSortR = 1024; // up to here the order is a rank count
 constexpr int kMaxSortR = 4096;  // up to here a bitonic sort; larger batches keep input order
+constexpr int kCompactStagedCu = 4096;  // cu_seqlens entries the compaction stages in smem
+
+// sum over g < n of src[g * stride] in the order g = 0, 1, 2, ... (the fixed order
+// every reduction of the column sums uses, so the fused step, the stand-alone
+// reduction and the exchange all give the same bits), with eight loads in flight.
+// Loads go through L2: the sums were written by another kernel or another GPU.
+__device__ __forceinline__ float ordered_sum(const float *src, int n, int stride) {
+    float s = 0.f;
+    int g = 0;
+    for (; g + 8 <= n; g += 8) {
+        float x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = __ldcg(src + static_cast<size_t>(g + u) * stride);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) s += x[u];
+    }
+    for (; g < n; ++g) s += __ldcg(src + static_cast<size_t>(g) * stride);
+    return s;
+}
 
 // masked_r = number of zero bytes in decoded[r*B .. r*B+B); 16-byte loads when
 // the row is 16-byte aligned.
@@ -222,20 +241,17 @@ __global__ void __launch_bounds__(256) select_compact_kernel(const SelectParams 
     // status says so and the slots are read as they are.
     if (p.ex_flags) ex_wait(p.ex_flags, p.Hkv * p.MT, p.ex_epoch, p.status);
     if (p.partial) {
-        // Loads through L2: the sums were written by another kernel (or GPU).
         if (j < B) {
-            const size_t lstride = static_cast<size_t>(p.R) * p.Hkv * p.MT * B;
+            const int n = p.Hkv * p.MT;
+            const size_t lstride = static_cast<size_t>(p.R) * n * B;
+            const float *col = p.partial + rb * n + j;  // group g of column j at col[g * B]
             float i0 = 0.f, i1 = 0.f;
             if (p.layers == 1) {  // only the layer-1 statistics exist: score = I1
-                for (int g = 0; g < p.Hkv * p.MT; ++g)
-                    i1 += __ldcg(p.partial + (rb * p.Hkv * p.MT) + static_cast<size_t>(g) * B + j);
+                i1 = ordered_sum(col, n, B);
                 raw_s[j] = i1;
             } else {
-                for (int g = 0; g < p.Hkv * p.MT; ++g) {
-                    const size_t idx = (rb * p.Hkv * p.MT) + static_cast<size_t>(g) * B + j;
-                    i0 += __ldcg(p.partial + idx);
-                    i1 += __ldcg(p.partial + lstride + idx);
-                }
+                i0 = ordered_sum(col, n, B);
+                i1 = ordered_sum(col + lstride, n, B);
                 raw_s[j] = i1 - i0;
                 if (p.i0_out) p.i0_out[rb + j] = i0;
             }
@@ -360,10 +376,9 @@ __global__ void __launch_bounds__(128) reduce_kernel(const ReduceParams p) {
     const int r = blockIdx.x, l = blockIdx.y, j = threadIdx.x, B = p.B;
     if (j < B) {
         const size_t rb = static_cast<size_t>(r) * B;
-        const float *part = p.partial + static_cast<size_t>(l) * p.R * p.Hkv * p.MT * B;
-        float s = 0.f;
-        for (int g = 0; g < p.Hkv * p.MT; ++g)
-            s += __ldcg(part + rb * p.Hkv * p.MT + static_cast<size_t>(g) * B + j);
+        const int n = p.Hkv * p.MT;
+        const float *part = p.partial + static_cast<size_t>(l) * p.R * n * B;
+        const float s = ordered_sum(part + rb * n + j, n, B);
         if (p.ex_world)
             ex_push(p.ex_bufs, p.R, B, p.ex_world, p.ex_rank, p.ex_epoch, l, r, j, s);
         else
@@ -376,10 +391,18 @@ __global__ void __launch_bounds__(128) reduce_kernel(const ReduceParams p) {
 
 // Stand-alone compaction: one warp per packed row, request found by binary search.
 __global__ void __launch_bounds__(256) compact_kernel(const CompactParams p) {
+    __shared__ int cu_s[kCompactStagedCu];
     pdl_wait();  // kept_idx and cu_seqlens come from the previous kernels
+    // The binary search runs in shared memory when cu_seqlens fits (one coalesced
+    // load per block instead of a chain of dependent global loads per row).
+    const bool staged = p.R + 1 <= kCompactStagedCu;
+    if (staged)
+        for (int i = threadIdx.x; i <= p.R; i += blockDim.x) cu_s[i] = p.cu_seqlens[i];
+    __syncthreads();
+    const int32_t *cu = staged ? cu_s : p.cu_seqlens;
     const int warps = blockDim.x >> 5;
-    const long long total = min(static_cast<long long>(p.cu_seqlens[p.R]), p.capacity);
-    if (blockIdx.x == 0 && threadIdx.x == 0 && p.cu_seqlens[p.R] > p.capacity)
+    const long long total = min(static_cast<long long>(cu[p.R]), p.capacity);
+    if (blockIdx.x == 0 && threadIdx.x == 0 && cu[p.R] > p.capacity)
         atomicOr(p.status, FOCUS_DEV_CAPACITY);
     const int lane = threadIdx.x & 31;
     const int nvec = p.H / 8;
@@ -388,11 +411,11 @@ __global__ void __launch_bounds__(256) compact_kernel(const CompactParams p) {
         int lo = 0, hi = p.R - 1;  // largest r with cu[r] <= row
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (p.cu_seqlens[mid] <= row) lo = mid; else hi = mid - 1;
+            if (cu[mid] <= row) lo = mid; else hi = mid - 1;
         }
         int jj;
         if (p.lists) {  // structural constraints: row t of request lo is its t-th list entry
-            const long long t = row - p.cu_seqlens[lo];
+            const long long t = row - cu[lo];
             jj = (t >= 0 && t < p.B) ? p.lists[static_cast<size_t>(lo) * p.B + t] : -1;
             if (lane == 0 && jj >= 0 && jj < p.B) p.kept_out[row] = jj;
         } else {
@@ -407,13 +430,12 @@ __global__ void __launch_bounds__(256) compact_kernel(const CompactParams p) {
                                         (static_cast<size_t>(lo) * p.B + jj) * nvec;
         uint4 *__restrict__ dst = reinterpret_cast<uint4 *>(p.packed) + static_cast<size_t>(row) * nvec;
         int c = lane;
-        for (; c + 96 < nvec; c += 128) {  // four 16-byte loads in flight per lane
-            const uint4 x0 = __ldg(src + c), x1 = __ldg(src + c + 32), x2 = __ldg(src + c + 64),
-                        x3 = __ldg(src + c + 96);
-            dst[c] = x0;
-            dst[c + 32] = x1;
-            dst[c + 64] = x2;
-            dst[c + 96] = x3;
+        for (; c + 7 * 32 < nvec; c += 8 * 32) {  // eight 16-byte loads in flight per lane
+            uint4 x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[u] = __ldg(src + c + 32 * u);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) dst[c + 32 * u] = x[u];
         }
         for (; c < nvec; c += 32) dst[c] = __ldg(src + c);
     }
