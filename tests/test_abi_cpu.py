@@ -14,6 +14,7 @@ import attention_delta_token_b200 as F
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "focus.h")
+HEADER_DIR = os.path.dirname(HEADER)
 
 OK, INVALID, UNSUPPORTED, CAPACITY, WORKSPACE, CUDA, DEVCHECK, TIMEOUT = range(8)
 A = 0x100000  # a 256-byte-aligned fake device address (never dereferenced here)
@@ -276,3 +277,46 @@ def test_exchange_entry_points_validation():
     assert selftest(world=9) == INVALID
     assert selftest(epoch=0) == INVALID
     assert selftest(R=200, world=4) == INVALID                   # too many blocks to co-reside
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "focus.h"
+
+int main(void) {
+    focus_dims_t d;
+    memset(&d, 0, sizeof d);
+    d.R = 4; d.B = 32; d.Hq = 32; d.Hkv = 8; d.head_dim = 128; d.hidden = 4096;
+    d.softmax_scale = 0.08838834764831845f; d.pool_window = 3;
+    if (focus_abi_version() != FOCUS_ABI_VERSION) return 1;
+    if (focus_workspace_size(&d) == 0 || focus_exchange_buffer_size(&d, 2) == 0) return 2;
+    if (strcmp(focus_status_string(FOCUS_ERR_TIMEOUT), "FOCUS_ERR_TIMEOUT") != 0) return 3;
+    /* host validation only: a NULL query is rejected before anything is launched */
+    if (focus_evict(&d, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL, NULL, NULL, NULL,
+                    NULL, NULL, 0, NULL, NULL, NULL, NULL, 0, NULL) != FOCUS_ERR_INVALID_ARGUMENT)
+        return 4;
+    printf("ok %zu\n", focus_workspace_size(&d));
+    return 0;
+}
+"""
+
+
+def test_c_program_links_and_calls_the_library(tmp_path):
+    """The boundary is a plain C ABI: a C99 program that includes only focus.h compiles,
+    links against libfocus.so and calls it (entry points that need no GPU)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_focus.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "use_focus"
+    libdir = os.path.dirname(F.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", HEADER_DIR,
+                    str(src), "-L", libdir, "-Wl,-rpath," + libdir, "-l:libfocus.so", "-o",
+                    str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert r.stdout.startswith("ok ")
+    assert int(r.stdout.split()[1]) == F.focus_workspace_size(dims())
