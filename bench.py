@@ -328,13 +328,24 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
 
     # ---- device-resident timing
+    graph = None
     sampler = ClockSampler(local_rank)
     with sampler:
         for _ in range(args.warmup):
             step()
         barrier()
+        if args.graph:
+            # the whole step captured once (its kernels keep their programmatic
+            # dependent launch edges) and replayed: one launch of host work per step
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=torch.cuda.Stream(dev)):
+                step()
+            graph.replay()
+            barrier()
         # The attention kernel is timed on every TRACE_EVERY-th step: events around it
         # break the launch overlap with the planner, so they are not on every step.
+        # A graph replay cannot be traced: then the same number of direct steps are
+        # traced right after the timed loop.
         traced = list(range(0, args.steps, TRACE_EVERY))
         ev_a = [torch.cuda.Event(enable_timing=True) for _ in traced]
         ev_b = [torch.cuda.Event(enable_timing=True) for _ in traced]
@@ -345,6 +356,9 @@ def run_ours(args, rank, world, local_rank):
         barrier()
         start.record(stream)
         for k in range(args.steps):
+            if graph is not None:
+                graph.replay()
+                continue
             if k % TRACE_EVERY == 0:
                 F.focus_set_trace_events(ev_a[k // TRACE_EVERY], ev_b[k // TRACE_EVERY])
             step()
@@ -352,6 +366,12 @@ def run_ours(args, rank, world, local_rank):
                 F.focus_set_trace_events(None, None)
         stop.record(stream)
         barrier()
+        if graph is not None:
+            for i in range(len(traced)):
+                F.focus_set_trace_events(ev_a[i], ev_b[i])
+                step()
+                F.focus_set_trace_events(None, None)
+            barrier()
     for w in (ws, tp_ws) if tp_ws is not None else (ws,):
         status = F.focus_read_device_status(w)
         if status != 0:
@@ -435,6 +455,7 @@ def run_ours(args, rank, world, local_rank):
                                 ", no all-reduce")),
                 "constraints": args.constraints, "score": args.score, "lse0": args.lse0,
                 "page_size": args.page_size, "dynamic_budget": args.dynamic_budget,
+                "launch": "CUDA graph replay" if args.graph else "direct C-ABI calls",
             },
             "decisions_per_s": world * counts["decisions"] / step_s,
             "roofline": {
@@ -444,6 +465,8 @@ def run_ours(args, rank, world, local_rank):
                 "algorithmic_bytes_per_launch": counts["attn_bytes"],
                 "ms_per_launch": attn_s_max * 1e3, "peak_source": f"{peak_src} (hbm_gbs)",
                 "launches_timed": len(traced),
+                "timed_on": ("direct steps after the graph-replay loop" if args.graph else
+                             "every 8th step of the timed loop"),
                 "note": f"frac of {peak_src} HBM copy bandwidth",
             },
             "roofline_step": {
@@ -560,6 +583,8 @@ def main():
     ap.add_argument("--tp-exchange", choices=["nccl", "p2p"], default="nccl",
                     help="with --tp-shards: NCCL all-reduce between two library calls, or the "
                          "exchange fused into the kernels over peer memory")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay the step as a captured CUDA graph in the timed loop")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -568,6 +593,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.tp_shards > 1 and (args.lse0 or args.page_size or args.dynamic_budget):
         ap.error("--tp-shards combines with --constraints and --score only")
+    if args.graph and args.tp_shards > 1 and (args.tp_exchange == "p2p" or args.gpus > 1):
+        ap.error("--graph: the exchange's epoch and the collective must run uncaptured")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

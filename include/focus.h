@@ -42,6 +42,13 @@
  *    `capacity` = sum_r k_r exactly.
  *  - Kept positions are written in ascending order per request; requests are
  *    packed in order: request r owns rows cu_seqlens[r] .. cu_seqlens[r+1]-1.
+ *  - CUDA graphs: every call that enqueues kernels may be captured into a graph
+ *    (it only launches kernels, with programmatic dependent launch between them,
+ *    and never synchronises).  Make one uncaptured call per process first (it
+ *    looks up the driver's tensor-map encoder).  Tensor maps hold the pointers
+ *    given at capture, so a replay reads and writes the same buffers: copy new
+ *    inputs into them before each replay.  focus_read_device_status synchronises
+ *    and cannot be captured.
  */
 #ifndef FOCUS_H_
 #define FOCUS_H_

@@ -806,3 +806,56 @@ def test_other_pool_windows_vs_oracle(window, orc):
     _, want = orc.delta_pool_mask(i0.double().cpu().numpy(), i1.double().cpu().numpy(),
                                   p.decoded.numpy(), window=window)
     assert_close_delta(delta.cpu().numpy(), want)
+
+
+def test_cuda_graph_replay_matches_direct_calls():
+    """focus_evict captured into a CUDA graph (four kernels with programmatic dependent
+    launch edges): replays on new inputs copied into the captured buffers give the same
+    bits as direct calls on those inputs."""
+    import attention_delta_token_b200 as F
+    p = synth.make_problem(1, seed=870, overrides=dict(R=8))
+    g = p.to("cuda")
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+    ws = F.Workspace(dims, "cuda")
+    # capacity for any decoded pattern of the same budgets: the replay's shape is fixed
+    cap = int(p.budget.clamp(min=0).clamp(max=p.B).sum())
+    kept = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+    packed = torch.zeros(cap, p.H, dtype=torch.bfloat16, device="cuda")
+    delta = torch.empty(p.R, p.B, device="cuda")
+
+    def step():
+        F.focus_evict(dims, g.q0, g.k0_prefix, g.k0_block, g.q1, g.k1_prefix, g.k1_block,
+                      g.cu_prefix, g.hidden, g.decoded, g.budget, kept, cu, packed, ws,
+                      delta_out=delta)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()  # the uncaptured first call
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for seed in (871, 872):
+        # new values in the same buffers: the prefix layout (cu_prefix) and the budgets
+        # stay, so the captured capacity still bounds every request's kept count
+        q = synth.make_problem(1, seed=seed, overrides=dict(R=8))
+        for name in ("q0", "k0_block", "q1", "k1_block", "hidden", "decoded"):
+            getattr(g, name).copy_(getattr(q, name))
+        gen = torch.Generator().manual_seed(seed)
+        for name in ("k0_prefix", "k1_prefix"):
+            t = getattr(g, name)
+            t.copy_((torch.randn(t.shape, generator=gen) / p.d ** 0.5).to(torch.bfloat16))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert F.focus_read_device_status(ws) == 0
+        got = [t.clone() for t in (kept, cu, packed.view(torch.int16), delta)]
+        step()
+        assert F.focus_read_device_status(ws) == 0
+        want = [kept, cu, packed.view(torch.int16), delta]
+        n = int(cu[-1])
+        assert n <= cap
+        assert torch.equal(got[1], want[1])
+        assert torch.equal(got[0][:n], want[0][:n]) and torch.equal(got[2][:n], want[2][:n])
+        assert torch.equal(got[3], want[3])
