@@ -66,8 +66,10 @@ focus_status_t check_dims(const focus_dims_t *d) {
     if (G > focus::kTileRows || focus::kTileRows % G != 0) return FOCUS_ERR_UNSUPPORTED_SHAPE;
     const long long rb = static_cast<long long>(d->R) * d->B;
     if (rb > (1ll << 30)) return FOCUS_ERR_UNSUPPORTED_SHAPE;
-    const long long ctas = static_cast<long long>(d->R) * 2 * d->Hkv * row_tiles(*d);
-    if (ctas > 0x7fffffffll) return FOCUS_ERR_UNSUPPORTED_SHAPE;
+    // Work items of the attention kernel; the schedule's item index (round x grid +
+    // offset) stays below 2^31 with room for one more round of the grid.
+    const long long items = static_cast<long long>(d->R) * 2 * d->Hkv * row_tiles(*d);
+    if (items > (1ll << 30)) return FOCUS_ERR_UNSUPPORTED_SHAPE;
     return FOCUS_OK;
 }
 

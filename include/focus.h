@@ -34,7 +34,8 @@
  *  - Shapes: 1 <= B <= 128; head_dim in {64, 128}; Hq % Hkv == 0 and
  *    G = Hq / Hkv divides 128; hidden % 8 == 0; pool_window odd and >= 1;
  *    R >= 1; constraints in 0..3 and score in 0..1 (else FOCUS_ERR_INVALID_ARGUMENT).  Other shapes
- *    return FOCUS_ERR_UNSUPPORTED_SHAPE.
+ *    return FOCUS_ERR_UNSUPPORTED_SHAPE, as do R * B > 2^30 and more than 2^30 attention
+ *    work items (R x 2 layers x Hkv x ceil(G * B / 128) row tiles).
  *  - Per-request budgets are clamped to [0, masked_r] on the device, so
  *    k_r = min(max(budget[r], 0), masked_r).  Without structural constraints
  *    (dims.constraints == 0) k_r depends only on `decoded` and `budget`, never on

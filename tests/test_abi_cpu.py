@@ -74,6 +74,8 @@ BAD_DIMS = [
     (dict(Hq=30, Hkv=8), UNSUPPORTED), (dict(Hq=24, Hkv=8), UNSUPPORTED),
     (dict(Hq=256, Hkv=1), UNSUPPORTED), (dict(hidden=4092), UNSUPPORTED),
     (dict(pool_window=2), UNSUPPORTED),
+    (dict(R=(1 << 30) // 32 + 1), UNSUPPORTED),                       # R * B > 2^30
+    (dict(R=1 << 29, B=1, Hq=2, Hkv=2, head_dim=64), UNSUPPORTED),    # 2^31 work items
 ]
 
 
