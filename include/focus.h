@@ -370,7 +370,10 @@ FOCUS_API focus_status_t focus_evict_from_importance(
  * first push.  Two slot parities make it safe for a rank to run one step ahead.
  * A flag that does not arrive within 2 s sets FOCUS_ERR_TIMEOUT in the device
  * status (read with focus_read_device_status); the sums are then not valid.
- * The workspace must not be shared with another stream while a push runs.
+ * The workspace must not be shared with another stream while a push runs.  The
+ * push counts its finished blocks in the workspace's status region;
+ * focus_clear_device_status resets that count too, so after an error clear the
+ * status of every rank's workspaces, zero the buffers and restart at epoch 1.
  */
 typedef struct {
     void *const *peer_buffers; /* DEVICE array [world] of device pointers: rank q's exchange
