@@ -25,6 +25,15 @@
 //               over the 128 rows (warp butterfly, then the four lane quadrants in
 //               fixed order) go to `partial`.  No float atomics: the result is
 //               deterministic and equal keys give bit-equal columns.
+// Split prefixes (small batches only): when the items would fill at most half of
+// the grid, each item's prefix is split into chunks of at least four key tiles,
+// one work item per chunk.  The chunks of an item come consecutively in the list,
+// the last one also taking the block tile.  The others publish their rows' (m, l)
+// and count themselves; the last waits for the count (bounded) and merges the
+// chunks' statistics in chunk order before forming the block weights.  A chunk only
+// ever waits for chunks listed before it, which never wait, and every CTA of the
+// persistent grid is resident, so the waits always end.  Compiled as a separate
+// instantiation (SPLIT), so the unsplit kernel is unchanged.
 // Exponentials run on the SFU (ex2.approx, fp32).  After a half-row's first full
 // tile the exps are taken against the running reference max without computing
 // each tile's max (the tile's sum reveals a rise).  At the metric shape the
@@ -58,14 +67,40 @@ struct AttnSmem {
 
 struct Item {
     int layer, r, kvh, mt, pstart, L, n_pre;
+    int chunk, n_chunks;  // this item's chunk of the request's prefix, of n_chunks
+    int t0, n_tiles;      // its prefix tiles start at t0; tiles in all (block tile included)
+    bool final;           // the last chunk: also takes the block tile and merges
+    int group;            // (layer, request, kv head, row tile) index of chunk_cnt/chunk_stat
     bool bad;
 };
 
+// Items per request rank: n_layers * Hkv * MT groups, each split into the
+// request's prefix chunks (chunk innermost, so a group's last chunk comes after
+// its other chunks in the list).
+// With SPLIT false (no split prefixes) the chunk fields are compile-time constants
+// (one chunk, tiles from 0, final) and the code folds to the unsplit loop.
+template <bool SPLIT>
 __device__ __forceinline__ Item decode_item(const AttnParams &p, int it) {
     Item w;
     const int per_req = p.n_layers * p.Hkv * p.MT;
-    const int rank = it / per_req;
-    int rem = it - rank * per_req;
+    int rank, rem;
+    if (SPLIT) {
+        int lo = 0, hi = p.R - 1;  // largest rank q with item_base[q] <= it
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.item_base[mid] <= it) lo = mid; else hi = mid - 1;
+        }
+        rank = lo;
+        rem = it - p.item_base[lo];
+        w.n_chunks = max(1, (p.item_base[lo + 1] - p.item_base[lo]) / per_req);
+        w.chunk = rem % w.n_chunks;
+        rem /= w.n_chunks;
+    } else {
+        rank = it / per_req;
+        rem = it - rank * per_req;
+        w.n_chunks = 1;
+        w.chunk = 0;
+    }
     w.layer = rem / (p.Hkv * p.MT);
     rem -= w.layer * p.Hkv * p.MT;
     w.kvh = rem / p.MT;
@@ -90,6 +125,12 @@ __device__ __forceinline__ Item decode_item(const AttnParams &p, int it) {
         w.pstart = 0;
     }
     w.n_pre = (w.L + kTileKeys - 1) / kTileKeys;
+    // chunk c of C takes prefix tiles [c * n_pre / C, (c + 1) * n_pre / C)
+    w.t0 = static_cast<int>(static_cast<long long>(w.chunk) * w.n_pre / w.n_chunks);
+    const int t1 = static_cast<int>(static_cast<long long>(w.chunk + 1) * w.n_pre / w.n_chunks);
+    w.final = w.chunk == w.n_chunks - 1;
+    w.n_tiles = (t1 - w.t0) + (w.final ? 1 : 0);
+    w.group = ((w.layer * p.R + w.r) * p.Hkv + w.kvh) * p.MT + w.mt;
     return w;
 }
 
@@ -102,6 +143,28 @@ __device__ __forceinline__ int item_of_round(int k) {
     const int g = static_cast<int>(gridDim.x);
     const int c = static_cast<int>(blockIdx.x);
     return k * g + ((k & 1) ? g - 1 - c : c);
+}
+
+// One thread waits until the counter reaches `target` (the group's other chunks
+// have published their row statistics).  Bounded: on timeout it sets
+// FOCUS_DEV_TIMEOUT and the abort flag; it also returns when another role aborted.
+__device__ __forceinline__ void wait_chunks(const unsigned int *cnt, unsigned int target,
+                                            uint32_t *status, volatile int *abort_flag) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        unsigned int v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+        if (v >= target) return;
+        if ((it & 63u) == 63u) {
+            if (*abort_flag) return;
+            if (global_timer_ns() - t0 > FOCUS_WAIT_LIMIT_NS) {
+                atomicOr(status, FOCUS_DEV_TIMEOUT);
+                *abort_flag = 1;
+                return;
+            }
+        }
+        __nanosleep(128);
+    }
 }
 
 // Loads 32 TMEM columns of this thread's lane into v[OFF .. OFF+31].
@@ -146,7 +209,7 @@ __device__ __forceinline__ float max64(const float *v) {
     return fmaxf(fmaxf(a, b), fmaxf(c, d));
 }
 
-template <int HEAD_DIM>
+template <int HEAD_DIM, bool SPLIT>
 __global__ void __launch_bounds__(kAttnThreads, 2)
 attn_stats_kernel(const __grid_constant__ AttnParams p) {
     using S = AttnSmem<HEAD_DIM>;
@@ -171,7 +234,6 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n_items = p.R * p.n_layers * p.Hkv * p.MT;
 
     // ---- setup
     if (threadIdx.x == 0) {
@@ -208,6 +270,7 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
     // Everything above overlaps the planner; the request order it writes is read below.
     pdl_launch_dependents();
     pdl_wait();
+    const int n_items = SPLIT ? p.item_base[p.R] : p.R * p.n_layers * p.Hkv * p.MT;
 
     if (warp == 0) {
         // ======================= TMA producer
@@ -219,7 +282,7 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
             int last_q = -1;   // item count of the last Q load issued
             int k = 0;
             for (int it = item_of_round(0); it < n_items; it = item_of_round(++k)) {
-                const Item w = decode_item(p, it);
+                const Item w = decode_item<SPLIT>(p, it);
                 if (w.bad) atomicOr(p.status, FOCUS_DEV_BAD_INPUT);
                 if (!mbar_wait(q_empty, (k & 1) ^ 1, p.status, abort_flag)) break;
                 mbar_arrive_expect_tx(q_full, S::kTileBytes);
@@ -229,7 +292,9 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
                                 w.r * p.B + w.mt * p.tok_per_tile, pol);
                 last_q = k;
                 bool ok = true;
-                for (int t = 0; t <= w.n_pre; ++t, ++kt) {
+                for (int i = 0; i < w.n_tiles; ++i, ++kt) {
+                    const int t = w.t0 + i;                              // prefix tile index
+                    const bool blk = w.final && i == w.n_tiles - 1;      // the block tile
                     const int s = kt % kStages;
                     const uint32_t ph = (kt / kStages) & 1;
                     if (!mbar_wait(&empty[s], ph ^ 1, p.status, abort_flag)) {
@@ -237,7 +302,7 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
                         break;
                     }
                     uint8_t *dst = sK + s * S::kTileBytes;
-                    if (t < w.n_pre && p.page_table) {
+                    if (!blk && p.page_table) {
                         // The tile's keys come from page_rows-row boxes of consecutive pages;
                         // boxes past the prefix are not loaded (their columns are masked).
                         const int first = t * kTileKeys;
@@ -257,7 +322,7 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
                                 tma_load_3d(dst + c * kChunkBytes + u * p.page_rows * 128,
                                             &p.tm_kp[w.layer], &full[s], c * 64, w.kvh, row, pol);
                         }
-                    } else if (t < w.n_pre) {
+                    } else if (!blk) {
                         mbar_arrive_expect_tx(&full[s], S::kTileBytes);
 #pragma unroll
                         for (int c = 0; c < S::kChunks; ++c)
@@ -289,9 +354,10 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
             int k = 0;
             bool ok = true;
             for (int it = item_of_round(0); ok && it < n_items; it = item_of_round(++k)) {
-                const Item w = decode_item(p, it);
+                const Item w = decode_item<SPLIT>(p, it);
                 if (!mbar_wait(q_full, k & 1, p.status, abort_flag)) break;
-                for (int t = 0; t <= w.n_pre; ++t, ++kt, ++st) {
+                for (int i = 0; i < w.n_tiles; ++i, ++kt, ++st) {
+                    const bool blk = w.final && i == w.n_tiles - 1;
                     const int s = kt % kStages;
                     const uint32_t ph = (kt / kStages) & 1;
                     const int buf = st & 1;
@@ -302,7 +368,7 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t idesc = (t < w.n_pre) ? idesc_pre : idesc_blk;
+                    const uint32_t idesc = blk ? idesc_blk : idesc_pre;
                     const uint32_t d_tmem = tmem_base + buf * kTileKeys;
                     const uint32_t b_base = smem_u32(sK + s * S::kTileBytes);
 #pragma unroll
@@ -330,13 +396,16 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
         const float2 c2 = make_float2(c, c);
         uint32_t st = 0;
         int k = 0;
+        int kf = 0;  // final chunks done (the reduction barrier completes once per final chunk)
         bool ok = true;
         for (int it = item_of_round(0); ok && it < n_items; it = item_of_round(++k)) {
-            const Item w = decode_item(p, it);
+            const Item w = decode_item<SPLIT>(p, it);
             const int rows_valid = min(kTileRows, p.G * p.B - w.mt * kTileRows);
             float m = -INFINITY;  // running max of the scaled logits (log2 domain), this half
             float l = 0.f;        // running sum of 2^(x - m), this half
-            for (int t = 0; t <= w.n_pre; ++t, ++st) {
+            for (int i = 0; i < w.n_tiles; ++i, ++st) {
+                const int t = w.t0 + i;
+                const bool blk = w.final && i == w.n_tiles - 1;
                 const int buf = st & 1;
                 const uint32_t bph = (st >> 1) & 1;
                 if (!mbar_wait(&s_full[buf], bph, p.status, abort_flag)) {
@@ -344,7 +413,7 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
                     break;
                 }
                 tc_fence_after();
-                const int ncols = (t < w.n_pre) ? min(kTileKeys, w.L - t * kTileKeys) : p.B;
+                const int ncols = blk ? p.B : min(kTileKeys, w.L - t * kTileKeys);
                 const int nh = min(max(ncols - col0, 0), kHalf);  // valid columns in this half
                 float v[kHalf];
                 if (nh > 0) {
@@ -358,7 +427,7 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s_empty[buf]);
 
-                if (t < w.n_pre) {
+                if (!blk) {
                     if (nh == kHalf && m != -INFINITY) {
                         // Against the running reference m, no tile max is needed: a tile whose
                         // values rose far above m shows up as a large sum (>= 2^20), and only
@@ -432,15 +501,32 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
                     }
                     stat[h * 128 + row] = make_float2(m, l);
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(stat_bar);
-                    if (!mbar_wait(stat_bar, k & 1, p.status, abort_flag)) {
+                    if (lane == 0) {
+                        // With a split prefix the other chunks' statistics must be published
+                        // first; the barrier passes the wait on to the other warps.
+                        if (sw == 0 && w.n_chunks > 1)
+                            wait_chunks(p.chunk_cnt + w.group, w.n_chunks - 1, p.status, abort_flag);
+                        mbar_arrive(stat_bar);
+                    }
+                    if (!mbar_wait(stat_bar, k & 1, p.status, abort_flag) ||
+                        (w.n_chunks > 1 && *abort_flag)) {
                         ok = false;
                         break;
                     }
                     const float2 s0 = stat[row], s1 = stat[128 + row];
                     float M = fmaxf(s0.x, s1.x);  // finite: half 0 always has a column
+                    // the other chunks' (m, l) of this row, merged in chunk order
+                    const int nc = w.n_chunks - 1;
+                    const float2 *cs =
+                        p.chunk_stat + static_cast<size_t>(w.group) * (p.chunk_max - 1) * 256;
+                    for (int q = 0; q < nc; ++q)
+                        M = fmax3(M, __ldcg(cs + q * 256 + row).x, __ldcg(cs + q * 256 + 128 + row).x);
                     float Ltot = s0.y * ex2(s0.x - M) + s1.y * ex2(s1.x - M);
-                    if (p.lse0 && w.layer == 0 && row < rows_valid) {
+                    for (int q = 0; q < nc; ++q) {
+                        const float2 a = __ldcg(cs + q * 256 + row), b = __ldcg(cs + q * 256 + 128 + row);
+                        Ltot += a.y * ex2(a.x - M) + b.y * ex2(b.x - M);
+                    }
+                    if (!SPLIT && p.lse0 && w.layer == 0 && row < rows_valid) {
                         // Given normaliser: p_ij = exp(s_ij - lse_i) = 2^(x_ij - lse_i log2 e).
                         const int tok = w.mt * p.tok_per_tile + row / p.G;
                         const int h = w.kvh * p.G + row % p.G;
@@ -462,7 +548,7 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
                     }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(red_bar);
-                    if (!mbar_wait(red_bar, k & 1, p.status, abort_flag)) {
+                    if (!mbar_wait(red_bar, kf & 1, p.status, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -470,10 +556,32 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
                     if (j < p.B) {
                         const float sum = ((red[0 * 128 + j] + red[1 * 128 + j]) + red[2 * 128 + j]) +
                                           red[3 * 128 + j];
+                        // (layer, request, kv head, row tile): the item's group
                         const size_t idx =
-                            ((((size_t)w.layer * p.R + w.r) * p.Hkv + w.kvh) * p.MT + w.mt) * p.B + j;
+                            SPLIT ? static_cast<size_t>(w.group) * p.B + j
+                                  : ((((size_t)w.layer * p.R + w.r) * p.Hkv + w.kvh) * p.MT + w.mt) * p.B + j;
                         p.partial[idx] = sum;
                     }
+                }
+            }
+            if (!ok) break;
+            if (w.final) {
+                ++kf;
+            } else {
+                // A chunk before the last: publish this row's (m, l) of its half, then
+                // count the chunk once every softmax warp has (release: barrier, fence,
+                // counter).
+                p.chunk_stat[(static_cast<size_t>(w.group) * (p.chunk_max - 1) + w.chunk) * 256 +
+                             h * 128 + row] = make_float2(m, l);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(stat_bar);
+                if (!mbar_wait(stat_bar, k & 1, p.status, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (sw == 0 && lane == 0) {
+                    __threadfence();
+                    atomicAdd(p.chunk_cnt + w.group, 1u);
                 }
             }
         }
@@ -502,27 +610,32 @@ size_t attn_smem_bytes(int head_dim) {
     return head_dim == 64 ? AttnSmem<64>::kAlloc : AttnSmem<128>::kAlloc;
 }
 
+template <int HEAD_DIM, bool SPLIT>
+cudaError_t launch_attn_variant(const AttnParams &p, long long grid, cudaStream_t stream, bool pdl) {
+    const int smem = AttnSmem<HEAD_DIM>::kAlloc;
+    cudaError_t e = cudaFuncSetAttribute(attn_stats_kernel<HEAD_DIM, SPLIT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    return launch_kernel(attn_stats_kernel<HEAD_DIM, SPLIT>, dim3(static_cast<unsigned>(grid)),
+                         dim3(kAttnThreads), smem, stream, pdl, p);
+}
+
 cudaError_t launch_attn_stats(const AttnParams &p, int head_dim, cudaStream_t stream, bool pdl) {
-    const long long items = static_cast<long long>(p.R) * p.n_layers * p.Hkv * p.MT;
+    // With split prefixes each item has up to chunk_max chunks (the exact count is
+    // the planner's); CTAs beyond the items exit at once.
+    const bool split = p.chunk_max > 1;
+    const long long items = static_cast<long long>(p.R) * p.n_layers * p.Hkv * p.MT *
+                            (split ? p.chunk_max : 1);
     if (items <= 0) return cudaSuccess;
     const long long grid = items < 2ll * sm_count() ? items : 2ll * sm_count();
-    if (head_dim == 64) {
-        const int smem = AttnSmem<64>::kAlloc;
-        cudaError_t e = cudaFuncSetAttribute(attn_stats_kernel<64>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        e = launch_kernel(attn_stats_kernel<64>, dim3(static_cast<unsigned>(grid)), dim3(kAttnThreads),
-                          smem, stream, pdl, p);
-        if (e != cudaSuccess) return e;
-    } else {
-        const int smem = AttnSmem<128>::kAlloc;
-        cudaError_t e = cudaFuncSetAttribute(attn_stats_kernel<128>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        e = launch_kernel(attn_stats_kernel<128>, dim3(static_cast<unsigned>(grid)), dim3(kAttnThreads),
-                          smem, stream, pdl, p);
-        if (e != cudaSuccess) return e;
-    }
+    cudaError_t e;
+    if (head_dim == 64)
+        e = split ? launch_attn_variant<64, true>(p, grid, stream, pdl)
+                  : launch_attn_variant<64, false>(p, grid, stream, pdl);
+    else
+        e = split ? launch_attn_variant<128, true>(p, grid, stream, pdl)
+                  : launch_attn_variant<128, false>(p, grid, stream, pdl);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -33,10 +33,30 @@ int row_tiles(const focus_dims_t &d) {
     return (G * d.B + focus::kTileRows - 1) / focus::kTileRows;
 }
 
+// Prefix chunks per attention work item.  A batch whose (layer, request, kv head,
+// row tile) items would occupy at most half of the B200's persistent grid
+// (2 CTAs x 148 SMs) leaves SMs idle, so each item's prefix is split into up to
+// enough chunks for about two waves (at most 16 chunks, each of at least
+// kMinChunkTiles key tiles).  Larger batches are not split: a chunk costs a Q
+// load and a merge, which only pays where SMs would otherwise idle.  Depends on
+// the dims only, so the workspace size does.
+constexpr long long kSplitMaxItems = 148;
+constexpr long long kSplitTargetItems = 2 * 296;
+constexpr int kMaxChunks = 16;
+
+int chunk_max_for(const focus_dims_t &d) {
+    const long long items = 2ll * d.R * d.Hkv * row_tiles(d);
+    if (items > kSplitMaxItems) return 1;
+    const long long c = (kSplitTargetItems + items - 1) / items;
+    return static_cast<int>(c < kMaxChunks ? c : kMaxChunks);
+}
+
 // Workspace: [status 256 B][order: R int32][partial: 2 x R x Hkv x MT x B fp32]
 //            [lists: R x B int32][counts: R int32]   (retained positions under constraints)
+//            and with split prefixes (chunk_max_for > 1): [item_base: R+1 int32]
+//            [chunk_cnt: 2 x R x Hkv x MT uint32][chunk_stat: groups x (chunk_max-1) x 256 float2]
 struct WsLayout {
-    size_t status, order, partial, lists, counts, total;
+    size_t status, order, partial, lists, counts, item_base, chunk_cnt, chunk_stat, total;
 };
 
 WsLayout ws_layout(const focus_dims_t &d) {
@@ -44,10 +64,17 @@ WsLayout ws_layout(const focus_dims_t &d) {
     w.status = 0;
     w.order = kAlign;
     w.partial = w.order + round_up(sizeof(int32_t) * static_cast<size_t>(d.R), kAlign);
-    const size_t np = 2ull * d.R * d.Hkv * row_tiles(d) * d.B;
-    w.lists = w.partial + round_up(sizeof(float) * np, kAlign);
+    const size_t groups = 2ull * d.R * d.Hkv * row_tiles(d);
+    w.lists = w.partial + round_up(sizeof(float) * groups * d.B, kAlign);
     w.counts = w.lists + round_up(sizeof(int32_t) * static_cast<size_t>(d.R) * d.B, kAlign);
     w.total = w.counts + round_up(sizeof(int32_t) * static_cast<size_t>(d.R), kAlign);
+    w.item_base = w.chunk_cnt = w.chunk_stat = w.total;
+    const int cm = chunk_max_for(d);
+    if (cm > 1) {
+        w.chunk_cnt = w.item_base + round_up(sizeof(int32_t) * (static_cast<size_t>(d.R) + 1), kAlign);
+        w.chunk_stat = w.chunk_cnt + round_up(sizeof(uint32_t) * groups, kAlign);
+        w.total = w.chunk_stat + round_up(sizeof(float2) * groups * (cm - 1) * 256, kAlign);
+    }
     return w;
 }
 
@@ -198,6 +225,13 @@ focus_status_t setup_attention(AttnParams &p, const focus_dims_t &d, int layers,
                                int prefix_box = focus::kTileKeys, const float *lse0 = nullptr) {
     memset(&p, 0, sizeof p);
     fill_common(p, d, cu_prefix, total_prefix, ws, layers);
+    p.chunk_max = lse0 ? 1 : chunk_max_for(d);  // layer 0 has no prefix to split with lse0
+    if (p.chunk_max > 1) {
+        const WsLayout w = ws_layout(d);
+        p.item_base = reinterpret_cast<const int32_t *>(ws + w.item_base);
+        p.chunk_cnt = reinterpret_cast<unsigned int *>(ws + w.chunk_cnt);
+        p.chunk_stat = reinterpret_cast<float2 *>(ws + w.chunk_stat);
+    }
     if (layers == 1) {
         FOCUS_TRY(encode_layer(p, 0, d, l1.q, l1.k_prefix, total_prefix, l1.k_block, prefix_box));
         p.tm_q[1] = p.tm_q[0];
@@ -212,6 +246,17 @@ focus_status_t setup_attention(AttnParams &p, const focus_dims_t &d, int layers,
     FOCUS_TRY(encode_layer(p, 1, d, l1.q, l1.k_prefix, total_prefix, l1.k_block, prefix_box));
     p.lse0 = lse0;
     return FOCUS_OK;
+}
+
+// The planner's share of a split-prefix launch: per-rank item offsets and zeroed
+// chunk counters.
+void plan_split(focus::PlanParams &pp, const AttnParams &p) {
+    if (p.chunk_max <= 1) return;
+    pp.chunk_max = p.chunk_max;
+    pp.per_req = p.n_layers * p.Hkv * p.MT;
+    pp.n_groups = p.n_layers * p.R * p.Hkv * p.MT;
+    pp.item_base = const_cast<int32_t *>(p.item_base);
+    pp.chunk_cnt = p.chunk_cnt;
 }
 
 focus_status_t check_attn_inputs(const focus_dims_t &d, const void *q, const void *k_prefix,
@@ -299,6 +344,7 @@ focus_status_t focus_attn_stats(const focus_dims_t *dims, const void *q, const v
     pp.status = p.status;
     pp.R = d.R;
     pp.B = d.B;
+    plan_split(pp, p);
     FOCUS_CUDA(focus::launch_plan(pp, s));
     FOCUS_CUDA(launch_attn_traced(p, d.head_dim, s));
     focus::ReduceParams rp{p.partial, importance, d.R, d.B, d.Hkv, p.MT, 1};
@@ -578,6 +624,7 @@ focus_status_t evict_impl(const focus_dims_t *dims, const focus_evict_args_t &x)
     pp.capacity = x.capacity;
     pp.R = d.R;
     pp.B = d.B;
+    plan_split(pp, p);
     FOCUS_CUDA(focus::launch_plan(pp, s));
     FOCUS_CUDA(launch_attn_traced(p, d.head_dim, s, /*pdl=*/true));
 
@@ -618,6 +665,7 @@ focus_status_t partial_importance_impl(const focus_dims_t *dims, const void *q0,
     pp.status = p.status;
     pp.R = d.R;
     pp.B = d.B;
+    plan_split(pp, p);
     FOCUS_CUDA(focus::launch_plan(pp, s));
     FOCUS_CUDA(launch_attn_traced(p, d.head_dim, s, /*pdl=*/true));
     focus::ReduceParams rp;

@@ -63,7 +63,26 @@ struct AttnParams {
     const int32_t *page_table;  // [R, max_pages]
     const int32_t *prefix_len;  // [R]
     int page_size, max_pages, num_pages, page_rows;
+    // Split prefixes (chunk_max > 1, small batches): a request's prefix tiles are
+    // split evenly into prefix_chunks(L, chunk_max) chunks, one work item each, the
+    // last of which also takes the block tile.  The items of request rank q are
+    // [item_base[q], item_base[q+1]) (chunk innermost).  Every chunk but the last
+    // writes its rows' (m, l) to chunk_stat and counts itself in chunk_cnt[group];
+    // the last waits for the count and merges in chunk order.
+    int chunk_max;
+    const int32_t *item_base;   // [R+1] by request rank (written by the planner)
+    unsigned int *chunk_cnt;    // [n_layers][R][Hkv][MT] (zeroed by the planner)
+    float2 *chunk_stat;         // [n_layers][R][Hkv][MT][chunk_max - 1][2 halves][128 rows]
 };
+
+// Prefix chunks of a request with L prefix keys: at most chunk_max, each of at
+// least kMinChunkTiles key tiles.
+constexpr int kMinChunkTiles = 4;
+__host__ __device__ inline int prefix_chunks(int L, int chunk_max) {
+    const int n_pre = (L > 0 ? L : 0) / kTileKeys + ((L > 0 && L % kTileKeys) ? 1 : 0);
+    const int c = n_pre / kMinChunkTiles;
+    return c < 1 ? 1 : (c < chunk_max ? c : chunk_max);
+}
 
 size_t attn_smem_bytes(int head_dim);
 cudaError_t launch_attn_stats(const AttnParams &p, int head_dim, cudaStream_t stream,
@@ -80,6 +99,12 @@ struct PlanParams {
     uint32_t *status;
     long long capacity;
     int R, B;
+    // Split prefixes (item_base != null): per-rank item offsets of the attention
+    // kernel, prefix_chunks(L, chunk_max) * per_req items per request, and the
+    // chunk counters zeroed.
+    int chunk_max, per_req, n_groups;
+    int32_t *item_base;        // [R+1]
+    unsigned int *chunk_cnt;   // [n_groups]
 };
 cudaError_t launch_plan(const PlanParams &p, cudaStream_t stream);
 

@@ -162,6 +162,27 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
         }
     }
 
+    if (p.item_base) {
+        // Split prefixes: the attention items of request rank q start at item_base[q];
+        // the counters the last chunks wait on start from zero.
+        __syncthreads();  // the order above was written by other threads of this block
+        int running = 0;
+        for (int base = 0; base < R; base += kPlanThreads) {
+            const int q = base + threadIdx.x;
+            int n = 0;
+            if (q < R) {
+                const int r = p.order ? p.order[q] : q;
+                n = prefix_chunks(prefix_length(p, r), p.chunk_max) * p.per_req;
+            }
+            int total;
+            const int ex = block_exclusive_scan(n, warp_tot, total);
+            if (q < R) p.item_base[q] = running + ex;
+            running += total;
+        }
+        if (threadIdx.x == 0) p.item_base[R] = running;
+        for (int i = threadIdx.x; i < p.n_groups; i += blockDim.x) p.chunk_cnt[i] = 0;
+    }
+
     if (p.cu_seqlens) {
         int running = 0;
         if (threadIdx.x == 0) p.cu_seqlens[0] = 0;

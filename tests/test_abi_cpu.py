@@ -52,14 +52,33 @@ def dims(**kw):
     return F.make_dims(**base)
 
 
+def _split_bytes(R, Hkv, MT):
+    """Split-prefix regions: item_base (R+1 int32), chunk counters and chunk statistics
+    ((chunk_max - 1) x 256 float2 per group), each rounded to 256; none for batches of
+    more than 148 (layer, request, kv head, row tile) groups."""
+    groups = 2 * R * Hkv * MT
+    if groups > 148:
+        return 0
+    cm = min(16, -(-592 // groups))
+    up = lambda x: -(-x // 256) * 256
+    return up(4 * (R + 1)) + up(4 * groups) + up(8 * groups * (cm - 1) * 256)
+
+
 def test_workspace_size():
     d = dims()
     n = F.focus_workspace_size(d)
     # status (256) + order (R int32, rounded to 256) + 2 layers x R x Hkv x MT x B fp32
     # + retained lists (R x B int32) + counts (R int32), each rounded to 256
-    assert n == 256 + 256 + 2 * 4 * 8 * 1 * 32 * 4 + 512 + 256
+    base = 256 + 256 + 2 * 4 * 8 * 1 * 32 * 4 + 512 + 256
+    assert n == base + _split_bytes(4, 8, 1)
+    assert _split_bytes(4, 8, 1) == 256 + 256 + 8 * 64 * 9 * 256    # 64 groups: 10 chunks
+    assert _split_bytes(10, 8, 1) == 0                                # 160 groups: no split
     d3 = dims(B=128)  # G*B = 512 -> 4 row tiles
-    assert F.focus_workspace_size(d3) == 256 + 256 + 2 * 4 * 8 * 4 * 128 * 4 + 2048 + 256
+    assert F.focus_workspace_size(d3) == (256 + 256 + 2 * 4 * 8 * 4 * 128 * 4 + 2048 + 256 +
+                                          _split_bytes(4, 8, 4))
+    big = dims(R=256)  # 4096 groups: no split regions
+    assert F.focus_workspace_size(big) == (256 + 1024 + 2 * 256 * 8 * 32 * 4 + 256 * 32 * 4 +
+                                           1024)
     assert F._lib.focus_workspace_size(None) == 0
     assert F._lib.focus_workspace_size(ctypes.byref(dims(B=0))) == 0
 

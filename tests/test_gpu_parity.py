@@ -859,3 +859,81 @@ def test_cuda_graph_replay_matches_direct_calls():
         assert torch.equal(got[1], want[1])
         assert torch.equal(got[0][:n], want[0][:n]) and torch.equal(got[2][:n], want[2][:n])
         assert torch.equal(got[3], want[3])
+
+
+SPLIT_CASES = {
+    # (config, overrides): batches of at most 148 (layer, request, kv head, row tile)
+    # groups, so each group's prefix is split into chunks merged by the last one
+    "r1_l13k": (1, dict(R=1, prefix=("uniform", 12000, 13000))),
+    "r3_mixed": (1, dict(R=3, prefix=("uniform", 300, 6000))),
+    "r2_b128_mt4": (3, dict(R=2, prefix=("uniform", 3000, 5000))),
+    "r4_d64_g16": (1, dict(R=4, d=64, Hq=32, Hkv=2, prefix=("uniform", 2000, 9000))),
+}
+
+
+@pytest.mark.parametrize("case", sorted(SPLIT_CASES))
+def test_split_prefix_vs_oracle_and_deterministic(case, orc):
+    """Split prefixes (several CTAs per (layer, request, kv head, row tile), merged by
+    the last chunk) against the oracle, bit-identical on a second run, and the
+    stand-alone one-layer call splits the same way (bit-identical importance)."""
+    import attention_delta_token_b200 as F
+    cfg, ov = SPLIT_CASES[case]
+    p = synth.make_problem(cfg, seed=880 + sorted(SPLIT_CASES).index(case), wide_logits=True,
+                           overrides=ov)
+    assert 2 * p.R * p.Hkv * -(-p.Hq // p.Hkv * p.B // 128) <= 148
+    ref = orc.evict(p)
+    g = p.to("cuda")
+    a = run_evict(g)
+    _compare_full(p, a, ref)
+    b = run_evict(g)
+    for key in ("i0", "i1", "delta", "kept", "packed", "cu_seqlens"):
+        np.testing.assert_array_equal(a[key], b[key], err_msg=key)
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+    ws = F.Workspace(dims)
+    i1 = torch.empty(p.R, p.B, device="cuda")
+    F.focus_attn_stats(dims, g.q1, g.k1_prefix, g.cu_prefix, g.k1_block, i1, ws)
+    assert F.focus_read_device_status(ws) == 0
+    np.testing.assert_array_equal(i1.cpu().numpy(), a["i1"].astype(np.float32))
+
+
+def test_split_prefix_paged_and_constrained(orc):
+    """Split prefixes through the paged layout and with structural constraints."""
+    import attention_delta_token_b200 as F
+    p = synth.make_problem(1, seed=890, wide_logits=True,
+                           overrides=dict(R=2, prefix=("uniform", 4000, 7000)))
+    ref = orc.evict(p)
+    g = p.to("cuda")
+    packed_out = run_evict(g)
+    pg = synth.to_paged(p, 64, seed=890).to("cuda")
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+    ws = F.Workspace(dims, "cuda")
+    cap = F.plan_capacity(p.decoded, p.budget)
+    kept = torch.empty(cap, dtype=torch.int32, device="cuda")
+    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+    packed = torch.empty(cap, p.H, dtype=torch.bfloat16, device="cuda")
+    i0 = torch.empty(p.R, p.B, device="cuda")
+    i1 = torch.empty(p.R, p.B, device="cuda")
+    F.focus_evict_paged(dims, g.q0, pg.k0_pages, g.k0_block, g.q1, pg.k1_pages, g.k1_block,
+                        pg.page_table, pg.prefix_len, g.hidden, g.decoded, g.budget, kept, cu,
+                        packed, ws, i0_out=i0, i1_out=i1)
+    assert F.focus_read_device_status(ws) == 0
+    # the same chunks over the same keys: bit-identical to the packed layout
+    np.testing.assert_array_equal(i0.cpu().numpy(), packed_out["i0"].astype(np.float32))
+    np.testing.assert_array_equal(i1.cpu().numpy(), packed_out["i1"].astype(np.float32))
+    out = run_evict(g, constraints=3)
+    ref3 = orc.evict(p, constraints=3)
+    assert out["status"] == 0
+    assert_close_delta(out["delta"], ref3["pooled"])
+    check_structured(out["kept"], out["cu_seqlens"], ref3["kept"], ref3["cu_seqlens"],
+                     ref3["pooled"], p.decoded.numpy(), p.budget.numpy())
+
+
+def test_split_prefix_malformed_cu_prefix_reports():
+    """A malformed prefix offset in a split batch: the request is computed with no
+    prefix (its chunks carry no tiles), FOCUS_ERR_DEVICE_CHECK is reported, and no
+    last chunk waits past its bound."""
+    p = synth.make_problem(1, seed=895, overrides=dict(R=3, prefix=("uniform", 3000, 4000)))
+    g = p.to("cuda")
+    g.cu_prefix[2] = g.cu_prefix[3] + 5  # request 1 ends after request 2's end
+    out = run_evict(g)
+    assert out["status"] == 6  # FOCUS_ERR_DEVICE_CHECK, not a timeout
