@@ -227,15 +227,26 @@ def job_throughput(world: int, blocks_per_rank: int, seconds_per_step: float) ->
     return world * blocks_per_rank / seconds_per_step
 
 
+def workload_config(args):
+    """The benchmark's workload: a synthetic config with the command line's overrides
+    (both arms use the same one)."""
+    cfg = synth.CONFIGS[args.config]
+    if args.requests:
+        cfg = synth.FocusConfig(**{**cfg.__dict__, "R": args.requests,
+                                   "name": f"{cfg.name}_r{args.requests}"})
+    if args.prefix:
+        lo, hi = args.prefix
+        cfg = synth.FocusConfig(**{**cfg.__dict__, "prefix": ("uniform", lo, hi),
+                                   "name": f"{cfg.name}_l{lo}_{hi}"})
+    return cfg
+
+
 def run_ours(args, rank, world, local_rank):
     import attention_delta_token_b200 as F
     dist = torch.distributed if world > 1 else None
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    cfg = synth.CONFIGS[args.config]
-    if args.requests:
-        cfg = synth.FocusConfig(**{**cfg.__dict__, "R": args.requests,
-                                   "name": f"{cfg.name}_r{args.requests}"})
+    cfg = workload_config(args)
     tp = args.tp_shards
     # head-sharded ranks all work on the same requests; request-sharded ones on their own
     seed = rank_seed(args.config, 0 if tp > 1 else rank)
@@ -514,9 +525,9 @@ def cpu_baseline(p, target_s: float = 12.0) -> dict:
 def run_reference(args):
     """The float64 CPU oracle on host cores; each step a bounded sample of the workload."""
     import oracle
-    cfg = synth.CONFIGS[args.config]
+    cfg = workload_config(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    p = synth.make_problem(cfg, seed=args.config, device=dev)
+    p = synth.make_problem(cfg, seed=rank_seed(args.config, 0), device=dev)
     threads = oracle.num_threads()
     n = max(1, min(p.R, threads // max(1, p.Hkv)))
     subsets = {}
@@ -545,7 +556,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": cfg.name, "R": p.R, "B": p.B, "Hq": p.Hq, "Hkv": p.Hkv, "d": p.d,
-                   "hidden": p.H, "prefix": list(cfg.prefix), "seed": args.config},
+                   "hidden": p.H, "prefix": list(cfg.prefix), "seed": rank_seed(args.config, 0)},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": f"{n} requests per step, cycling through the {p.R}-block "
                                    f"workload; float64, OpenMP over request x kv-head pairs"},
@@ -564,6 +575,8 @@ def main():
     ap.add_argument("--config", type=int, default=synth.METRIC_CONFIG)
     ap.add_argument("--requests", type=int, default=0,
                     help="override the workload's request count (same shape; for profiling)")
+    ap.add_argument("--prefix", type=int, nargs=2, metavar=("LO", "HI"), default=None,
+                    help="override the prefix lengths: uniform in [LO, HI] keys (same shape otherwise)")
     ap.add_argument("--constraints", type=int, default=0, choices=[0, 1, 2, 3],
                     help="structural constraints on the retained set (bit 1: predecessors, "
                          "bit 2: masked tokens left of the rightmost candidate)")
