@@ -32,8 +32,10 @@
 // and count themselves; the last waits for the count (bounded) and merges the
 // chunks' statistics in chunk order before forming the block weights.  A chunk only
 // ever waits for chunks listed before it, which never wait, and every CTA of the
-// persistent grid is resident, so the waits always end.  Compiled as a separate
-// instantiation (SPLIT), so the unsplit kernel is unchanged.
+// persistent grid is resident (2 per SM: launch bounds cap the registers at 96,
+// 2 x 104 KB of shared memory and 2 x 256 TMEM columns fit an SM), so the waits
+// end; they are bounded all the same.  Compiled as a separate instantiation
+// (SPLIT), so the unsplit kernel is unchanged.
 // Exponentials run on the SFU (ex2.approx, fp32).  After a half-row's first full
 // tile the exps are taken against the running reference max without computing
 // each tile's max (the tile's sum reveals a rise).  At the metric shape the
