@@ -119,8 +119,9 @@ typedef struct {
 /* Bytes of workspace every entry point below needs for `dims` (256-byte aligned). */
 FOCUS_API size_t focus_workspace_size(const focus_dims_t *dims);
 
-/* Zero the workspace's device status word (enqueued on `stream`).  Call once
- * before the first use of a workspace and whenever the status should restart. */
+/* Zero the workspace's status region (enqueued on `stream`): the device status
+ * word and the peer exchange's block counter.  Call once before the first use of
+ * a workspace and whenever the status should restart. */
 FOCUS_API focus_status_t focus_clear_device_status(void *workspace, size_t workspace_bytes, void *stream);
 
 /*
