@@ -937,3 +937,52 @@ def test_split_prefix_malformed_cu_prefix_reports():
     g.cu_prefix[2] = g.cu_prefix[3] + 5  # request 1 ends after request 2's end
     out = run_evict(g)
     assert out["status"] == 6  # FOCUS_ERR_DEVICE_CHECK, not a timeout
+
+
+@pytest.mark.parametrize("case", ["sdar_r8_wide", "block128_r3"])
+def test_all_options_together_vs_oracle(case, orc):
+    """focus_evict_ex with every option at once: paged prefix keys (64-token pages), the
+    layer-0 row log-sum-exps given, the dynamic budget and both structural constraints,
+    against the oracle run with the same options."""
+    import attention_delta_token_b200 as F
+    cfg, ov, wide = STRUCTURED_CASES[case]
+    p = synth.make_problem(cfg, seed=910, wide_logits=wide, overrides=ov)
+    lse = _row_lse(p).float()
+    avg = np.random.default_rng(9).uniform(0.0, 4.0, size=p.R).astype(np.float32)
+    ref = orc.evict(p, constraints=3, lse0=lse.double().numpy(), decode_avg=avg.astype(np.float64))
+    g = p.to("cuda")
+    pg = synth.to_paged(p, 64, seed=910).to("cuda")
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, 3)
+    ws = F.Workspace(dims)
+    cap = F.plan_capacity(p.decoded, None, 3, dynamic=True)
+    kept = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+    packed = torch.zeros(cap, p.H, dtype=torch.bfloat16, device="cuda")
+    delta = torch.empty(p.R, p.B, device="cuda")
+    i0 = torch.empty_like(delta)
+    i1 = torch.empty_like(delta)
+    kout = torch.full((p.R,), -1, dtype=torch.int32, device="cuda")
+    F.focus_evict_ex(dims, q0=g.q0, k0_block=g.k0_block, lse0=lse.cuda(), q1=g.q1,
+                     k1_prefix=pg.k1_pages, k1_block=g.k1_block, page_table=pg.page_table,
+                     prefix_len=pg.prefix_len, hidden=g.hidden, decoded=g.decoded,
+                     decode_avg=torch.from_numpy(avg).cuda(), budget_alpha=1.5, budget_out=kout,
+                     kept_idx=kept, cu_seqlens=cu, packed=packed, ws=ws, delta_out=delta,
+                     i0_out=i0, i1_out=i1)
+    assert F.focus_read_device_status(ws) == 0
+    assert_close_importance(i0.cpu().numpy(), ref["i0"], "I0 from lse")
+    assert_close_importance(i1.cpu().numpy(), ref["i1"], "I1 (paged)")
+    assert_close_delta(delta.cpu().numpy(), ref["pooled"])
+    kg = kout.cpu().numpy()
+    dec = p.decoded.numpy()
+    decided = [r for r in range(p.R) if kg[r] == ref["budget"][r]]
+    assert len(decided) >= p.R // 2
+    cu_h = cu.cpu().numpy()
+    n = int(cu_h[-1])
+    # retained sets of the requests whose budget the oracle agrees on (the oracle run on
+    # exactly those requests, as check_structured indexes them)
+    sub = orc.evict(p.subset(decided), constraints=3, lse0=lse[decided].double().numpy(),
+                    decode_avg=avg[decided].astype(np.float64))
+    check_structured(kept[:n].cpu().numpy(), cu_h, sub["kept"], sub["cu_seqlens"], sub["pooled"],
+                     dec, kg, requests=decided)
+    check_packed(packed[:n].view(torch.int16).cpu().numpy().view(np.uint16),
+                 kept[:n].cpu().numpy(), cu_h, hidden_bits(p))
