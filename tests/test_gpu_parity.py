@@ -986,3 +986,37 @@ def test_all_options_together_vs_oracle(case, orc):
                      dec, kg, requests=decided)
     check_packed(packed[:n].view(torch.int16).cpu().numpy().view(np.uint16),
                  kept[:n].cpu().numpy(), cu_h, hidden_bits(p))
+
+
+def test_paged_bad_entries_report():
+    """A page index outside the pool (the copy falls back to page 0, in bounds) and a
+    prefix length beyond the request's pages (computed with no prefix) are reported as
+    FOCUS_ERR_DEVICE_CHECK; the call stays in bounds and later calls are unaffected."""
+    import attention_delta_token_b200 as F
+    p = synth.make_problem(1, seed=920, overrides=dict(R=3, prefix=("uniform", 300, 600)))
+    g = p.to("cuda")
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+    cap = F.plan_capacity(p.decoded, p.budget)
+
+    def call(pg):
+        ws = F.Workspace(dims)
+        kept = torch.empty(cap, dtype=torch.int32, device="cuda")
+        cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+        packed = torch.empty(cap, p.H, dtype=torch.bfloat16, device="cuda")
+        F.focus_evict_paged(dims, g.q0, pg.k0_pages, g.k0_block, g.q1, pg.k1_pages, g.k1_block,
+                            pg.page_table, pg.prefix_len, g.hidden, g.decoded, g.budget, kept, cu,
+                            packed, ws)
+        return F.focus_read_device_status(ws)
+
+    pg = synth.to_paged(p, 64, seed=920).to("cuda")
+    assert call(pg) == 0
+    bad = synth.to_paged(p, 64, seed=920).to("cuda")
+    bad.page_table[1, 0] = bad.k1_pages.shape[0] + 5     # past the pool
+    assert call(bad) == 6
+    bad = synth.to_paged(p, 64, seed=920).to("cuda")
+    bad.page_table[2, 1] = -1
+    assert call(bad) == 6
+    bad = synth.to_paged(p, 64, seed=920).to("cuda")
+    bad.prefix_len[0] = bad.page_table.shape[1] * 64 + 1  # longer than its pages
+    assert call(bad) == 6
+    assert call(pg) == 0
