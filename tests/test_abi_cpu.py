@@ -341,3 +341,29 @@ def test_c_program_links_and_calls_the_library(tmp_path):
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
     assert r.stdout.startswith("ok ")
     assert int(r.stdout.split()[1]) == F.focus_workspace_size(dims())
+
+
+def test_binding_rejects_bad_tensors_before_the_library():
+    """The Python binding only marshals: it refuses host tensors, wrong dtypes and
+    non-contiguous views (with the argument's name) before anything reaches the C ABI."""
+    d = dims(R=1, B=32, Hq=4, Hkv=2, head_dim=64, hidden=256)
+    cpu = torch.zeros(4, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="q0: must be a CUDA tensor"):
+        F._ptr(cpu, torch.bfloat16, "q0")
+    with pytest.raises(TypeError, match="expected a torch.Tensor"):
+        F._ptr([1, 2], None, "q1")
+    meta = torch.empty(8, 8, dtype=torch.float32, device="meta")
+    with pytest.raises(ValueError):
+        F._ptr(meta, torch.float32, "delta")  # not a CUDA tensor either
+    assert F._ptr(None, torch.float32, "delta_out") is None
+    with pytest.raises(ValueError, match="importance must be"):
+        F.focus_partial_importance(d, None, None, None, None, None, None, None,
+                                   torch.zeros(3, 1, 32), None)
+    with pytest.raises(ValueError, match="importance must be"):
+        F.focus_evict_from_importance(d, torch.zeros(2, 2, 32), None, None, None, None, None,
+                                      None, None)
+    with pytest.raises(ValueError, match="one address per rank"):
+        F.focus_partial_importance_push(d, None, None, None, None, None, None, None,
+                                        torch.zeros(3, dtype=torch.int64), 0, 2, 1, None)
+    with pytest.raises(F.FocusError):
+        F.focus_exchange_buffer_size(d, 9)
