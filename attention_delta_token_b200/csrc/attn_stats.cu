@@ -94,9 +94,19 @@ __device__ __forceinline__ Item decode_item(const AttnParams &p, int it) {
         }
         rank = lo;
         rem = it - p.item_base[lo];
-        w.n_chunks = max(1, (p.item_base[lo + 1] - p.item_base[lo]) / per_req);
-        w.chunk = rem % w.n_chunks;
-        rem /= w.n_chunks;
+        // With layer 0's log-sum-exps given its groups stream no prefix: they come
+        // first, one item each, then the split groups, chunk innermost.
+        const int single = (p.lse0 && p.n_layers == 2) ? p.Hkv * p.MT : 0;
+        if (rem < single) {
+            w.n_chunks = 1;
+            w.chunk = 0;
+        } else {
+            const int items = p.item_base[lo + 1] - p.item_base[lo];
+            w.n_chunks = max(1, (items - single) / (per_req - single));
+            const int r2 = rem - single;
+            w.chunk = r2 % w.n_chunks;
+            rem = single + r2 / w.n_chunks;
+        }
     } else {
         rank = it / per_req;
         rem = it - rank * per_req;
@@ -528,7 +538,7 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
                         const float2 a = __ldcg(cs + q * 256 + row), b = __ldcg(cs + q * 256 + 128 + row);
                         Ltot += a.y * ex2(a.x - M) + b.y * ex2(b.x - M);
                     }
-                    if (!SPLIT && p.lse0 && w.layer == 0 && row < rows_valid) {
+                    if (p.lse0 && w.layer == 0 && row < rows_valid) {
                         // Given normaliser: p_ij = exp(s_ij - lse_i) = 2^(x_ij - lse_i log2 e).
                         const int tok = w.mt * p.tok_per_tile + row / p.G;
                         const int h = w.kvh * p.G + row % p.G;

@@ -225,7 +225,7 @@ focus_status_t setup_attention(AttnParams &p, const focus_dims_t &d, int layers,
                                int prefix_box = focus::kTileKeys, const float *lse0 = nullptr) {
     memset(&p, 0, sizeof p);
     fill_common(p, d, cu_prefix, total_prefix, ws, layers);
-    p.chunk_max = lse0 ? 1 : chunk_max_for(d);  // layer 0 has no prefix to split with lse0
+    p.chunk_max = chunk_max_for(d);
     if (p.chunk_max > 1) {
         const WsLayout w = ws_layout(d);
         p.item_base = reinterpret_cast<const int32_t *>(ws + w.item_base);
@@ -253,7 +253,9 @@ focus_status_t setup_attention(AttnParams &p, const focus_dims_t &d, int layers,
 void plan_split(focus::PlanParams &pp, const AttnParams &p) {
     if (p.chunk_max <= 1) return;
     pp.chunk_max = p.chunk_max;
-    pp.per_req = p.n_layers * p.Hkv * p.MT;
+    // With layer 0's log-sum-exps given, its groups have no prefix: one item each.
+    pp.single_groups = (p.lse0 && p.n_layers == 2) ? p.Hkv * p.MT : 0;
+    pp.per_req = p.n_layers * p.Hkv * p.MT - pp.single_groups;
     pp.n_groups = p.n_layers * p.R * p.Hkv * p.MT;
     pp.item_base = const_cast<int32_t *>(p.item_base);
     pp.chunk_cnt = p.chunk_cnt;

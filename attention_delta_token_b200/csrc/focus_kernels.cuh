@@ -100,9 +100,10 @@ struct PlanParams {
     long long capacity;
     int R, B;
     // Split prefixes (item_base != null): per-rank item offsets of the attention
-    // kernel, prefix_chunks(L, chunk_max) * per_req items per request, and the
-    // chunk counters zeroed.
-    int chunk_max, per_req, n_groups;
+    // kernel, single_groups + prefix_chunks(L, chunk_max) * per_req items per
+    // request (single_groups: layer-0 groups that stream no prefix when layer 0's
+    // row log-sum-exps are given), and the chunk counters zeroed.
+    int chunk_max, per_req, single_groups, n_groups;
     int32_t *item_base;        // [R+1]
     unsigned int *chunk_cnt;   // [n_groups]
 };

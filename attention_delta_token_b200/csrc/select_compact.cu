@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
             int n = 0;
             if (q < R) {
                 const int r = p.order ? p.order[q] : q;
-                n = prefix_chunks(prefix_length(p, r), p.chunk_max) * p.per_req;
+                n = p.single_groups + prefix_chunks(prefix_length(p, r), p.chunk_max) * p.per_req;
             }
             int total;
             const int ex = block_exclusive_scan(n, warp_tot, total);

@@ -1020,3 +1020,39 @@ def test_paged_bad_entries_report():
     bad.prefix_len[0] = bad.page_table.shape[1] * 64 + 1  # longer than its pages
     assert call(bad) == 6
     assert call(pg) == 0
+
+
+def test_split_prefix_with_lse0_vs_oracle(orc):
+    """Split prefixes with layer 0's row log-sum-exps given: the layer-0 groups (block keys
+    only) stay whole, the layer-1 groups are split; against the oracle's importance from
+    the LSE, and bit-identical on a second run."""
+    import attention_delta_token_b200 as F
+    p = synth.make_problem(1, seed=930, wide_logits=True,
+                           overrides=dict(R=2, prefix=("uniform", 8000, 9000)))
+    assert 2 * p.R * p.Hkv <= 148  # a split batch
+    lse = _row_lse(p).float()
+    ref = orc.evict(p, lse0=lse.double().numpy())
+    g = p.to("cuda")
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+    cap = F.plan_capacity(p.decoded, p.budget)
+    outs = []
+    for _ in range(2):
+        ws = F.Workspace(dims)
+        kept = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+        cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+        packed = torch.zeros(cap, p.H, dtype=torch.bfloat16, device="cuda")
+        i0 = torch.empty(p.R, p.B, device="cuda")
+        i1 = torch.empty_like(i0)
+        delta = torch.empty_like(i0)
+        F.focus_evict_with_lse0(dims, lse.cuda(), g.q0, g.k0_block, g.q1, g.k1_prefix, g.k1_block,
+                                g.cu_prefix, g.hidden, g.decoded, g.budget, kept, cu, packed, ws,
+                                delta_out=delta, i0_out=i0, i1_out=i1)
+        assert F.focus_read_device_status(ws) == 0
+        outs.append([t.cpu() for t in (i0, i1, delta, kept, cu)])
+    i0, i1, delta, kept, cu = outs[0]
+    assert_close_importance(i0.numpy(), ref["i0"], "I0 from lse")
+    assert_close_importance(i1.numpy(), ref["i1"], "I1 (split)")
+    assert_close_delta(delta.numpy(), ref["pooled"])
+    check_selection(kept.numpy(), cu.numpy(), ref["pooled"], p.decoded.numpy(), p.budget.numpy())
+    for a, b in zip(outs[0], outs[1]):
+        assert torch.equal(a, b)
