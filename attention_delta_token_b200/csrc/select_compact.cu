@@ -103,8 +103,9 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int *warp_tot, int &t
 
 // One CTA: (a) the processing order of the requests, longest prefix first
 // (ranks of (L desc, r asc) keys), so the attention CTAs of the longest requests
-// start in the first wave; (b) k_r and cu_seqlens (depend only on decoded and
-// budget) and the capacity check.
+// start in the first wave; (b) with split prefixes, each request's first
+// attention item and zeroed chunk counters; (c) k_r and cu_seqlens (depend only on
+// decoded and budget) and the capacity check.
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) {
     __shared__ unsigned long long keys[kMaxSortR];
     __shared__ int warp_tot[33];
