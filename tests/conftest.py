@@ -11,6 +11,15 @@ for _p in (ROOT, os.path.join(ROOT, "tests")):
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    # The in-tree CUDA library must match the sources before the package is imported: a
+    # fresh checkout has no libfocus.so (the oracle builds itself on first use).  Nothing
+    # happens when it is up to date.
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_focus_build", os.path.join(ROOT, "attention_delta_token_b200", "build.py"))
+    builder = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(builder)
+    builder.build()
 
 
 @pytest.fixture(scope="session")
