@@ -1056,3 +1056,75 @@ def test_split_prefix_with_lse0_vs_oracle(orc):
     check_selection(kept.numpy(), cu.numpy(), ref["pooled"], p.decoded.numpy(), p.budget.numpy())
     for a, b in zip(outs[0], outs[1]):
         assert torch.equal(a, b)
+
+
+def _guarded(n, dtype, fill, guard=256):
+    """A device buffer of n elements with `guard` sentinel elements on each side; returns
+    (whole, inner view).  Integer sentinels for integer dtypes, NaN bit patterns otherwise."""
+    whole = torch.empty(n + 2 * guard, dtype=dtype, device="cuda")
+    whole.view(torch.uint8).fill_(fill)
+    return whole, whole[guard:guard + n]
+
+
+def _guards_intact(whole, n, fill, guard=256):
+    b = whole.view(torch.uint8)
+    per = whole.element_size()
+    return bool((b[:guard * per] == fill).all()) and bool((b[(guard + n) * per:] == fill).all())
+
+
+@pytest.mark.parametrize("mode", ["plain", "constraints", "split", "paged", "static"])
+def test_outputs_and_workspace_guard_zones(mode):
+    """Canary zones before and after every output buffer and the workspace stay
+    untouched: no kernel writes outside the ranges the ABI gives it."""
+    import attention_delta_token_b200 as F
+    ov = dict(R=3, prefix=("uniform", 4000, 6000)) if mode == "split" else \
+        dict(R=20, prefix=("uniform", 100, 900))
+    p = synth.make_problem(1, seed=940, overrides=ov)
+    g = p.to("cuda")
+    constraints = 3 if mode == "constraints" else 0
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, constraints)
+    cap = F.plan_capacity(p.decoded, p.budget, constraints)
+    fill = 0xA5
+    bufs = {
+        "kept": (cap, torch.int32), "cu": (p.R + 1, torch.int32),
+        "packed": (cap * p.H, torch.bfloat16), "delta": (p.R * p.B, torch.float32),
+        "i0": (p.R * p.B, torch.float32), "i1": (p.R * p.B, torch.float32),
+    }
+    whole, inner = {}, {}
+    for k, (n, dt) in bufs.items():
+        whole[k], inner[k] = _guarded(n, dt, fill)
+    ws_bytes = F.focus_workspace_size(dims)
+    ws_whole, ws_inner = _guarded(ws_bytes, torch.uint8, fill, guard=4096)
+    ws = F.Workspace.__new__(F.Workspace)
+    ws.nbytes, ws.buf = ws_bytes, ws_inner
+    assert ws_inner.data_ptr() % 256 == 0
+    F.focus_clear_device_status(ws)
+    packed = inner["packed"].view(cap, p.H)
+    if mode == "paged":
+        pg = synth.to_paged(p, 64, seed=940).to("cuda")
+        F.focus_evict_paged(dims, g.q0, pg.k0_pages, g.k0_block, g.q1, pg.k1_pages, g.k1_block,
+                            pg.page_table, pg.prefix_len, g.hidden, g.decoded, g.budget,
+                            inner["kept"], inner["cu"], packed, ws,
+                            delta_out=inner["delta"].view(p.R, p.B),
+                            i0_out=inner["i0"].view(p.R, p.B), i1_out=inner["i1"].view(p.R, p.B))
+    elif mode == "static":
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        F.focus_evict_static_scratch(dims, g.q0, g.k0_prefix, g.k0_block, g.q1, g.k1_prefix,
+                                     g.k1_block, g.cu_prefix, g.hidden, g.decoded, g.budget,
+                                     inner["kept"], inner["cu"], packed, device_status=st,
+                                     delta_out=inner["delta"].view(p.R, p.B),
+                                     i0_out=inner["i0"].view(p.R, p.B),
+                                     i1_out=inner["i1"].view(p.R, p.B))
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+    else:
+        F.focus_evict(dims, g.q0, g.k0_prefix, g.k0_block, g.q1, g.k1_prefix, g.k1_block,
+                      g.cu_prefix, g.hidden, g.decoded, g.budget, inner["kept"], inner["cu"],
+                      packed, ws, delta_out=inner["delta"].view(p.R, p.B),
+                      i0_out=inner["i0"].view(p.R, p.B), i1_out=inner["i1"].view(p.R, p.B))
+    if mode != "static":
+        assert F.focus_read_device_status(ws) == 0
+    torch.cuda.synchronize()
+    for k, (n, _) in bufs.items():
+        assert _guards_intact(whole[k], n, fill), k
+    assert _guards_intact(ws_whole, ws_bytes, fill, guard=4096), "workspace"
