@@ -14,6 +14,8 @@
 #include <mutex>
 #include <thread>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "focus.h"
 #include "focus_device.cuh"
 #include "focus_kernels.cuh"
@@ -21,6 +23,15 @@
 namespace {
 
 using focus::AttnParams;
+
+// A named range around each call, for profiler timelines (NVTX; without a tool
+// attached it costs a few nanoseconds).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 constexpr size_t kAlign = 256;
 
@@ -326,6 +337,7 @@ focus_status_t focus_attn_stats(const focus_dims_t *dims, const void *q, const v
                                 const int32_t *cu_prefix, int64_t total_prefix,
                                 const void *k_block, float *importance, void *workspace,
                                 size_t workspace_bytes, void *stream) {
+    NvtxRange nvtx_range("focus_attn_stats");
     FOCUS_TRY(check_dims(dims));
     const focus_dims_t &d = *dims;
     FOCUS_TRY(check_attn_inputs(d, q, k_prefix, cu_prefix, total_prefix, k_block));
@@ -357,6 +369,7 @@ focus_status_t focus_attn_stats(const focus_dims_t *dims, const void *q, const v
 focus_status_t focus_importance_delta(const focus_dims_t *dims, const float *i0, const float *i1,
                                       const uint8_t *decoded, float *delta, float *raw_delta,
                                       void *stream) {
+    NvtxRange nvtx_range("focus_importance_delta");
     FOCUS_TRY(check_dims(dims));
     FOCUS_TRY(check_ptr(i0, 4));
     FOCUS_TRY(check_ptr(i1, 4));
@@ -372,6 +385,7 @@ focus_status_t focus_topk_select(const focus_dims_t *dims, const float *delta,
                                  const uint8_t *decoded, const int32_t *budget, int32_t *kept_idx,
                                  int32_t *cu_seqlens, int64_t capacity, void *workspace,
                                  size_t workspace_bytes, void *stream) {
+    NvtxRange nvtx_range("focus_topk_select");
     FOCUS_TRY(check_dims(dims));
     const focus_dims_t &d = *dims;
     FOCUS_TRY(check_ptr(delta, 4));
@@ -429,6 +443,7 @@ focus_status_t focus_topk_select(const focus_dims_t *dims, const float *delta,
 focus_status_t focus_compact(const focus_dims_t *dims, const void *hidden, const int32_t *kept_idx,
                              const int32_t *cu_seqlens, void *packed, int64_t capacity,
                              void *workspace, size_t workspace_bytes, void *stream) {
+    NvtxRange nvtx_range("focus_compact");
     FOCUS_TRY(check_dims(dims));
     const focus_dims_t &d = *dims;
     FOCUS_TRY(check_ptr(hidden, 16));
@@ -550,6 +565,7 @@ focus_status_t launch_tail(const focus_dims_t &d, const Tail &t, uint8_t *ws, cu
 }
 
 focus_status_t evict_impl(const focus_dims_t *dims, const focus_evict_args_t &x) {
+    NvtxRange nvtx_range("focus_evict");
     FOCUS_TRY(check_dims(dims));
     const focus_dims_t &d = *dims;
     const bool layer1_only = d.score == FOCUS_SCORE_LAYER1;
@@ -645,6 +661,7 @@ focus_status_t partial_importance_impl(const focus_dims_t *dims, const void *q0,
                                        int64_t total_prefix, float *importance,
                                        const focus_exchange_t *ex, void *workspace,
                                        size_t workspace_bytes, void *stream) {
+    NvtxRange nvtx_range("focus_partial_importance");
     FOCUS_TRY(check_dims(dims));
     const focus_dims_t &d = *dims;
     const bool layer1_only = d.score == FOCUS_SCORE_LAYER1;
@@ -700,6 +717,7 @@ focus_status_t evict_from_sums(const focus_dims_t *dims, const float *sums, int 
                                int32_t *cu_seqlens, void *packed, int64_t capacity,
                                float *delta_out, void *workspace, size_t workspace_bytes,
                                void *stream) {
+    NvtxRange nvtx_range("focus_evict_from_importance");
     const focus_dims_t &d = *dims;
     FOCUS_TRY(check_ptr(hidden, 16));
     FOCUS_TRY(check_ptr(decoded, 1));
