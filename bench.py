@@ -490,7 +490,9 @@ def run_ours(args, rank, world, local_rank):
             "clocks": clocks,
             # plan, attention statistics, select, (scan,) compact; split into two calls
             # (tp): plan, attention, reduce + plan, select, (scan,) compact
-            "gpu_launches": ((5 if args.constraints else 4) + (2 if tp > 1 else 0)) * args.steps,
+            # (list mode: structural constraints or the dynamic budget add the scan kernel)
+            "gpu_launches": ((5 if (args.constraints or args.dynamic_budget) else 4) +
+                             (2 if tp > 1 else 0)) * args.steps,
             "e2e": e2e,
             "impl": "ours",
         }
