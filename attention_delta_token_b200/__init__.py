@@ -23,6 +23,7 @@ __all__ = [
     "focus_clear_device_status", "focus_read_device_status", "focus_attn_stats",
     "focus_importance_delta", "focus_topk_select", "focus_compact", "focus_evict",
     "focus_status_string", "focus_abi_version", "focus_set_trace_events", "plan_capacity",
+    "focus_plan_capacity",
     "focus_evict_static_scratch", "STATIC_SCRATCH_BYTES", "focus_selftest_wait_timeout",
     "focus_partial_importance", "focus_evict_from_importance", "FocusExchange",
     "focus_exchange_buffer_size", "focus_partial_importance_push", "focus_evict_from_exchange",
@@ -91,6 +92,7 @@ def _load() -> ctypes.CDLL:
     D = ctypes.POINTER(FocusDims)
     sig = {
         "focus_workspace_size": (sz, [D]),
+        "focus_plan_capacity": (ctypes.c_int, [D, P, P, ctypes.c_int, ctypes.POINTER(i64)]),
         "focus_clear_device_status": (ctypes.c_int, [P, sz, P]),
         "focus_read_device_status": (ctypes.c_int, [P, P, ctypes.c_int]),
         "focus_attn_stats": (ctypes.c_int, [D, P, P, P, i64, P, P, P, sz, P]),
@@ -467,24 +469,29 @@ def focus_selftest_wait_timeout(status, elapsed_ns, limit_ns: int, stream=None):
                                          _stream(stream)), "focus_selftest_wait_timeout")
 
 
-def plan_capacity(decoded, budget, constraints: int = 0, dynamic: bool = False) -> int:
-    """Rows the packed batch needs: sum_r k_r with k_r = min(max(budget_r, 0), masked_r)
-    (with `dynamic`, k_r = masked_r: the dynamic budget never exceeds it).
+def focus_plan_capacity(dims: FocusDims, decoded, budget=None, dynamic: bool = False) -> int:
+    """Rows the packed batch needs (the C entry point of the same name): the kept count
+    of every request from the scheduler's `decoded` [R, B] uint8 and `budget` [R] int32,
+    exact without structural constraints, an upper bound with them (see focus.h).
+    Tensors on any device; they are copied to host memory, which the call reads."""
+    dec = decoded.detach().to("cpu", torch.uint8).contiguous()
+    if tuple(dec.shape) != (dims.R, dims.B):
+        raise ValueError(f"decoded must be [{dims.R}, {dims.B}]")
+    bud = None
+    if not dynamic:
+        bud = budget.detach().to("cpu", torch.int32).contiguous()
+        if tuple(bud.shape) != (dims.R,):
+            raise ValueError(f"budget must be [{dims.R}]")
+    out = ctypes.c_int64(-1)
+    _ok(_lib.focus_plan_capacity(ctypes.byref(dims), ctypes.c_void_p(dec.data_ptr()),
+                                 ctypes.c_void_p(bud.data_ptr()) if bud is not None else None,
+                                 int(bool(dynamic)), ctypes.byref(out)), "focus_plan_capacity")
+    return int(out.value)
 
-    Host-side planning helper for the scheduler that owns `decoded` and
-    `budget`: without structural constraints the kept-row counts never depend on
-    the attention data, so this is exact.  With constraints it is the upper bound
-    sum_r min(B, masked_r + k_r) over requests with k_r > 0 (candidates, their
-    predecessors and the other masked tokens)."""
-    dec = decoded.detach().cpu()
-    masked = (dec == 0).sum(dim=1).to(torch.int64)
-    if dynamic:  # a dynamic budget is at most the number of masked positions
-        k = masked
-    else:
-        bud = budget.detach().cpu().to(torch.int64)
-        k = torch.minimum(bud.clamp(min=0), masked)
-    if not constraints:
-        return int(k.sum())
-    B = dec.shape[1]
-    bound = torch.where(k > 0, torch.clamp(masked + k, max=B), torch.zeros_like(k))
-    return int(bound.sum())
+
+def plan_capacity(decoded, budget, constraints: int = 0, dynamic: bool = False) -> int:
+    """focus_plan_capacity for a batch described only by its arrays (the dims it needs
+    are R, B and the constraint bits; the other fields are placeholders)."""
+    R, B = int(decoded.shape[0]), int(decoded.shape[1])
+    dims = make_dims(R, B, 1, 1, 64, 8, 1.0, 1, constraints)
+    return focus_plan_capacity(dims, decoded, budget, dynamic)

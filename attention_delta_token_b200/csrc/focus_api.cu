@@ -292,6 +292,30 @@ size_t focus_workspace_size(const focus_dims_t *dims) {
     return ws_layout(*dims).total;
 }
 
+focus_status_t focus_plan_capacity(const focus_dims_t *dims, const uint8_t *decoded_host,
+                                   const int32_t *budget_host, int dynamic,
+                                   int64_t *capacity_out) {
+    FOCUS_TRY(check_dims(dims));
+    if (!decoded_host || !capacity_out || (!dynamic && !budget_host))
+        return FOCUS_ERR_INVALID_ARGUMENT;
+    const focus_dims_t &d = *dims;
+    int64_t rows = 0;
+    for (int r = 0; r < d.R; ++r) {
+        const uint8_t *dec = decoded_host + static_cast<size_t>(r) * d.B;
+        int64_t masked = 0;
+        for (int j = 0; j < d.B; ++j) masked += dec[j] == 0;
+        // a dynamic budget is at most the masked count; a given one is clamped to it
+        const int64_t want = dynamic ? masked : (budget_host[r] > 0 ? budget_host[r] : 0);
+        const int64_t k = want < masked ? want : masked;
+        if (d.constraints == 0)
+            rows += k;
+        else if (k > 0)
+            rows += masked + k < d.B ? masked + k : d.B;
+    }
+    *capacity_out = rows;
+    return FOCUS_OK;
+}
+
 focus_status_t focus_clear_device_status(void *workspace, size_t workspace_bytes, void *stream) {
     if (!workspace || !aligned(workspace, kAlign) || workspace_bytes < kAlign)
         return FOCUS_ERR_WORKSPACE;
@@ -564,31 +588,41 @@ focus_status_t launch_tail(const focus_dims_t &d, const Tail &t, uint8_t *ws, cu
     return FOCUS_OK;
 }
 
-focus_status_t evict_impl(const focus_dims_t *dims, const focus_evict_args_t &x) {
-    NvtxRange nvtx_range("focus_evict");
+// What the host validation of a fused call derives from its arguments.
+struct EvictInputs {
+    const int32_t *cu_prefix;  // packed offsets, or the paged prefix lengths
+    long long total_prefix;    // rows of the prefix buffers (or page-pool rows)
+    int prefix_box;            // rows per prefix TMA box
+    Paging pg;
+    bool paged;
+};
+
+// Every host-side check of the fused step, in order; nothing is enqueued.
+focus_status_t check_evict(const focus_dims_t *dims, const focus_evict_args_t &x, EvictInputs *in) {
     FOCUS_TRY(check_dims(dims));
     const focus_dims_t &d = *dims;
     const bool layer1_only = d.score == FOCUS_SCORE_LAYER1;
     const bool dynamic = x.decode_avg != nullptr;
-    const int32_t *cu_prefix = x.cu_prefix;
-    long long total_prefix = x.total_prefix;
-    int prefix_box = focus::kTileKeys;
-    const Paging pg{x.page_table, x.prefix_len, x.max_pages, x.num_pages, x.page_size};
-    const Paging *paging = x.page_table ? &pg : nullptr;
-    if (paging) {  // the page pools stand in for the packed prefix buffers
-        FOCUS_TRY(check_paging(*paging));
-        total_prefix = static_cast<long long>(paging->num_pages) * paging->page_size;
-        prefix_box = paging->page_size < focus::kTileKeys ? paging->page_size : focus::kTileKeys;
-        cu_prefix = paging->prefix_len;  // only checked for presence below; lengths come from here
+    in->cu_prefix = x.cu_prefix;
+    in->total_prefix = x.total_prefix;
+    in->prefix_box = focus::kTileKeys;
+    in->pg = Paging{x.page_table, x.prefix_len, x.max_pages, x.num_pages, x.page_size};
+    in->paged = x.page_table != nullptr;
+    if (in->paged) {  // the page pools stand in for the packed prefix buffers
+        FOCUS_TRY(check_paging(in->pg));
+        in->total_prefix = static_cast<long long>(in->pg.num_pages) * in->pg.page_size;
+        in->prefix_box = in->pg.page_size < focus::kTileKeys ? in->pg.page_size : focus::kTileKeys;
+        in->cu_prefix = in->pg.prefix_len;  // only checked for presence below; lengths come from here
     }
     if (x.lse0) {
         if (layer1_only) return FOCUS_ERR_INVALID_ARGUMENT;
         FOCUS_TRY(check_ptr(x.lse0, 4));
-        FOCUS_TRY(check_attn_inputs(d, x.q0, nullptr, cu_prefix, 0, x.k0_block));
+        FOCUS_TRY(check_attn_inputs(d, x.q0, nullptr, in->cu_prefix, 0, x.k0_block));
     } else if (!layer1_only) {
-        FOCUS_TRY(check_attn_inputs(d, x.q0, x.k0_prefix, cu_prefix, total_prefix, x.k0_block));
+        FOCUS_TRY(check_attn_inputs(d, x.q0, x.k0_prefix, in->cu_prefix, in->total_prefix,
+                                    x.k0_block));
     }
-    FOCUS_TRY(check_attn_inputs(d, x.q1, x.k1_prefix, cu_prefix, total_prefix, x.k1_block));
+    FOCUS_TRY(check_attn_inputs(d, x.q1, x.k1_prefix, in->cu_prefix, in->total_prefix, x.k1_block));
     FOCUS_TRY(check_ptr(x.hidden, 16));
     FOCUS_TRY(check_ptr(x.decoded, 1));
     if (dynamic) {
@@ -608,7 +642,20 @@ focus_status_t evict_impl(const focus_dims_t *dims, const focus_evict_args_t &x)
     if (x.i0_out) FOCUS_TRY(check_ptr(x.i0_out, 4));
     if (x.i1_out) FOCUS_TRY(check_ptr(x.i1_out, 4));
     FOCUS_TRY(check_ws(d, x.workspace, x.workspace_bytes));
-    FOCUS_TRY(get_encoder());
+    return get_encoder();
+}
+
+focus_status_t evict_impl(const focus_dims_t *dims, const focus_evict_args_t &x) {
+    NvtxRange nvtx_range("focus_evict");
+    EvictInputs in;
+    FOCUS_TRY(check_evict(dims, x, &in));
+    const focus_dims_t &d = *dims;
+    const bool layer1_only = d.score == FOCUS_SCORE_LAYER1;
+    const bool dynamic = x.decode_avg != nullptr;
+    const int32_t *cu_prefix = in.cu_prefix;
+    const long long total_prefix = in.total_prefix;
+    const int prefix_box = in.prefix_box;
+    const Paging *paging = in.paged ? &in.pg : nullptr;
     cudaStream_t s = static_cast<cudaStream_t>(x.stream);
     uint8_t *ws = static_cast<uint8_t *>(x.workspace);
 
@@ -752,6 +799,16 @@ focus_status_t evict_from_sums(const focus_dims_t *dims, const float *sums, int 
 }
 
 }  // namespace
+
+namespace focus {
+
+focus_status_t evict_check(const focus_dims_t *dims, const focus_evict_args_t *args) {
+    if (!args) return FOCUS_ERR_INVALID_ARGUMENT;
+    EvictInputs in;
+    return check_evict(dims, *args, &in);
+}
+
+}  // namespace focus
 
 extern "C" {
 

@@ -14,9 +14,17 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <string.h>
+
 #include <mutex>
 
 #include "focus.h"
+
+namespace focus {
+// The fused step's host validation (focus_api.cu): every check focus_evict_ex makes
+// before it enqueues work, with nothing enqueued.
+focus_status_t evict_check(const focus_dims_t *dims, const focus_evict_args_t *args);
+}  // namespace focus
 
 namespace {
 
@@ -28,7 +36,10 @@ constexpr int kMaxDevices = 256;
 std::mutex g_mu;
 void *g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of g_scratch on the current device, looked up once per device.
+// Device address of g_scratch on the current device, looked up once per device and
+// kept for the life of the process.  A cudaDeviceReset (or anything else that tears
+// down and rebuilds the device's primary context) reloads the module and may move the
+// array, so the library must not be used on a device across such a reset.
 focus_status_t scratch_address(void **out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
@@ -63,13 +74,38 @@ extern "C" focus_status_t focus_evict_static_scratch(
     void *scratch = nullptr;
     focus_status_t st = scratch_address(&scratch);
     if (st != FOCUS_OK) return st;
+    focus_evict_args_t x;
+    memset(&x, 0, sizeof x);
+    x.q0 = q0;
+    x.k0_prefix = k0_prefix;
+    x.k0_block = k0_block;
+    x.q1 = q1;
+    x.k1_prefix = k1_prefix;
+    x.k1_block = k1_block;
+    x.cu_prefix = cu_prefix;
+    x.total_prefix = total_prefix;
+    x.hidden = hidden;
+    x.decoded = decoded;
+    x.budget = budget;
+    x.kept_idx = kept_idx;
+    x.cu_seqlens = cu_seqlens;
+    x.packed = packed;
+    x.capacity = capacity;
+    x.delta_out = delta_out;
+    x.i0_out = i0_out;
+    x.i1_out = i1_out;
+    x.workspace = scratch;
+    x.workspace_bytes = FOCUS_STATIC_SCRATCH_BYTES;
+    x.stream = stream;
+    // Every argument is checked before anything is enqueued: a call that is refused
+    // leaves the array, and the status word another call may still report, untouched.
+    st = focus::evict_check(dims, &x);
+    if (st != FOCUS_OK) return st;
     // The array keeps the previous call's contents; only the status word must
     // start at zero (everything else is fully rewritten before it is read).
     st = focus_clear_device_status(scratch, FOCUS_STATIC_SCRATCH_BYTES, stream);
     if (st != FOCUS_OK) return st;
-    st = focus_evict(dims, q0, k0_prefix, k0_block, q1, k1_prefix, k1_block, cu_prefix,
-                     total_prefix, hidden, decoded, budget, kept_idx, cu_seqlens, packed, capacity,
-                     delta_out, i0_out, i1_out, scratch, FOCUS_STATIC_SCRATCH_BYTES, stream);
+    st = focus_evict_ex(dims, &x);
     if (st != FOCUS_OK) return st;
     if (device_status &&
         cudaMemcpyAsync(device_status, scratch, sizeof(uint32_t), cudaMemcpyDeviceToDevice,

@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define FOCUS_ABI_VERSION 4
+#define FOCUS_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define FOCUS_API __attribute__((visibility("default")))
@@ -118,6 +118,28 @@ typedef struct {
 
 /* Bytes of workspace every entry point below needs for `dims` (256-byte aligned). */
 FOCUS_API size_t focus_workspace_size(const focus_dims_t *dims);
+
+/*
+ * Rows of the packed batch (the `capacity` to allocate), computed on the host from
+ * HOST copies of the scheduler's own arrays; nothing touches the GPU.
+ * "What carries the argument" (pith.science review page): each block keeps its
+ * top-K still-masked tokens under its budget, so request r keeps
+ *   k_r = min(max(budget_host[r], 0), masked_r),  masked_r = #{j : decoded_host[r*B + j] == 0}
+ * rows, and without structural constraints (dims->constraints == 0) the batch has
+ * exactly sum_r k_r rows -- the value cu_seqlens[R] will hold.  With `dynamic`
+ * (the budget is computed on the device from the delta, focus_evict_ex with
+ * decode_avg) k_r is bounded by masked_r and budget_host is not read (may be
+ * NULL).  With constraints the retained count depends on the attention data and
+ * the result is the upper bound sum over requests with k_r > 0 of
+ * min(B, masked_r + k_r) (candidates, their predecessors, the other masked tokens).
+ *   decoded_host [R, B] uint8 (host), budget_host [R] int32 (host), *capacity_out
+ *   (host) receives the row count.
+ * Returns FOCUS_ERR_INVALID_ARGUMENT for a null pointer (budget_host only when
+ * dynamic is 0) and the check_dims errors of the other entry points for bad dims.
+ */
+FOCUS_API focus_status_t focus_plan_capacity(const focus_dims_t *dims, const uint8_t *decoded_host,
+                                             const int32_t *budget_host, int dynamic,
+                                             int64_t *capacity_out);
 
 /* Zero the workspace's status region (enqueued on `stream`): the device status
  * word and the peer exchange's block counter.  Call once before the first use of
@@ -439,10 +461,21 @@ FOCUS_API focus_status_t focus_selftest_exchange(const float *partials, void *co
  *    on `stream` after the kernels.
  *  - Returns FOCUS_ERR_WORKSPACE when focus_workspace_size(dims) exceeds
  *    FOCUS_STATIC_SCRATCH_BYTES (shapes that large need focus_evict), otherwise
- *    the same codes as focus_evict.
+ *    the same codes as focus_evict.  The largest batch is set by the workspace
+ *    formula: 256 B + the request order (4 R) + the column sums (8 R Hkv MT B,
+ *    MT = ceil(Hq B / (128 Hkv))) + the retained lists (4 R B) + the counts (4 R),
+ *    each rounded up to 256 B, plus the split-prefix regions of batches with at
+ *    most 148 attention item groups: 3,840 requests at Hq 32 / Hkv 8 / B 32,
+ *    251 at B 128, 991 at Hkv 4 / B 64.
+ *  - Every argument is checked before anything is enqueued, so a refused call
+ *    leaves the array (and a status word another call is about to report)
+ *    untouched.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current; `stream` must belong to
- *    the current device).  Make that first call before any stream capture.
+ *    the current device) and keeps it for the life of the process.  Make that
+ *    first call before any stream capture.  A cudaDeviceReset (or anything else
+ *    that destroys and recreates the device's primary context) may move the
+ *    array: do not use this entry point on a device after such a reset.
  *  - All calls on a device share the one array and it keeps the last call's
  *    contents: each call clears the status word and rewrites the rest before
  *    reading it.  Calls whose kernels overlap on the GPU (different streams, or

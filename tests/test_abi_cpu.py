@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol():
 def test_status_strings_and_version():
     for code, name in F.STATUS.items():
         assert F.focus_status_string(code) == name
-    assert F.focus_abi_version() == 4
+    assert F.focus_abi_version() == 5
 
 
 def dims(**kw):
@@ -367,3 +367,47 @@ def test_binding_rejects_bad_tensors_before_the_library():
                                         torch.zeros(3, dtype=torch.int64), 0, 2, 1, None)
     with pytest.raises(F.FocusError):
         F.focus_exchange_buffer_size(d, 9)
+
+
+def test_plan_capacity_equals_the_oracle_row_count(orc):
+    """focus_plan_capacity (host arithmetic behind the C ABI): without constraints it
+    equals the oracle's cu_seqlens[R] for any delta; with constraints it bounds the
+    oracle's retained count; with a dynamic budget it bounds every budget the oracle
+    can choose.  Budgets include negative, zero and over-large values."""
+    import synth
+    rng = np.random.default_rng(11)
+    for cfg, R in ((1, 40), (3, 9), (4, 70)):
+        p = synth.make_problem(cfg, seed=40 + cfg, overrides=dict(R=R, prefix=("fixed", 0)))
+        dec = p.decoded.numpy()
+        bud = rng.integers(-3, p.B + 5, size=p.R).astype(np.int32)
+        pooled = np.where(dec != 0, -np.inf, rng.normal(size=dec.shape))
+        _, cu, _ = orc.select(pooled, dec, bud)
+        d0 = dims(R=p.R, B=p.B)
+        assert F.focus_plan_capacity(d0, p.decoded, torch.from_numpy(bud)) == int(cu[-1])
+        assert F.plan_capacity(p.decoded, torch.from_numpy(bud)) == int(cu[-1])
+        for c in (1, 2, 3):
+            _, cu_s, _ = orc.select_structured(pooled, dec, bud, c)
+            cap = F.focus_plan_capacity(dims(R=p.R, B=p.B, constraints=c), p.decoded,
+                                        torch.from_numpy(bud))
+            assert cap >= int(cu_s[-1])
+        avg = rng.uniform(0, 40, size=p.R)
+        k_dyn = orc.dynamic_budget(pooled, dec, avg)
+        _, cu_d, _ = orc.select(pooled, dec, k_dyn)
+        assert F.focus_plan_capacity(d0, p.decoded, None, dynamic=True) >= int(cu_d[-1])
+        assert F.focus_plan_capacity(d0, p.decoded, None, dynamic=True) == int((dec == 0).sum())
+
+
+def test_plan_capacity_rejects_bad_arguments():
+    d0 = dims(R=2, B=8)
+    out = ctypes.c_int64(-1)
+    dec = np.zeros((2, 8), np.uint8)
+    bud = np.ones(2, np.int32)
+    P = lambda a: ctypes.c_void_p(a.ctypes.data)
+    assert F._lib.focus_plan_capacity(ctypes.byref(d0), None, P(bud), 0, ctypes.byref(out)) == INVALID
+    assert F._lib.focus_plan_capacity(ctypes.byref(d0), P(dec), None, 0, ctypes.byref(out)) == INVALID
+    assert F._lib.focus_plan_capacity(ctypes.byref(d0), P(dec), None, 1, ctypes.byref(out)) == OK
+    assert out.value == 16
+    assert F._lib.focus_plan_capacity(ctypes.byref(d0), P(dec), P(bud), 0, None) == INVALID
+    bad = dims(R=2, B=200)
+    assert F._lib.focus_plan_capacity(ctypes.byref(bad), P(dec), P(bud), 0,
+                                      ctypes.byref(out)) == UNSUPPORTED
