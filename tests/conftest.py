@@ -26,3 +26,20 @@ def pytest_configure(config):
 def orc():
     import oracle
     return oracle.default()
+
+
+# Per-config selection reports of the parity tests (how many kept sets were
+# checked exactly, how many fell in the tie band), printed after the run.
+PARITY_REPORT = []
+
+
+@pytest.fixture(scope="session")
+def parity_report():
+    return PARITY_REPORT
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    if PARITY_REPORT:
+        terminalreporter.section("selection parity (kept sets checked against the oracle)")
+        for line in PARITY_REPORT:
+            terminalreporter.write_line(line)

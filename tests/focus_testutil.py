@@ -10,6 +10,8 @@ Tolerances (bf16 inputs, fp32 accumulation on the GPU, float64 in the oracle):
 """
 from __future__ import annotations
 
+import math
+
 import numpy as np
 import torch
 
@@ -95,31 +97,126 @@ def check_selection(kept_gpu, cu_gpu, pooled_oracle, decoded, budget, requests=N
     return exact, len(list(reqs)), tie_only
 
 
-def check_structured(kept_gpu, cu_gpu, kept_oracle, cu_oracle, pooled_oracle, decoded, budget,
-                     requests=None):
-    """Retained sets under structural constraints.  A request whose candidate set is
-    decided by a margin (oracle k-th and (k+1)-th pooled values more than 2e-3 apart)
-    must match the oracle exactly; requests inside the tie band only need a valid,
-    ascending, unique set.  Returns (n_exact, n_checked)."""
-    pooled_oracle = np.asarray(pooled_oracle, np.float64)
+def selection_margin(raw_row, pooled_row, decoded_row, k) -> float:
+    """How far the oracle's selection of one request is from a different answer.
+
+    The k-th largest masked pooled value v_k is the cut.  Pooled values are window
+    maxima of the raw delta, so equal values at neighbouring positions are copies of
+    one raw value (and duplicated keys give equal raw values); such exact ties are
+    broken by position identically on both sides.  What can move the cut is another
+    raw value close to v_k, pooled or hidden inside a window, so the margin is the
+    distance from v_k to the nearest raw delta of the block that differs from it;
+    infinite when k is 0 or every masked position is kept.
+    """
+    masked = np.flatnonzero(np.asarray(decoded_row) == 0)
+    if k == 0 or k >= masked.size:
+        return float("inf")
+    vk = np.sort(np.asarray(pooled_row, np.float64)[masked])[::-1][k - 1]
+    raw = np.asarray(raw_row, np.float64)
+    other = raw[raw != vk]
+    return float(np.min(np.abs(other - vk))) if other.size else float("inf")
+
+
+def selection_margins(ref, decoded, budget) -> np.ndarray:
+    """selection_margin of every request of an oracle result (budget clamped as the
+    method clamps it)."""
+    decoded = np.asarray(decoded)
+    budget = np.asarray(budget)
+    out = np.empty(decoded.shape[0])
+    for r in range(decoded.shape[0]):
+        k = min(max(int(budget[r]), 0), int((decoded[r] == 0).sum()))
+        out[r] = selection_margin(ref["delta"][r], ref["pooled"][r], decoded[r], k)
+    return out
+
+
+def check_selection_all(kept_gpu, cu_gpu, ref, decoded, budget, orc):
+    """Every request's kept set against the oracle's selection from its pooled delta
+    (`ref["pooled"]`, raw delta `ref["delta"]`) under `budget`.  Requests decided by a
+    margin (selection_margin > TIE_TOL) must match exactly; the others must satisfy
+    the tie rule of check_selection.  Returns a report dict."""
+    decoded = np.asarray(decoded)
+    budget = np.asarray(budget)
+    want, want_cu, _ = orc.select(ref["pooled"], decoded, budget)
+    margins = selection_margins(ref, decoded, budget)
+    exact, n, tie_only = check_selection(kept_gpu, cu_gpu, ref["pooled"], decoded, budget)
+    decided = margins > TIE_TOL
+    for r in np.flatnonzero(decided):
+        np.testing.assert_array_equal(kept_gpu[cu_gpu[r]:cu_gpu[r + 1]],
+                                      want[want_cu[r]:want_cu[r + 1]],
+                                      err_msg=f"request {r} (margin {margins[r]:.3g})")
+    return dict(requests=n, exact=exact, tie_band=int((~decided).sum()),
+                exact_in_tie_band=int(exact - decided.sum()), decided=int(decided.sum()),
+                min_margin=float(margins.min()) if n else float("inf"))
+
+
+def check_structured(kept_gpu, cu_gpu, cand_gpu, cand_cu_gpu, ref, decoded, budget, constraints,
+                     orc):
+    """Retained sets under structural constraints, every request.
+
+    cand_gpu / cand_cu_gpu are the GPU's plain top-k candidates on the same inputs
+    (a constraints = 0 call: the same delta, so the same candidates); they must pass
+    check_selection_all against the oracle's plain selection under `budget`.  The
+    retained list must then be the constraint closure of those candidates
+    (predecessors, masked positions left of the rightmost one), which the oracle's
+    own structured selection computes from a 0/1 indicator of the candidates.
+    Requests decided by a margin must also equal the oracle's retained list under
+    `budget`.  Returns the candidates' report with the structured exact count added.
+    """
     decoded = np.asarray(decoded)
     budget = np.asarray(budget)
     R, B = decoded.shape
-    reqs = range(R) if requests is None else requests
+    rep = check_selection_all(cand_gpu, cand_cu_gpu, ref, decoded, budget, orc)
+    ind = np.where(decoded != 0, -np.inf, 0.0)
+    counts = np.zeros(R, np.int32)
+    for r in range(R):
+        c = cand_gpu[cand_cu_gpu[r]:cand_cu_gpu[r + 1]]
+        ind[r, c] = 1.0
+        counts[r] = c.size
+    closure, closure_cu, _ = orc.select_structured(ind, decoded, counts, constraints)
+    np.testing.assert_array_equal(cu_gpu, closure_cu, err_msg="cu_seqlens vs the candidates' closure")
+    want, want_cu, _ = orc.select_structured(ref["pooled"], decoded, budget, constraints)
+    margins = selection_margins(ref, decoded, budget)
     exact = 0
-    for i, r in enumerate(reqs):
+    for r in range(R):
         got = kept_gpu[cu_gpu[r]:cu_gpu[r + 1]]
-        assert (np.diff(got) > 0).all() and ((got >= 0) & (got < B)).all(), (r, got)
-        orow = pooled_oracle[i]
-        masked = np.flatnonzero(decoded[r] == 0)
-        k = min(max(int(budget[r]), 0), masked.size)
-        vals = np.sort(orow[masked])[::-1]
-        decided = k == 0 or k == masked.size or vals[k - 1] - vals[k] > TIE_TOL
-        if decided:
-            want = kept_oracle[cu_oracle[i]:cu_oracle[i + 1]]
-            np.testing.assert_array_equal(got, want, err_msg=f"retained set of request {r}")
-            exact += 1
-    return exact, len(list(reqs))
+        np.testing.assert_array_equal(got, closure[closure_cu[r]:closure_cu[r + 1]],
+                                      err_msg=f"request {r}: not the closure of its candidates")
+        oref = want[want_cu[r]:want_cu[r + 1]]
+        if margins[r] > TIE_TOL:
+            np.testing.assert_array_equal(got, oref, err_msg=f"retained set of request {r}")
+        exact += int(np.array_equal(got, oref))
+    rep["structured_exact"] = exact
+    return rep
+
+
+def check_dynamic_budget(k_gpu, pooled, decoded, decode_avg, alpha=1.5, band=1e-2):
+    """The GPU's dynamic budgets against the oracle's reading of Eq. 4,
+    K = min(max(ceil(alpha * avg), n, 1), masked) with n the masked positions whose pooled
+    delta exceeds their mean plus one population standard deviation.  n is bounded by
+    the counts above the threshold moved by +-`band` (values that close to it may be
+    counted either way), and ceil(alpha * avg) by its float32 and float64 values; every
+    request's budget must lie within the bounds (equal to the oracle's where they
+    meet).  Returns the number of requests whose bounds meet."""
+    k_gpu = np.asarray(k_gpu)
+    decoded = np.asarray(decoded)
+    avg = np.asarray(decode_avg, np.float32)
+    pinned = 0
+    for r in range(decoded.shape[0]):
+        m = decoded[r] == 0
+        if not m.any():
+            assert k_gpu[r] == 0, (r, k_gpu[r])
+            pinned += 1
+            continue
+        D = np.asarray(pooled[r], np.float64)[m]
+        thr = D.mean() + D.std()
+        n_lo, n_hi = int((D > thr + band).sum()), int((D > thr - band).sum())
+        a = max(float(avg[r]), 0.0)
+        bases = (math.ceil(alpha * a), math.ceil(float(np.float32(alpha) * np.float32(a))))
+        lo = min(max(min(bases), n_lo, 1), int(m.sum()))
+        hi = min(max(max(bases), n_hi, 1), int(m.sum()))
+        assert lo <= k_gpu[r] <= hi, (r, int(k_gpu[r]), lo, hi)
+        pinned += int(lo == hi)
+    return pinned
 
 
 def check_packed(packed, kept, cu, hidden_bits, requests=None):

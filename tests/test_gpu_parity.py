@@ -3,8 +3,7 @@
 Small cases are compared element by element; they span several 128-key tiles,
 ragged tails, several 128-row query tiles, both head dims, GQA group sizes
 1..16, odd block sizes and empty prefixes.  The five full-size workloads run in
-the launch configuration the benchmark times and are compared on sampled
-requests, which the oracle computes one by one.
+the launch configuration the benchmark times and are compared on every request.
 """
 import os
 
@@ -13,8 +12,9 @@ import pytest
 import torch
 
 import synth
-from focus_testutil import (assert_close_delta, assert_close_importance, check_packed,
-                            check_selection, check_structured, hidden_bits, run_evict)
+from focus_testutil import (assert_close_delta, assert_close_importance, check_dynamic_budget,
+                            check_packed, check_selection, check_selection_all, check_structured,
+                            hidden_bits, run_evict)
 
 pytestmark = pytest.mark.gpu
 
@@ -43,14 +43,14 @@ def orc():
     return oracle.default()
 
 
-def _compare_full(p, out, ref):
+def _compare_full(p, out, ref, orc):
     assert out["status"] == 0, out["status"]
     assert_close_importance(out["i0"], ref["i0"], "I0")
     assert_close_importance(out["i1"], ref["i1"], "I1")
     assert_close_delta(out["delta"], ref["pooled"])
     np.testing.assert_array_equal(out["cu_seqlens"], ref["cu_seqlens"])
-    check_selection(out["kept"], out["cu_seqlens"], ref["pooled"], p.decoded.cpu().numpy(),
-                    p.budget.cpu().numpy())
+    check_selection_all(out["kept"], out["cu_seqlens"], ref, p.decoded.cpu().numpy(),
+                        p.budget.cpu().numpy(), orc)
     check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))
 
 
@@ -61,41 +61,40 @@ def test_small_elementwise(case, orc):
                            overrides=ov)
     ref = orc.evict(p)
     out = run_evict(p.to("cuda"))
-    _compare_full(p, out, ref)
+    _compare_full(p, out, ref, orc)
 
 
-def _sample_requests(p, n=6):
-    L = p.prefix_len
-    dec = p.decoded.cpu().numpy()
-    masked = (dec == 0).sum(1)
-    pick = [int(np.argmax(L)), int(np.argmin(L)), int(np.argmax(masked)), int(np.argmin(masked))]
-    pick += [r for (r, _, _) in p.tie_pairs[:2]]
-    rng = np.random.default_rng(0)
-    pick += rng.choice(p.R, size=min(p.R, n), replace=False).tolist()
-    return sorted(set(pick))
+def _report(parity_report, what, rep):
+    line = (f"{what}: exact {rep['exact']}/{rep['requests']} kept sets "
+            f"(decided by a margin > 2e-3: {rep['decided']}, all exact; tie band: "
+            f"{rep['tie_band']}, of which exact {rep['exact_in_tie_band']}); "
+            f"smallest margin {rep['min_margin']:.2e}")
+    if "structured_exact" in rep:
+        line += f"; retained lists equal to the oracle's: {rep['structured_exact']}"
+    parity_report.append(line)
 
 
+@pytest.mark.parametrize("wide", [False, True], ids=["literal", "wide"])
 @pytest.mark.parametrize("cfg", [0, 1, 2, 3, 4])
-def test_full_config_sampled(cfg, orc):
-    """The benchmark's launch configuration on the full workload; the oracle checks a
-    sample of requests one by one, and cu_seqlens in full."""
-    p = synth.make_problem(cfg)
+def test_full_config_every_request(cfg, wide, orc, parity_report):
+    """The five workloads at full size, in the benchmark's launch configuration, against
+    the oracle on every request: I0, I1 and the pooled delta element by element,
+    cu_seqlens and packed rows exactly, and every kept set -- exactly where the oracle's
+    selection is decided by a margin, else under the tie rule.  Run with the workloads'
+    own value scale and with wide logits (Q, K ~ N(0, 1)), where margins are larger."""
+    p = synth.make_problem(cfg, wide_logits=wide)
     out = run_evict(p.to("cuda"))
-    assert out["status"] == 0
-    req = _sample_requests(p)
-    sub = p.subset(req)
-    ref = orc.evict(sub)
-    assert_close_importance(out["i0"][req], ref["i0"], "I0")
-    assert_close_importance(out["i1"][req], ref["i1"], "I1")
-    assert_close_delta(out["delta"][req], ref["pooled"])
-    # cu_seqlens in full: the kept counts do not depend on the attention data
-    _, cu_all, _ = orc.select(np.zeros((p.R, p.B)), p.decoded, p.budget)
-    np.testing.assert_array_equal(out["cu_seqlens"], cu_all)
-    check_selection(out["kept"], out["cu_seqlens"], ref["pooled"], p.decoded.cpu().numpy(),
-                    p.budget.cpu().numpy(), requests=req)
+    ref = orc.evict(p)
+    assert out["status"] == 0, out["status"]
+    assert_close_importance(out["i0"], ref["i0"], "I0")
+    assert_close_importance(out["i1"], ref["i1"], "I1")
+    assert_close_delta(out["delta"], ref["pooled"])
+    np.testing.assert_array_equal(out["cu_seqlens"], ref["cu_seqlens"])
+    rep = check_selection_all(out["kept"], out["cu_seqlens"], ref, p.decoded.numpy(),
+                              p.budget.numpy(), orc)
     check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))
-    # every request: valid selection shape
-    assert np.isfinite(out["i0"]).all() and np.isfinite(out["i1"]).all()
+    _report(parity_report, f"{synth.CONFIGS[cfg].name} ({'wide' if wide else 'literal'} logits)",
+            rep)
 
 
 def test_duplicate_keys_give_equal_columns():
@@ -195,7 +194,7 @@ def test_zero_budget_and_all_decoded(orc):
     p.decoded = dec
     ref = orc.evict(p)
     out = run_evict(p.to("cuda"))
-    _compare_full(p, out, ref)
+    _compare_full(p, out, ref, orc)
     assert out["cu_seqlens"][1] == 0 and out["cu_seqlens"][2] == 0
 
 
@@ -248,19 +247,22 @@ STRUCTURED_CASES = {
 @pytest.mark.parametrize("case", sorted(STRUCTURED_CASES))
 def test_structural_constraints_vs_oracle(case, constraints, orc):
     """Retained sets with the structural constraints ("What carries the argument"):
-    candidates plus predecessors and/or masked tokens left of the rightmost one."""
-    from focus_testutil import check_structured
+    candidates plus predecessors and/or masked tokens left of the rightmost one.  Every
+    request's list is the closure of the GPU's own top-k candidates (checked against the
+    oracle's selection), and equals the oracle's list where a margin decides it."""
     cfg, ov, wide = STRUCTURED_CASES[case]
     p = synth.make_problem(cfg, seed=300 + constraints, wide_logits=wide, overrides=ov)
     ref = orc.evict(p, constraints=constraints)
-    out = run_evict(p.to("cuda"), constraints=constraints)
-    assert out["status"] == 0, out["status"]
+    g = p.to("cuda")
+    out = run_evict(g, constraints=constraints)
+    cand = run_evict(g)
+    assert out["status"] == 0 and cand["status"] == 0
+    np.testing.assert_array_equal(out["delta"], cand["delta"])  # same delta, same candidates
     assert_close_importance(out["i0"], ref["i0"], "I0")
     assert_close_importance(out["i1"], ref["i1"], "I1")
     assert_close_delta(out["delta"], ref["pooled"])
-    exact, n = check_structured(out["kept"], out["cu_seqlens"], ref["kept"], ref["cu_seqlens"],
-                                ref["pooled"], p.decoded.numpy(), p.budget.numpy())
-    assert exact >= n // 2, (exact, n)
+    check_structured(out["kept"], out["cu_seqlens"], cand["kept"], cand["cu_seqlens"], ref,
+                     p.decoded.numpy(), p.budget.numpy(), constraints, orc)
     check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))
 
 
@@ -286,29 +288,24 @@ def test_structural_topk_select_exact(orc):
         np.testing.assert_array_equal(kept[:int(ocu[-1])].cpu().numpy(), okept)
 
 
-def test_structural_full_config_sampled(orc):
-    """Constraints on a full-size workload in the benchmark's launch configuration,
-    checked on sampled requests; cu_seqlens must be consistent with the lists."""
-    from focus_testutil import check_structured
-    p = synth.make_problem(4, wide_logits=True)
-    out = run_evict(p.to("cuda"), constraints=3)
-    assert out["status"] == 0
-    req = _sample_requests(p)
-    ref = orc.evict(p.subset(req), constraints=3)
-    assert_close_delta(out["delta"][req], ref["pooled"])
-    # compare the sampled requests' retained sets
-    got_kept, got_cu = [], [0]
-    for r in req:
-        seg = out["kept"][out["cu_seqlens"][r]:out["cu_seqlens"][r + 1]]
-        got_kept.append(seg)
-        got_cu.append(got_cu[-1] + len(seg))
-    got_kept = np.concatenate(got_kept) if got_kept else np.zeros(0, np.int32)
-    dec = p.decoded.numpy()[req]
-    bud = p.budget.numpy()[req]
-    exact, n = check_structured(got_kept, np.array(got_cu), ref["kept"], ref["cu_seqlens"],
-                                ref["pooled"], dec, bud)
-    assert exact >= n // 2, (exact, n)
+@pytest.mark.parametrize("cfg,wide", [(4, True), (2, False)], ids=["ragged_wide", "metric_literal"])
+def test_structural_full_config_every_request(cfg, wide, orc, parity_report):
+    """Both constraints on a full-size workload in the benchmark's launch configuration:
+    every request's retained list is the closure of the GPU's top-k candidates, which
+    match the oracle's selection (exactly where a margin decides it)."""
+    p = synth.make_problem(cfg, wide_logits=wide)
+    g = p.to("cuda")
+    out = run_evict(g, constraints=3)
+    cand = run_evict(g)
+    assert out["status"] == 0 and cand["status"] == 0
+    np.testing.assert_array_equal(out["delta"], cand["delta"])
+    ref = orc.evict(p)
+    assert_close_delta(out["delta"], ref["pooled"])
+    rep = check_structured(out["kept"], out["cu_seqlens"], cand["kept"], cand["cu_seqlens"], ref,
+                           p.decoded.numpy(), p.budget.numpy(), 3, orc)
     check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))
+    _report(parity_report, f"{synth.CONFIGS[cfg].name} ({'wide' if wide else 'literal'} logits), "
+            "constraints 3", rep)
 
 
 @pytest.mark.parametrize("case", ["sdar_r8_wide", "ragged_r10_ties", "tiny"])
@@ -323,8 +320,8 @@ def test_layer1_score_vs_oracle(case, orc):
     assert np.isnan(out["i0"]).all()  # left untouched
     assert_close_importance(out["i1"], ref["i1"], "I1")
     assert_close_delta(out["delta"], ref["pooled"])
-    check_selection(out["kept"], out["cu_seqlens"], ref["pooled"], p.decoded.numpy(),
-                    p.budget.numpy())
+    check_selection_all(out["kept"], out["cu_seqlens"], ref, p.decoded.numpy(),
+                        p.budget.numpy(), orc)
     check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))
 
 
@@ -372,8 +369,8 @@ def test_evict_with_lse0_vs_oracle(case, orc):
     assert_close_importance(i1.cpu().numpy(), ref["i1"], "I1")
     assert_close_delta(delta.cpu().numpy(), ref["pooled"])
     np.testing.assert_array_equal(cu.cpu().numpy(), ref["cu_seqlens"])
-    check_selection(kept.cpu().numpy(), cu.cpu().numpy(), ref["pooled"], p.decoded.numpy(),
-                    p.budget.numpy())
+    check_selection_all(kept.cpu().numpy(), cu.cpu().numpy(), ref, p.decoded.numpy(),
+                        p.budget.numpy(), orc)
     check_packed(packed.view(torch.int16).cpu().numpy().view(np.uint16), kept.cpu().numpy(),
                  cu.cpu().numpy(), hidden_bits(p))
 
@@ -408,8 +405,8 @@ def test_evict_paged_vs_oracle(page_size, orc):
     assert_close_importance(i1.cpu().numpy(), ref["i1"], "I1")
     assert_close_delta(delta.cpu().numpy(), ref["pooled"])
     np.testing.assert_array_equal(cu.cpu().numpy(), ref["cu_seqlens"])
-    check_selection(kept.cpu().numpy(), cu.cpu().numpy(), ref["pooled"], p.decoded.numpy(),
-                    p.budget.numpy())
+    check_selection_all(kept.cpu().numpy(), cu.cpu().numpy(), ref, p.decoded.numpy(),
+                        p.budget.numpy(), orc)
     check_packed(packed.view(torch.int16).cpu().numpy().view(np.uint16), kept.cpu().numpy(),
                  cu.cpu().numpy(), hidden_bits(p))
 
@@ -440,55 +437,63 @@ def test_evict_paged_matches_packed_bitwise():
         np.testing.assert_array_equal(kept.cpu().numpy(), want["kept"])
 
 
-@pytest.mark.parametrize("case,constraints", [("sdar_r8_wide", 0), ("ragged_r10_ties", 0),
-                                              ("block128_r3", 0), ("sdar_r8_wide", 3)])
-def test_dynamic_budget_vs_oracle(case, constraints, orc):
-    """Dynamic budget (Eq. 4 as read): the GPU's K_r equals the oracle's wherever no
-    masked pooled delta lies within 1e-2 of the mean + std threshold; the selection
-    under the GPU's K_r matches the oracle's under the same K_r."""
+def _evict_dynamic(p, g, avg, constraints, **extra):
+    """focus_evict_ex with the dynamic budget on the GPU problem `g`; returns numpy kept,
+    cu_seqlens, budgets, pooled delta and packed rows.  `extra` passes further options
+    (lse0, page pools) through to the call."""
     import attention_delta_token_b200 as F
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, constraints)
+    ws = F.Workspace(dims)
+    cap = F.plan_capacity(p.decoded, None, constraints, dynamic=True)
+    kept = torch.full((max(cap, 1),), -1, dtype=torch.int32, device="cuda")[:cap]
+    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+    packed = torch.zeros(max(cap, 1), p.H, dtype=torch.bfloat16, device="cuda")[:cap]
+    delta = torch.empty(p.R, p.B, device="cuda")
+    kout = torch.full((p.R,), -1, dtype=torch.int32, device="cuda")
+    args = dict(q0=g.q0, k0_prefix=g.k0_prefix, k0_block=g.k0_block, q1=g.q1,
+                k1_prefix=g.k1_prefix, k1_block=g.k1_block, cu_prefix=g.cu_prefix)
+    args.update(extra)
+    F.focus_evict_ex(dims, **args, hidden=g.hidden, decoded=g.decoded,
+                     decode_avg=torch.from_numpy(np.asarray(avg, np.float32)).cuda(),
+                     budget_alpha=1.5, budget_out=kout, kept_idx=kept, cu_seqlens=cu,
+                     packed=packed, ws=ws, delta_out=delta)
+    status = F.focus_read_device_status(ws)
+    cu_h = cu.cpu().numpy()
+    n = int(cu_h[-1])
+    return dict(status=status, kept=kept[:n].cpu().numpy(), cu_seqlens=cu_h,
+                budget=kout.cpu().numpy(), delta=delta.cpu().numpy().astype(np.float64),
+                packed=packed[:n].view(torch.int16).cpu().numpy().view(np.uint16))
+
+
+@pytest.mark.parametrize("case,constraints", [("sdar_r8_wide", 0), ("ragged_r10_ties", 0),
+                                              ("block128_r3", 0), ("sdar_r8_wide", 3),
+                                              ("ragged_r10_ties", 3)])
+def test_dynamic_budget_vs_oracle(case, constraints, orc):
+    """Dynamic budget (Eq. 4 as read): every request's K_r lies within the oracle's bounds
+    (equal to the oracle's K_r wherever no masked pooled delta lies within 1e-2 of the
+    mean + std threshold); the kept sets under the GPU's own K_r match the oracle's
+    selection under the same K_r (with constraints: the closure of the candidates)."""
     cfg, ov, wide = STRUCTURED_CASES[case]
     p = synth.make_problem(cfg, seed=700, wide_logits=wide, overrides=ov)
     rng = np.random.default_rng(7)
     avg = rng.uniform(0.0, 4.0, size=p.R).astype(np.float32)
-    ref = orc.evict(p, constraints=constraints, decode_avg=avg.astype(np.float64))
+    ref = orc.evict(p, decode_avg=avg.astype(np.float64))
     g = p.to("cuda")
-    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, constraints)
-    ws = F.Workspace(dims)
-    cap = F.plan_capacity(p.decoded, None, constraints, dynamic=True)
-    kept = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
-    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
-    packed = torch.zeros(cap, p.H, dtype=torch.bfloat16, device="cuda")
-    delta = torch.empty(p.R, p.B, device="cuda")
-    kout = torch.full((p.R,), -1, dtype=torch.int32, device="cuda")
-    F.focus_evict_ex(dims, q0=g.q0, k0_prefix=g.k0_prefix, k0_block=g.k0_block, q1=g.q1,
-                     k1_prefix=g.k1_prefix, k1_block=g.k1_block, cu_prefix=g.cu_prefix,
-                     hidden=g.hidden, decoded=g.decoded, decode_avg=torch.from_numpy(avg).cuda(),
-                     budget_alpha=1.5, budget_out=kout, kept_idx=kept, cu_seqlens=cu,
-                     packed=packed, ws=ws, delta_out=delta)
-    assert F.focus_read_device_status(ws) == 0
-    assert_close_delta(delta.cpu().numpy(), ref["pooled"])
-    kg = kout.cpu().numpy()
+    out = _evict_dynamic(p, g, avg, constraints)
+    assert out["status"] == 0
+    assert_close_delta(out["delta"], ref["pooled"])
     dec = p.decoded.numpy()
-    checked = 0
-    for r in range(p.R):
-        m = dec[r] == 0
-        assert (kg[r] == 0) if not m.any() else (1 <= kg[r] <= m.sum())
-        D = ref["pooled"][r][m]
-        if D.size == 0:
-            continue
-        thr = D.mean() + D.std()
-        if np.all(np.abs(D - thr) > 1e-2):
-            assert kg[r] == ref["budget"][r], (r, kg[r], ref["budget"][r])
-            checked += 1
-    assert checked >= p.R // 2, checked
-    # selection under the GPU's own budgets
-    cu_h = cu.cpu().numpy()
-    kept_h = kept[:int(cu_h[-1])].cpu().numpy()
+    kg = out["budget"]
+    check_dynamic_budget(kg, ref["pooled"], dec, avg)
     if constraints == 0:
-        check_selection(kept_h, cu_h, ref["pooled"], dec, kg)
-    check_packed(packed[:int(cu_h[-1])].view(torch.int16).cpu().numpy().view(np.uint16), kept_h,
-                 cu_h, hidden_bits(p))
+        check_selection_all(out["kept"], out["cu_seqlens"], ref, dec, kg, orc)
+    else:
+        cand = _evict_dynamic(p, g, avg, 0)
+        np.testing.assert_array_equal(cand["delta"], out["delta"])
+        np.testing.assert_array_equal(cand["budget"], kg)
+        check_structured(out["kept"], out["cu_seqlens"], cand["kept"], cand["cu_seqlens"], ref,
+                         dec, kg, constraints, orc)
+    check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))
 
 
 def test_head_sharded_two_way_matches_fused(orc):
@@ -524,8 +529,8 @@ def test_head_sharded_two_way_matches_fused(orc):
     assert_close_importance(total[1].cpu().numpy(), fused["i1"], "I1 sharded vs fused")
     ref = orc.evict(p)
     assert_close_delta(delta.cpu().numpy(), ref["pooled"])
-    check_selection(kept.cpu().numpy(), cu.cpu().numpy(), ref["pooled"], p.decoded.numpy(),
-                    p.budget.numpy())
+    check_selection_all(kept.cpu().numpy(), cu.cpu().numpy(), ref, p.decoded.numpy(),
+                        p.budget.numpy(), orc)
     check_packed(packed.view(torch.int16).cpu().numpy().view(np.uint16), kept.cpu().numpy(),
                  cu.cpu().numpy(), hidden_bits(p))
 
@@ -593,17 +598,15 @@ def test_edge_shapes_vs_oracle(case, orc):
     cfg, ov = EDGE_CASES[case]
     p = synth.make_problem(cfg, seed=900 + sorted(EDGE_CASES).index(case), wide_logits=True,
                            overrides=ov)
-    req = list(range(p.R)) if p.R <= 64 else _sample_requests(p, n=40)
-    ref = orc.evict(p.subset(req))
+    ref = orc.evict(p)
     out = run_evict(p.to("cuda"))
     assert out["status"] == 0
-    assert_close_importance(out["i0"][req], ref["i0"], "I0")
-    assert_close_importance(out["i1"][req], ref["i1"], "I1")
-    assert_close_delta(out["delta"][req], ref["pooled"])
-    _, cu_all, _ = orc.select(np.zeros((p.R, p.B)), p.decoded, p.budget)
-    np.testing.assert_array_equal(out["cu_seqlens"], cu_all)
-    check_selection(out["kept"], out["cu_seqlens"], ref["pooled"], p.decoded.numpy(),
-                    p.budget.numpy(), requests=req)
+    assert_close_importance(out["i0"], ref["i0"], "I0")
+    assert_close_importance(out["i1"], ref["i1"], "I1")
+    assert_close_delta(out["delta"], ref["pooled"])
+    np.testing.assert_array_equal(out["cu_seqlens"], ref["cu_seqlens"])
+    check_selection_all(out["kept"], out["cu_seqlens"], ref, p.decoded.numpy(),
+                        p.budget.numpy(), orc)
     check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))
 
 
@@ -745,7 +748,6 @@ def test_dynamic_budget_degenerate_blocks(constraints, orc):
     single masked token is kept (K = 1, its sigma is 0), a fully masked block with a huge
     historical yield is capped at the masked count, a zero yield still keeps one token; the
     budgets, kept sets and packed rows equal the oracle's."""
-    import attention_delta_token_b200 as F
     p = synth.make_problem(1, seed=850, wide_logits=True, overrides=dict(R=4))
     dec = p.decoded.numpy()
     dec[0] = 1
@@ -753,38 +755,26 @@ def test_dynamic_budget_degenerate_blocks(constraints, orc):
     dec[1, 7] = 0
     dec[2] = 0
     avg = np.array([3.0, 2.0, 1000.0, 0.0], np.float32)
-    ref = orc.evict(p, constraints=constraints, decode_avg=avg.astype(np.float64))
+    ref = orc.evict(p, decode_avg=avg.astype(np.float64))
     np.testing.assert_array_equal(ref["budget"][:3], [0, 1, p.B])
     g = p.to("cuda")
-    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, constraints)
-    ws = F.Workspace(dims)
-    cap = F.plan_capacity(p.decoded, None, constraints, dynamic=True)
-    kept = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
-    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
-    packed = torch.zeros(cap, p.H, dtype=torch.bfloat16, device="cuda")
-    kout = torch.full((p.R,), -1, dtype=torch.int32, device="cuda")
-    F.focus_evict_ex(dims, q0=g.q0, k0_prefix=g.k0_prefix, k0_block=g.k0_block, q1=g.q1,
-                     k1_prefix=g.k1_prefix, k1_block=g.k1_block, cu_prefix=g.cu_prefix,
-                     hidden=g.hidden, decoded=g.decoded, decode_avg=torch.from_numpy(avg).cuda(),
-                     budget_alpha=1.5, budget_out=kout, kept_idx=kept, cu_seqlens=cu,
-                     packed=packed, ws=ws)
-    assert F.focus_read_device_status(ws) == 0
-    np.testing.assert_array_equal(kout.cpu().numpy()[:3], ref["budget"][:3])
-    cu_h = cu.cpu().numpy()
+    out = _evict_dynamic(p, g, avg, constraints)
+    assert out["status"] == 0
+    kg = out["budget"]
+    np.testing.assert_array_equal(kg[:3], ref["budget"][:3])
+    check_dynamic_budget(kg, ref["pooled"], dec, avg)
+    cu_h = out["cu_seqlens"]
     assert cu_h[1] == 0                       # the fully decoded block keeps nothing
-    assert list(kept[cu_h[1]:cu_h[2]].cpu().numpy()) == (
+    assert list(out["kept"][cu_h[1]:cu_h[2]]) == (
         [6, 7] if constraints & 1 else [7])   # the lone masked token (and its predecessor)
     assert cu_h[3] - cu_h[2] == p.B           # the fully masked block is kept whole
-    n = int(cu_h[-1])
-    check_packed(packed[:n].view(torch.int16).cpu().numpy().view(np.uint16),
-                 kept[:n].cpu().numpy(), cu_h, hidden_bits(p))
-    kg = kout.cpu().numpy()
-    if kg[3] == ref["budget"][3]:  # request 3's budget is decided by a margin in the oracle
-        if constraints:
-            check_structured(kept[:n].cpu().numpy(), cu_h, ref["kept"], ref["cu_seqlens"],
-                             ref["pooled"], dec, kg)
-        else:
-            check_selection(kept[:n].cpu().numpy(), cu_h, ref["pooled"], dec, kg)
+    check_packed(out["packed"], out["kept"], cu_h, hidden_bits(p))
+    if constraints:
+        cand = _evict_dynamic(p, g, avg, 0)
+        check_structured(out["kept"], cu_h, cand["kept"], cand["cu_seqlens"], ref, dec, kg,
+                         constraints, orc)
+    else:
+        check_selection_all(out["kept"], cu_h, ref, dec, kg, orc)
 
 
 @pytest.mark.parametrize("window", [1, 5, 7])
@@ -797,7 +787,7 @@ def test_other_pool_windows_vs_oracle(window, orc):
     assert p.pool_window == window
     ref = orc.evict(p)
     g = p.to("cuda")
-    _compare_full(p, run_evict(g), ref)
+    _compare_full(p, run_evict(g), ref, orc)
     dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, window)
     i0 = torch.from_numpy(ref["i0"]).float().cuda()
     i1 = torch.from_numpy(ref["i1"]).float().cuda()
@@ -884,7 +874,7 @@ def test_split_prefix_vs_oracle_and_deterministic(case, orc):
     ref = orc.evict(p)
     g = p.to("cuda")
     a = run_evict(g)
-    _compare_full(p, a, ref)
+    _compare_full(p, a, ref, orc)
     b = run_evict(g)
     for key in ("i0", "i1", "delta", "kept", "packed", "cu_seqlens"):
         np.testing.assert_array_equal(a[key], b[key], err_msg=key)
@@ -921,11 +911,11 @@ def test_split_prefix_paged_and_constrained(orc):
     np.testing.assert_array_equal(i0.cpu().numpy(), packed_out["i0"].astype(np.float32))
     np.testing.assert_array_equal(i1.cpu().numpy(), packed_out["i1"].astype(np.float32))
     out = run_evict(g, constraints=3)
-    ref3 = orc.evict(p, constraints=3)
     assert out["status"] == 0
-    assert_close_delta(out["delta"], ref3["pooled"])
-    check_structured(out["kept"], out["cu_seqlens"], ref3["kept"], ref3["cu_seqlens"],
-                     ref3["pooled"], p.decoded.numpy(), p.budget.numpy())
+    np.testing.assert_array_equal(out["delta"], packed_out["delta"])
+    assert_close_delta(out["delta"], ref["pooled"])
+    check_structured(out["kept"], out["cu_seqlens"], packed_out["kept"], packed_out["cu_seqlens"],
+                     ref, p.decoded.numpy(), p.budget.numpy(), 3, orc)
 
 
 def test_split_prefix_malformed_cu_prefix_reports():
@@ -943,49 +933,31 @@ def test_split_prefix_malformed_cu_prefix_reports():
 def test_all_options_together_vs_oracle(case, orc):
     """focus_evict_ex with every option at once: paged prefix keys (64-token pages), the
     layer-0 row log-sum-exps given, the dynamic budget and both structural constraints,
-    against the oracle run with the same options."""
-    import attention_delta_token_b200 as F
+    against the oracle run with the same options: every request's budget within the
+    oracle's bounds, every retained list the closure of candidates that match the
+    oracle's selection under the GPU's budgets."""
     cfg, ov, wide = STRUCTURED_CASES[case]
     p = synth.make_problem(cfg, seed=910, wide_logits=wide, overrides=ov)
     lse = _row_lse(p).float()
     avg = np.random.default_rng(9).uniform(0.0, 4.0, size=p.R).astype(np.float32)
-    ref = orc.evict(p, constraints=3, lse0=lse.double().numpy(), decode_avg=avg.astype(np.float64))
+    ref = orc.evict(p, lse0=lse.double().numpy(), decode_avg=avg.astype(np.float64))
     g = p.to("cuda")
     pg = synth.to_paged(p, 64, seed=910).to("cuda")
-    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window, 3)
-    ws = F.Workspace(dims)
-    cap = F.plan_capacity(p.decoded, None, 3, dynamic=True)
-    kept = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
-    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
-    packed = torch.zeros(cap, p.H, dtype=torch.bfloat16, device="cuda")
-    delta = torch.empty(p.R, p.B, device="cuda")
-    i0 = torch.empty_like(delta)
-    i1 = torch.empty_like(delta)
-    kout = torch.full((p.R,), -1, dtype=torch.int32, device="cuda")
-    F.focus_evict_ex(dims, q0=g.q0, k0_block=g.k0_block, lse0=lse.cuda(), q1=g.q1,
-                     k1_prefix=pg.k1_pages, k1_block=g.k1_block, page_table=pg.page_table,
-                     prefix_len=pg.prefix_len, hidden=g.hidden, decoded=g.decoded,
-                     decode_avg=torch.from_numpy(avg).cuda(), budget_alpha=1.5, budget_out=kout,
-                     kept_idx=kept, cu_seqlens=cu, packed=packed, ws=ws, delta_out=delta,
-                     i0_out=i0, i1_out=i1)
-    assert F.focus_read_device_status(ws) == 0
-    assert_close_importance(i0.cpu().numpy(), ref["i0"], "I0 from lse")
-    assert_close_importance(i1.cpu().numpy(), ref["i1"], "I1 (paged)")
-    assert_close_delta(delta.cpu().numpy(), ref["pooled"])
-    kg = kout.cpu().numpy()
+    opts = dict(q0=g.q0, k0_prefix=None, k0_block=g.k0_block, lse0=lse.cuda(), q1=g.q1,
+                k1_prefix=pg.k1_pages, k1_block=g.k1_block, cu_prefix=None,
+                page_table=pg.page_table, prefix_len=pg.prefix_len)
+    out = _evict_dynamic(p, g, avg, 3, **opts)
+    cand = _evict_dynamic(p, g, avg, 0, **opts)
+    assert out["status"] == 0 and cand["status"] == 0
+    np.testing.assert_array_equal(out["delta"], cand["delta"])
+    np.testing.assert_array_equal(out["budget"], cand["budget"])
+    assert_close_delta(out["delta"], ref["pooled"])
     dec = p.decoded.numpy()
-    decided = [r for r in range(p.R) if kg[r] == ref["budget"][r]]
-    assert len(decided) >= p.R // 2
-    cu_h = cu.cpu().numpy()
-    n = int(cu_h[-1])
-    # retained sets of the requests whose budget the oracle agrees on (the oracle run on
-    # exactly those requests, as check_structured indexes them)
-    sub = orc.evict(p.subset(decided), constraints=3, lse0=lse[decided].double().numpy(),
-                    decode_avg=avg[decided].astype(np.float64))
-    check_structured(kept[:n].cpu().numpy(), cu_h, sub["kept"], sub["cu_seqlens"], sub["pooled"],
-                     dec, kg, requests=decided)
-    check_packed(packed[:n].view(torch.int16).cpu().numpy().view(np.uint16),
-                 kept[:n].cpu().numpy(), cu_h, hidden_bits(p))
+    kg = out["budget"]
+    check_dynamic_budget(kg, ref["pooled"], dec, avg)
+    check_structured(out["kept"], out["cu_seqlens"], cand["kept"], cand["cu_seqlens"], ref, dec,
+                     kg, 3, orc)
+    check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))
 
 
 def test_paged_bad_entries_report():
@@ -1053,7 +1025,7 @@ def test_split_prefix_with_lse0_vs_oracle(orc):
     assert_close_importance(i0.numpy(), ref["i0"], "I0 from lse")
     assert_close_importance(i1.numpy(), ref["i1"], "I1 (split)")
     assert_close_delta(delta.numpy(), ref["pooled"])
-    check_selection(kept.numpy(), cu.numpy(), ref["pooled"], p.decoded.numpy(), p.budget.numpy())
+    check_selection_all(kept.numpy(), cu.numpy(), ref, p.decoded.numpy(), p.budget.numpy(), orc)
     for a, b in zip(outs[0], outs[1]):
         assert torch.equal(a, b)
 
