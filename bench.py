@@ -125,7 +125,7 @@ class ClockSampler:
     """Reads SM clock and clock-event reasons through NVML every `period` seconds
     while the timed region runs.  Read-only: it changes no GPU setting."""
 
-    def __init__(self, device_index: int, period: float = 0.02):
+    def __init__(self, device_index: int, period: float = 0.001):
         self.samples = []
         self.period = period
         self.ok = False
@@ -393,6 +393,32 @@ def run_ours(args, rank, world, local_rank):
     attn_s_max = max_over_ranks(attn_s, dev)
     step_s = elapsed_max / args.steps
 
+    # ---- sustained: the same step repeated for about --sustained-seconds after the timed
+    # steps (not part of ms_per_step), so the line also shows the rate once the board has
+    # reached its power limit.  Every rank runs the same count (from the max-over-ranks time).
+    sustained = None
+    if args.sustained_seconds > 0:
+        n_sus = max(1, math.ceil(args.sustained_seconds / step_s))
+        s_sampler = ClockSampler(local_rank)
+        with s_sampler:
+            s3 = torch.cuda.Event(enable_timing=True)
+            t3 = torch.cuda.Event(enable_timing=True)
+            barrier()
+            s3.record(stream)
+            for _ in range(n_sus):
+                if graph is not None:
+                    graph.replay()
+                else:
+                    step()
+            t3.record(stream)
+            barrier()
+        sus_s = max_over_ranks(s3.elapsed_time(t3) / 1e3, dev) / n_sus
+        sustained = {"value": p.R / sus_s if tp > 1 else job_throughput(world, p.R, sus_s),
+                     "unit": UNIT, "ms_per_step": sus_s * 1e3, "steps": n_sus,
+                     "seconds": sus_s * n_sus, "clocks": s_sampler.summary()}
+        if F.focus_read_device_status(ws) != 0:
+            raise RuntimeError("device status after the sustained run")
+
     # ---- end to end: pinned host inputs -> device, the C-ABI call, result -> host
     e2e = None
     variant = args.score or args.lse0 or args.page_size or args.dynamic_budget or tp > 1
@@ -488,6 +514,7 @@ def run_ours(args, rank, world, local_rank):
                 "peaks": f"{peak_src}: hbm {hbm} GB/s, bf16 {tc} TFLOP/s",
             },
             "clocks": clocks,
+            "sustained": sustained,
             # plan, attention statistics, select, (scan,) compact; split into two calls
             # (tp): plan, attention, reduce + plan, select, (scan,) compact
             # (list mode: structural constraints or the dynamic budget add the scan kernel)
@@ -515,11 +542,37 @@ def cpu_baseline(p, target_s: float = 12.0) -> dict:
         t0 = time.perf_counter()
         oracle.evict(cpu_p)
         t = time.perf_counter() - t0
+    single = cpu_baseline_single_thread(p, target_s=target_s / 2)
     return {"value": n / t, "unit": UNIT, "cores": threads, "kind": "oracle",
             "seconds": t,
             "sample": f"requests 0..{n - 1} ({n} of {p.R} blocks) of the same workload; "
                       f"both layers' importance, delta, pooling, mask, top-K, compaction in "
-                      f"float64 (OpenMP over request x kv-head pairs)"}
+                      f"float64 (OpenMP over request x kv-head pairs)",
+            "single_thread": single}
+
+
+def cpu_baseline_single_thread(p, target_s: float = 6.0) -> dict:
+    """The same oracle on one host thread, on the first few requests of the workload
+    (2, then as many as fit in about `target_s`)."""
+    import oracle
+    threads = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        n = min(p.R, 2)
+        sub = p.subset(range(n)).to("cpu")
+        t0 = time.perf_counter()
+        oracle.evict(sub)
+        t = time.perf_counter() - t0
+        if t < target_s / 2 and n < p.R:
+            n = int(min(p.R, max(n + 1, round(n * target_s / max(t, 1e-3)))))
+            sub = p.subset(range(n)).to("cpu")
+            t0 = time.perf_counter()
+            oracle.evict(sub)
+            t = time.perf_counter() - t0
+    finally:
+        oracle.set_num_threads(threads)
+    return {"value": n / t, "unit": UNIT, "cores": 1, "seconds": t,
+            "sample": f"requests 0..{n - 1} ({n} of {p.R} blocks), one thread"}
 
 
 # ---------------------------------------------------------------- reference arm
@@ -600,6 +653,9 @@ def main():
                          "exchange fused into the kernels over peer memory")
     ap.add_argument("--graph", action="store_true",
                     help="replay the step as a captured CUDA graph in the timed loop")
+    ap.add_argument("--sustained-seconds", type=float, default=1.0,
+                    help="after the timed steps, repeat the step for about this long and report "
+                         "its rate and clocks separately (0: skip)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

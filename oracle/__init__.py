@@ -97,15 +97,21 @@ class Oracle:
                                                       P, i32, i32, P, P]
         lib.focus_oracle_dynamic_budget.argtypes = [i32, i32, P, P, P, f64, P]
         lib.focus_oracle_num_threads.argtypes = []
+        lib.focus_oracle_set_num_threads.argtypes = [i32]
         for fn in (lib.focus_oracle_importance, lib.focus_oracle_delta, lib.focus_oracle_select,
                    lib.focus_oracle_compact, lib.focus_oracle_num_threads,
                    lib.focus_oracle_select_structured, lib.focus_oracle_importance_lse,
-                   lib.focus_oracle_importance_paged, lib.focus_oracle_dynamic_budget):
+                   lib.focus_oracle_importance_paged, lib.focus_oracle_dynamic_budget,
+                   lib.focus_oracle_set_num_threads):
             fn.restype = ctypes.c_int
         self.lib = lib
 
     def num_threads(self) -> int:
         return int(self.lib.focus_oracle_num_threads())
+
+    def set_num_threads(self, n: int) -> int:
+        """Threads of the later calls (timing only: results do not depend on it)."""
+        return int(self.lib.focus_oracle_set_num_threads(int(n)))
 
     def importance(self, q, k_prefix, cu_prefix, k_block, *, Hq: int, Hkv: int,
                    scale: float) -> np.ndarray:
@@ -269,6 +275,10 @@ def default() -> Oracle:
 
 def num_threads() -> int:
     return default().num_threads()
+
+
+def set_num_threads(n: int) -> int:
+    return default().set_num_threads(n)
 
 
 def importance(*a, **k):

@@ -73,6 +73,19 @@ int focus_oracle_num_threads(void)
 #endif
 }
 
+/* Threads the following calls use (n >= 1); returns the count now in effect.  Only
+ * the timing of the CPU baseline changes it (single-thread and all-core runs). */
+int focus_oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n >= 1)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+    return focus_oracle_num_threads();
+}
+
 /*
  * Attention importance of one layer (the "column-wise sum of softmax attention
  * weights received by token j from all query tokens in the block").

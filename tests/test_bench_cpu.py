@@ -62,3 +62,16 @@ def test_workload_overrides():
     assert p.R == 4 and (p.prefix_len >= 15000).all() and (p.prefix_len <= 16000).all()
     assert bench.rank_seed(2, 0) == 2 and bench.rank_seed(2, 1) != 2
     assert np.isclose(bench.job_throughput(2, 256, 0.5), 1024.0)
+
+
+def test_cpu_baseline_reports_all_core_and_single_thread():
+    """The oracle's timing on the host: the all-core figure and a one-thread figure on
+    a sample of the same workload, with the thread count restored afterwards."""
+    import oracle
+    p = synth.make_problem(1, overrides=dict(R=4, prefix=("uniform", 0, 200)))
+    threads = oracle.num_threads()
+    cb = bench.cpu_baseline(p, target_s=0.2)
+    assert cb["kind"] == "oracle" and cb["cores"] == threads and cb["value"] > 0
+    one = cb["single_thread"]
+    assert one["cores"] == 1 and one["value"] > 0 and one["unit"] == "blocks/s"
+    assert oracle.num_threads() == threads
