@@ -590,6 +590,11 @@ EDGE_CASES = {
     "mqa_g32": (1, dict(R=3, Hq=32, Hkv=1, prefix=("uniform", 0, 400))),
     # d = 64 with 16 query heads per kv head
     "d64_g16": (1, dict(R=4, d=64, Hq=32, Hkv=2, prefix=("uniform", 0, 300))),
+    # the largest group: 128 query heads on one kv head, one block token per row tile
+    "g128_b4": (0, dict(R=3, B=4, Hq=128, Hkv=1, d=64, H=64, prefix=("uniform", 0, 300),
+                        decoded=("uniform", 0.0, 0.5), lift=("frac", 0.25), budget=("ceil", 0.5))),
+    # the largest block with 64 query heads per kv head: 64 row tiles per kv head
+    "g64_b128": (3, dict(R=2, d=64, Hq=64, Hkv=1, H=256, prefix=("uniform", 100, 400))),
 }
 
 
