@@ -114,6 +114,58 @@ def test_deterministic():
         np.testing.assert_array_equal(a[k], b[k], err_msg=k)
 
 
+def test_deterministic_full_ragged_workload():
+    """The ragged workload at full size (4,096 work items over the persistent grid, most of
+    them short): two calls give identical bits."""
+    p = synth.make_problem(4, wide_logits=True).to("cuda")
+    a, b = run_evict(p), run_evict(p)
+    for k in ("i0", "i1", "delta", "kept", "cu_seqlens", "packed"):
+        np.testing.assert_array_equal(a[k], b[k], err_msg=k)
+
+
+def test_consecutive_denoising_steps_vs_oracle(orc):
+    """One workspace and one set of output buffers across five denoising steps, as an
+    engine would use them: after each step a few of the kept (still-masked) tokens become
+    decoded and the budgets shrink with the masked counts; every step matches the oracle."""
+    import attention_delta_token_b200 as F
+    p = synth.make_problem(1, seed=77, wide_logits=True,
+                           overrides=dict(R=12, prefix=("uniform", 0, 900)))
+    g = p.to("cuda")
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+    ws = F.Workspace(dims)
+    kept = torch.empty(p.R * p.B, dtype=torch.int32, device="cuda")
+    cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+    packed = torch.empty(p.R * p.B, p.H, dtype=torch.bfloat16, device="cuda")
+    delta = torch.empty(p.R, p.B, device="cuda")
+    rng = np.random.default_rng(5)
+    for step in range(5):
+        dec = p.decoded.numpy()
+        masked = (dec == 0).sum(1)
+        p.budget = torch.from_numpy(np.maximum(1, np.ceil(0.3 * masked)).astype(np.int32))
+        p.budget[masked == 0] = 0
+        g.decoded, g.budget = p.decoded.cuda(), p.budget.cuda()
+        F.focus_evict(dims, g.q0, g.k0_prefix, g.k0_block, g.q1, g.k1_prefix, g.k1_block,
+                      g.cu_prefix, g.hidden, g.decoded, g.budget, kept, cu, packed, ws,
+                      delta_out=delta)
+        assert F.focus_read_device_status(ws) == 0, step
+        ref = orc.evict(p)
+        cu_h = cu.cpu().numpy()
+        n = int(cu_h[-1])
+        np.testing.assert_array_equal(cu_h, ref["cu_seqlens"])
+        assert_close_delta(delta.cpu().numpy(), ref["pooled"])
+        kept_h = kept[:n].cpu().numpy()
+        check_selection_all(kept_h, cu_h, ref, p.decoded.numpy(), p.budget.numpy(), orc)
+        check_packed(packed[:n].view(torch.int16).cpu().numpy().view(np.uint16), kept_h, cu_h,
+                     hidden_bits(p))
+        # the next step: up to two kept tokens per request are decoded
+        new = p.decoded.clone()
+        for r in range(p.R):
+            seg = kept_h[cu_h[r]:cu_h[r + 1]]
+            if seg.size:
+                new[r, rng.choice(seg, size=min(2, seg.size), replace=False)] = 1
+        p.decoded = new
+
+
 def test_standalone_chain_matches_fused():
     """attn_stats x2 -> importance_delta -> topk_select -> compact reproduces
     focus_evict bit for bit (same reduction order everywhere)."""
