@@ -13,8 +13,8 @@ import torch
 
 import synth
 from focus_testutil import (assert_close_delta, assert_close_importance, check_dynamic_budget,
-                            check_packed, check_selection, check_selection_all, check_structured,
-                            hidden_bits, run_evict)
+                            check_packed, check_selection_all, check_structured, hidden_bits,
+                            run_evict)
 
 pytestmark = pytest.mark.gpu
 
