@@ -97,6 +97,71 @@ def test_full_config_every_request(cfg, wide, orc, parity_report):
             rep)
 
 
+def _row_lse_on_device(g):
+    """Layer-0 row log-sum-exps [R, B, Hq] of a problem on the GPU, in float64 with torch
+    (setup: the input an engine's layer-0 attention forward hands over)."""
+    G = g.Hq // g.Hkv
+    cu = g.cu_prefix.cpu().numpy()
+    out = torch.empty(g.R, g.B, g.Hq, dtype=torch.float64, device=g.q0.device)
+    for r in range(g.R):
+        keys = torch.cat([g.k0_prefix[int(cu[r]):int(cu[r + 1])], g.k0_block[r]], 0).double()
+        q = g.q0[r].double()  # [B, Hq, d]
+        for kv in range(g.Hkv):
+            qs = q[:, kv * G:(kv + 1) * G].reshape(-1, g.d)
+            out[r, :, kv * G:(kv + 1) * G] = torch.logsumexp(
+                g.scale * (qs @ keys[:, kv].T), dim=-1).view(g.B, G)
+    return out
+
+
+@pytest.mark.parametrize("variant", ["paged64", "lse0", "score1", "dynamic"])
+def test_variants_full_metric_shape_every_request(variant, orc, parity_report):
+    """The options of the fused step at the metric shape (256 requests), every request
+    against the oracle run with the same option: paged prefix keys (64-token pages), the
+    layer-0 row log-sum-exps given, ranking by I1 alone, the dynamic budget."""
+    import attention_delta_token_b200 as F
+    p = synth.make_problem(2)
+    g = p.to("cuda")
+    dims = F.make_dims(p.R, p.B, p.Hq, p.Hkv, p.d, p.H, p.scale, p.pool_window)
+    budget = p.budget.numpy()
+    if variant == "score1":
+        out = run_evict(g, score=1)
+        ref = orc.evict(p, score=1)
+    elif variant == "dynamic":
+        avg = np.random.default_rng(12).uniform(0.0, 0.2 * p.B, size=p.R).astype(np.float32)
+        out = _evict_dynamic(p, g, avg, 0)
+        ref = orc.evict(p, decode_avg=avg.astype(np.float64))
+        check_dynamic_budget(out["budget"], ref["pooled"], p.decoded.numpy(), avg)
+        budget = out["budget"]
+    else:
+        ws = F.Workspace(dims)
+        cap = F.plan_capacity(p.decoded, p.budget)
+        kept = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+        cu = torch.empty(p.R + 1, dtype=torch.int32, device="cuda")
+        packed = torch.zeros(cap, p.H, dtype=torch.bfloat16, device="cuda")
+        delta = torch.empty(p.R, p.B, device="cuda")
+        if variant == "paged64":
+            pg = synth.to_paged(g, 64, seed=2)
+            F.focus_evict_paged(dims, g.q0, pg.k0_pages, g.k0_block, g.q1, pg.k1_pages, g.k1_block,
+                                pg.page_table, pg.prefix_len, g.hidden, g.decoded, g.budget, kept,
+                                cu, packed, ws, delta_out=delta)
+            ref = orc.evict(p)
+        else:
+            lse = _row_lse_on_device(g).float()  # both sides take the same float32 values
+            F.focus_evict_with_lse0(dims, lse, g.q0, g.k0_block, g.q1, g.k1_prefix, g.k1_block,
+                                    g.cu_prefix, g.hidden, g.decoded, g.budget, kept, cu, packed,
+                                    ws, delta_out=delta)
+            ref = orc.evict(p, lse0=lse.double().cpu().numpy())
+        st = F.focus_read_device_status(ws)
+        out = dict(status=st, kept=kept.cpu().numpy(), cu_seqlens=cu.cpu().numpy(),
+                   packed=packed.view(torch.int16).cpu().numpy().view(np.uint16),
+                   delta=delta.cpu().numpy().astype(np.float64))
+    assert out["status"] == 0
+    assert_close_delta(out["delta"], ref["pooled"])
+    rep = check_selection_all(out["kept"], out["cu_seqlens"], ref, p.decoded.numpy(), budget, orc)
+    check_packed(out["packed"], out["kept"], out["cu_seqlens"], hidden_bits(p))
+    _report(parity_report, f"sdar8b_r256_b32 ({variant})", rep)
+
+
 def test_duplicate_keys_give_equal_columns():
     """A duplicated block key (same K rows at both layers) gets bit-equal I columns."""
     p = synth.make_problem(4, overrides=dict(R=24, prefix=("loguniform", 900), tie_frac=0.5))
