@@ -467,6 +467,7 @@ def run_ours(args, rank, world, local_rank):
         workload = cfg.name
         clocks = sampler.summary()
         sm_hz = (clocks["sm_mhz"] or 1965.0) * 1e6
+        t_mufu = counts["exps"] / (16 * 148 * sm_hz)  # one SFU exp per (row, key): 16 per clock per SM
         result = {
             "metric": METRIC,
             "value": p.R / step_s if tp > 1 else job_throughput(world, p.R, step_s), "unit": UNIT,
@@ -508,8 +509,9 @@ def run_ours(args, rank, world, local_rank):
             },
             "roofline_step": {
                 "t_hbm_us": t_hbm * 1e6, "t_tensor_us": t_tc * 1e6,
-                "t_mufu_us": counts["exps"] / (16 * 148 * sm_hz) * 1e6,
-                "frac": max(t_hbm, t_tc) / step_s, "bytes": counts["bytes"],
+                "t_mufu_us": t_mufu * 1e6,
+                "frac": max(t_hbm, t_tc) / step_s,
+                "frac_with_sfu": max(t_hbm, t_tc, t_mufu) / step_s, "bytes": counts["bytes"],
                 "flops": counts["flops"], "exps": counts["exps"],
                 "peaks": f"{peak_src}: hbm {hbm} GB/s, bf16 {tc} TFLOP/s",
             },
