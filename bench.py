@@ -27,7 +27,6 @@ import math
 import os
 import statistics
 import sys
-import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -121,61 +120,112 @@ REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_c
            0x100: "display_clock_setting"}
 
 
+# The sampling loop runs in a child process of its own, so that it keeps its period
+# while this process waits for the GPU (a thread here would wait for the interpreter
+# lock).  It only reads NVML: SM clock and clock-event reasons, one line per sample,
+# until its standard input closes.
+_SAMPLER_SRC = r"""
+import select, sys, time
+import pynvml
+pynvml.nvmlInit()
+dev, period, out = sys.argv[1], float(sys.argv[2]), sys.argv[3]
+h = (pynvml.nvmlDeviceGetHandleByUUID(dev) if dev.startswith("GPU-")
+     else pynvml.nvmlDeviceGetHandleByIndex(int(dev)))
+with open(out, "w") as f:
+    f.write("max %d\n" % pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+    f.flush()
+    while True:
+        t = time.monotonic()
+        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+        rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+        f.write("%.6f %d %d\n" % (t, sm, rs))
+        if select.select([sys.stdin], [], [], period)[0]:
+            break
+"""
+
+
 class ClockSampler:
     """Reads SM clock and clock-event reasons through NVML every `period` seconds
-    while the timed region runs.  Read-only: it changes no GPU setting."""
+    (in a child process) while the timed region runs; `mark_start` / `mark_stop`
+    bracket the region the summary covers.  Read-only: it changes no GPU setting."""
 
-    def __init__(self, device_index: int, period: float = 0.001):
-        self.samples = []
+    def __init__(self, device_index: int, period: float = 0.0005):
+        self.samples = []      # (monotonic time, SM MHz, reason bits)
         self.period = period
-        self.ok = False
         self.sm_max = None
+        self.window = [None, None]
+        self._proc = None
+        self._file = None
         try:
-            import pynvml
-            pynvml.nvmlInit()
-            self.nv = pynvml
+            import pynvml  # noqa: F401  (the child needs it)
             try:
                 uuid = str(torch.cuda.get_device_properties(device_index).uuid)
-                if not uuid.startswith("GPU-"):
-                    uuid = "GPU-" + uuid
-                self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+                self.dev = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
             except Exception:
-                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
-            self.sm_max = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+                self.dev = str(device_index)
             self.ok = True
         except Exception:
             self.ok = False
-        self._stop = threading.Event()
-        self._t = None
-
-    def _run(self):
-        while not self._stop.is_set():
-            try:
-                sm = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
-                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                self.samples.append((sm, rs))
-            except Exception:
-                pass
-            time.sleep(self.period)
 
     def __enter__(self):
-        if self.ok:
-            self._t = threading.Thread(target=self._run, daemon=True)
-            self._t.start()
+        if not self.ok:
+            return self
+        import subprocess
+        import tempfile
+        fd, self._file = tempfile.mkstemp(prefix="focus_clocks_", suffix=".txt")
+        os.close(fd)
+        self._proc = subprocess.Popen(
+            [sys.executable, "-c", _SAMPLER_SRC, self.dev, str(self.period), self._file],
+            stdin=subprocess.PIPE, stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        t0 = time.monotonic()
+        while time.monotonic() - t0 < 20.0:  # until the first sample is written
+            if self._proc.poll() is not None:
+                break
+            with open(self._file) as f:
+                if len(f.read().splitlines()) >= 2:
+                    break
+            time.sleep(0.01)
         return self
 
+    def mark_start(self):
+        self.window[0] = time.monotonic()
+
+    def mark_stop(self):
+        self.window[1] = time.monotonic()
+
     def __exit__(self, *a):
-        self._stop.set()
-        if self._t:
-            self._t.join()
+        if self._proc is None:
+            return
+        try:
+            self._proc.stdin.close()
+            self._proc.wait(timeout=10)
+        except Exception:
+            self._proc.kill()
+        try:
+            for line in open(self._file).read().splitlines():
+                parts = line.split()
+                if parts[0] == "max":
+                    self.sm_max = int(parts[1])
+                elif len(parts) == 3:
+                    self.samples.append((float(parts[0]), int(parts[1]), int(parts[2])))
+        except Exception:
+            pass
+        finally:
+            os.unlink(self._file)
 
     def summary(self) -> dict:
-        if not self.ok or not self.samples:
+        sel = self.samples
+        lo, hi = self.window
+        if lo is not None and hi is not None:
+            inside = [x for x in self.samples if lo <= x[0] <= hi]
+            if inside:
+                sel = inside
+        if not sel:
             return {"sm_mhz": None, "sm_max_mhz": self.sm_max, "reasons": [], "samples": 0}
-        sms = [s for s, _ in self.samples]
+        sms = [sm for _, sm, _ in sel]
         bits = 0
-        for _, r in self.samples:
-            bits |= int(r)
+        for _, _, r in sel:
+            bits |= r
         names = [n for b, n in REASONS.items() if bits & b and n != "gpu_idle"]
         return {"sm_mhz": float(statistics.median(sms)), "sm_max_mhz": self.sm_max,
                 "reasons": names, "samples": len(sms)}
@@ -365,6 +415,7 @@ def run_ours(args, rank, world, local_rank):
         start = torch.cuda.Event(enable_timing=True)
         stop = torch.cuda.Event(enable_timing=True)
         barrier()
+        sampler.mark_start()
         start.record(stream)
         for k in range(args.steps):
             if graph is not None:
@@ -377,6 +428,7 @@ def run_ours(args, rank, world, local_rank):
                 F.focus_set_trace_events(None, None)
         stop.record(stream)
         barrier()
+        sampler.mark_stop()
         if graph is not None:
             for i in range(len(traced)):
                 F.focus_set_trace_events(ev_a[i], ev_b[i])
