@@ -279,6 +279,9 @@ __global__ void __launch_bounds__(256) select_compact_kernel(const SelectParams 
             }
             if (p.i1_out) p.i1_out[rb + j] = i1;
             if (p.raw_out) p.raw_out[rb + j] = raw_s[j];
+            // I is a sum of softmax weights, finite for any finite Q and K: a non-finite
+            // value means non-finite inputs (out of contract), reported, not ranked silently.
+            if (!isfinite(raw_s[j])) atomicOr(p.status, FOCUS_DEV_BAD_INPUT);
         }
         __syncthreads();
         if (j < B) {
@@ -287,7 +290,11 @@ __global__ void __launch_bounds__(256) select_compact_kernel(const SelectParams 
             if (p.delta_out) p.delta_out[rb + j] = d;
         }
     } else {
-        if (j < B) val_s[j] = p.delta_in[rb + j];
+        if (j < B) {
+            val_s[j] = p.delta_in[rb + j];
+            // still-masked positions carry finite scores; anything else is out of contract
+            if (dec_s[j] == 0 && !isfinite(val_s[j])) atomicOr(p.status, FOCUS_DEV_BAD_INPUT);
+        }
     }
     __syncthreads();
 

@@ -76,7 +76,8 @@ typedef enum {
     FOCUS_ERR_CAPACITY = 3,          /* device: sum k_r > capacity (extra rows not written) */
     FOCUS_ERR_WORKSPACE = 4,         /* workspace null, misaligned or too small            */
     FOCUS_ERR_CUDA = 5,              /* a CUDA runtime/driver call failed                  */
-    FOCUS_ERR_DEVICE_CHECK = 6,      /* device: malformed cu_prefix or kept index          */
+    FOCUS_ERR_DEVICE_CHECK = 6,      /* device: malformed cu_prefix, page or kept index, or
+                                        non-finite inputs (seen as non-finite importance) */
     FOCUS_ERR_TIMEOUT = 7            /* device wait gave up, or status read timed out      */
 } focus_status_t;
 
@@ -198,7 +199,8 @@ FOCUS_API focus_status_t focus_importance_delta(const focus_dims_t *dims, const 
  *   delta [R, B] float32 (as produced by focus_importance_delta); budget [R] int32;
  *   kept_idx [capacity] int32 out; cu_seqlens [R + 1] int32 out.
  * Rows beyond `capacity` are not written and FOCUS_ERR_CAPACITY is set in the
- * device status (cu_seqlens is still complete).
+ * device status (cu_seqlens is still complete).  A non-finite delta at a still-masked
+ * position is out of contract and sets FOCUS_ERR_DEVICE_CHECK.
  */
 FOCUS_API focus_status_t focus_topk_select(const focus_dims_t *dims, const float *delta,
                                  const uint8_t *decoded, const int32_t *budget, int32_t *kept_idx,
@@ -224,6 +226,9 @@ FOCUS_API focus_status_t focus_compact(const focus_dims_t *dims, const void *hid
  * and i1_out ([R, B] float32) are optional (NULL skips them).  With
  * dims.score == FOCUS_SCORE_LAYER1 the layer-0 arguments may be NULL, I0 is not
  * computed (i0_out is left untouched) and delta_out holds the pooled, masked I1.
+ * Non-finite Q or K values are out of contract: they make the importance of their
+ * request non-finite, which sets FOCUS_ERR_DEVICE_CHECK; every access stays in
+ * bounds and the other requests are unaffected.
  */
 FOCUS_API focus_status_t focus_evict(const focus_dims_t *dims, const void *q0, const void *k0_prefix,
                            const void *k0_block, const void *q1, const void *k1_prefix,
@@ -457,8 +462,8 @@ FOCUS_API focus_status_t focus_selftest_exchange(const float *partials, void *co
  *  - Arguments and results are those of focus_evict, minus the workspace.
  *  - device_status (nullable, device pointer, 4-byte aligned) receives the
  *    call's raw device status bits: 1 = rows beyond `capacity`, 2 = malformed
- *    cu_prefix or kept index, 4 = a kernel wait gave up; 0 = fine.  It is written
- *    on `stream` after the kernels.
+ *    cu_prefix, page or kept index, or non-finite inputs, 4 = a kernel wait
+ *    gave up; 0 = fine.  It is written on `stream` after the kernels.
  *  - Returns FOCUS_ERR_WORKSPACE when focus_workspace_size(dims) exceeds
  *    FOCUS_STATIC_SCRATCH_BYTES (shapes that large need focus_evict), otherwise
  *    the same codes as focus_evict.  The largest batch is set by the workspace

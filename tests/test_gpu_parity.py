@@ -335,6 +335,35 @@ def test_malformed_cu_prefix_reports():
     assert out["status"] == 6  # FOCUS_ERR_DEVICE_CHECK
 
 
+def test_non_finite_inputs_are_reported_and_contained(orc):
+    """A NaN in one request's layer-1 queries (out of contract) makes that request's
+    importance non-finite: the call reports FOCUS_ERR_DEVICE_CHECK, cu_seqlens keeps its
+    count-based values, and every other request still matches the oracle."""
+    p = synth.make_problem(1, seed=55, wide_logits=True, overrides=dict(R=6, prefix=("uniform", 100, 600)))
+    bad = 2
+    q1 = p.q1.clone()
+    q1[bad, 0, 0, 0] = float("nan")
+    p.q1 = q1
+    out = run_evict(p.to("cuda"))
+    assert out["status"] == 6  # FOCUS_ERR_DEVICE_CHECK
+    good = [r for r in range(p.R) if r != bad]
+    sub = p.subset(good)
+    ref = orc.evict(sub)
+    _, cu_all, _ = orc.select(np.zeros((p.R, p.B)), p.decoded, p.budget)
+    np.testing.assert_array_equal(out["cu_seqlens"], cu_all)
+    assert_close_importance(out["i0"], orc.evict(p)["i0"], "I0 (layer 0 has no NaN)")
+    assert_close_delta(out["delta"][good], ref["pooled"])
+    kept, cu, packed = [], [0], []
+    for r in good:
+        a, b = int(out["cu_seqlens"][r]), int(out["cu_seqlens"][r + 1])
+        kept.append(out["kept"][a:b])
+        packed.append(out["packed"][a:b])
+        cu.append(cu[-1] + (b - a))
+    check_selection_all(np.concatenate(kept), np.array(cu), ref, sub.decoded.numpy(),
+                        sub.budget.numpy(), orc)
+    check_packed(np.concatenate(packed), np.concatenate(kept), np.array(cu), hidden_bits(sub))
+
+
 def test_bounded_wait_times_out_and_reports():
     """A kernel waiting on a barrier that never completes gives up after its limit,
     reports FOCUS_DEV_TIMEOUT in the status word, and leaves the context usable."""
