@@ -335,6 +335,22 @@ def test_malformed_cu_prefix_reports():
     assert out["status"] == 6  # FOCUS_ERR_DEVICE_CHECK
 
 
+@pytest.mark.parametrize("factor", [0.0, 0.5, 2.0])
+def test_softmax_scale_other_than_default(factor, orc):
+    """softmax_scale is an argument: zero (every row's softmax uniform over its keys), half
+    and twice 1/sqrt(d), against the oracle with the same scale."""
+    import dataclasses
+    p = synth.make_problem(1, seed=61, wide_logits=True, overrides=dict(R=5, prefix=("uniform", 0, 500)))
+    p = dataclasses.replace(p, scale=p.scale * factor)
+    ref = orc.evict(p)
+    out = run_evict(p.to("cuda"))
+    _compare_full(p, out, ref, orc)
+    if factor == 0.0:  # uniform rows: I_j = B Hq / N_r for every block column
+        N = p.prefix_len + p.B
+        np.testing.assert_allclose(out["i1"], (p.B * p.Hq / N)[:, None] * np.ones((1, p.B)),
+                                   rtol=1e-5)
+
+
 def test_non_finite_inputs_are_reported_and_contained(orc):
     """A NaN in one request's layer-1 queries (out of contract) makes that request's
     importance non-finite: the call reports FOCUS_ERR_DEVICE_CHECK, cu_seqlens keeps its
