@@ -315,6 +315,20 @@ def test_zero_budget_and_all_decoded(orc):
     assert out["cu_seqlens"][1] == 0 and out["cu_seqlens"][2] == 0
 
 
+def test_nothing_kept_anywhere(orc):
+    """Every budget zero: the packed batch is empty (capacity 0), cu_seqlens is all zeros, the
+    importance is still computed and matches the oracle."""
+    p = synth.make_problem(1, overrides=dict(R=5, prefix=("uniform", 0, 300)))
+    p.budget = torch.zeros(p.R, dtype=torch.int32)
+    out = run_evict(p.to("cuda"))
+    assert out["status"] == 0
+    np.testing.assert_array_equal(out["cu_seqlens"], np.zeros(p.R + 1, np.int32))
+    assert out["kept"].size == 0 and out["packed"].shape[0] == 0
+    ref = orc.evict(p)
+    assert_close_importance(out["i1"], ref["i1"], "I1")
+    assert_close_delta(out["delta"], ref["pooled"])
+
+
 def test_capacity_overflow_reports_and_stays_in_bounds():
     import attention_delta_token_b200 as F
     p = synth.make_problem(1, overrides=dict(R=4, prefix=("uniform", 0, 300))).to("cuda")
@@ -752,6 +766,9 @@ EDGE_CASES = {
     "mqa_g32": (1, dict(R=3, Hq=32, Hkv=1, prefix=("uniform", 0, 400))),
     # d = 64 with 16 query heads per kv head
     "d64_g16": (1, dict(R=4, d=64, Hq=32, Hkv=2, prefix=("uniform", 0, 300))),
+    # prefixes ending just before, at and just after a 128-key tile boundary
+    "tile_edges_128": (1, dict(R=12, prefix=("uniform", 127, 129))),
+    "tile_edges_256": (4, dict(R=12, prefix=("uniform", 255, 257))),
     # the largest group: 128 query heads on one kv head, one block token per row tile
     "g128_b4": (0, dict(R=3, B=4, Hq=128, Hkv=1, d=64, H=64, prefix=("uniform", 0, 300),
                         decoded=("uniform", 0.0, 0.5), lift=("frac", 0.25), budget=("ceil", 0.5))),
