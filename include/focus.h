@@ -43,13 +43,14 @@
  *    `capacity` = sum_r k_r exactly.
  *  - Kept positions are written in ascending order per request; requests are
  *    packed in order: request r owns rows cu_seqlens[r] .. cu_seqlens[r+1]-1.
- *  - CUDA graphs: every call that enqueues kernels may be captured into a graph
- *    (it only launches kernels, with programmatic dependent launch between them,
- *    and never synchronises).  Make one uncaptured call per process first (it
- *    looks up the driver's tensor-map encoder).  Tensor maps hold the pointers
- *    given at capture, so a replay reads and writes the same buffers: copy new
- *    inputs into them before each replay.  focus_read_device_status synchronises
- *    and cannot be captured.
+ *  - CUDA graphs: every call that takes the caller's workspace and enqueues
+ *    kernels may be captured into a graph (it only launches kernels, with
+ *    programmatic dependent launch between them, and never synchronises); this
+ *    note does not cover focus_evict_static_scratch.  Make one uncaptured call
+ *    per process first (it looks up the driver's tensor-map encoder).  Tensor
+ *    maps hold the pointers given at capture, so a replay reads and writes the
+ *    same buffers: copy new inputs into them before each replay.
+ *    focus_read_device_status synchronises and cannot be captured.
  */
 #ifndef FOCUS_H_
 #define FOCUS_H_
@@ -477,8 +478,7 @@ FOCUS_API focus_status_t focus_selftest_exchange(const float *partials, void *co
  *    untouched.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current; `stream` must belong to
- *    the current device) and keeps it for the life of the process.  Make that
- *    first call before any stream capture.  A cudaDeviceReset (or anything else
+ *    the current device) and keeps it for the life of the process.  A cudaDeviceReset (or anything else
  *    that destroys and recreates the device's primary context) may move the
  *    array: do not use this entry point on a device after such a reset.
  *  - All calls on a device share the one array and it keeps the last call's
