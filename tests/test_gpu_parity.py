@@ -760,6 +760,12 @@ EDGE_CASES = {
     "r1500_tiny_heads": (0, dict(R=1500, B=8, Hq=2, Hkv=1, d=64, H=64, prefix=("uniform", 0, 200),
                                  decoded=("uniform", 0.0, 0.5), lift=("frac", 0.2),
                                  budget=("ceil", 0.3))),
+    # the last batch ordered by a rank count (1024), the last one sorted (4096; the compaction
+    # no longer stages cu_seqlens in shared memory) and the first one kept in input order
+    **{f"r{R}_tiny_heads": (0, dict(R=R, B=8, Hq=2, Hkv=1, d=64, H=64, prefix=("uniform", 0, 200),
+                                    decoded=("uniform", 0.0, 0.5), lift=("frac", 0.2),
+                                    budget=("ceil", 0.3)))
+       for R in (1024, 4096, 4097)},
     # one very long prefix: 157 key tiles in one work item
     "long_prefix_20k": (1, dict(R=2, prefix=("uniform", 19000, 20000))),
     # multi-query attention: all 32 query heads read one kv head (4 tokens per row tile)
