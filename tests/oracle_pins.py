@@ -352,6 +352,17 @@ def pin_topk_bruteforce(orc):
         assert kept.tolist() == best[1], (vals, dec, K, kept, best)
 
 
+def pin_topk_signed_zeros(orc):
+    """-0.0 and +0.0 are the same value: they tie, and the lower position wins whatever
+    the sign (an order on the bit patterns would put every +0.0 first)."""
+    pooled = np.array([[-0.0, 0.0, -0.0, 0.0, 1.0, -1.0],
+                       [0.0, -0.0, 0.0, -0.0, -0.0, 0.0]], np.float64)
+    dec = np.zeros((2, 6), np.uint8)
+    kept, cu, st = orc.select(pooled, dec, np.array([3, 4], np.int32))
+    assert st == 0 and cu.tolist() == [0, 3, 7]
+    assert kept.tolist() == [0, 1, 4] + [0, 1, 2, 3]
+
+
 def pin_capacity_status(orc):
     """Selecting more rows than the packed buffer holds is reported, cu_seqlens is
     still complete, and only the rows that fit are written."""
@@ -461,7 +472,8 @@ PINS = [
     pin_block_permutation_equivariance, pin_key_shift_invariance, pin_gqa_expansion,
     pin_heads_sum, pin_requests_independent, pin_library_softmax_columns,
     pin_delta_sign_and_pool, pin_pool_spreads_decoded_neighbour, pin_topk_lexsort,
-    pin_topk_bruteforce, pin_capacity_status, pin_compact_fancy_indexing, pin_hand_evict,
+    pin_topk_bruteforce, pin_topk_signed_zeros, pin_capacity_status, pin_compact_fancy_indexing,
+    pin_hand_evict,
     pin_hand_structural, pin_structural_properties, pin_importance_lse_matches_full,
     pin_importance_lse_closed_form, pin_paged_prefix_matches_packed, pin_hand_dynamic_budget,
     pin_dynamic_budget_bounds,

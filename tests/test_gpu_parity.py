@@ -303,6 +303,45 @@ def test_standalone_steps_vs_oracle(orc):
     assert F.focus_read_device_status(ws) == 0
 
 
+def test_signed_zero_ties_vs_oracle(orc):
+    """-0.0 and +0.0 tie (the lower position wins whatever the sign), in the selection
+    call and after the delta step, whose I1 - I0 and MaxPool1D produce zeros of both
+    signs; kept sets bit-exact against the oracle."""
+    import attention_delta_token_b200 as F
+    rng = np.random.default_rng(41)
+    R, B = 24, 32
+    dims = F.make_dims(R, B, 32, 8, 128, 4096)
+    ws = F.Workspace(dims)
+    dec = (rng.random((R, B)) < 0.25).astype(np.uint8)
+    budget = rng.integers(1, B, size=R).astype(np.int32)
+    dec_g = torch.from_numpy(dec).cuda()
+    bud_g = torch.from_numpy(budget).cuda()
+    cap = F.plan_capacity(torch.from_numpy(dec), torch.from_numpy(budget))
+    # scores drawn from {-0.5, -0.0, +0.0, +0.5}: most cuts fall inside a run of zeros
+    vals = rng.choice(np.array([-0.5, -0.0, 0.0, 0.5], np.float32), size=(R, B))
+    vals[dec != 0] = -np.inf
+    assert (np.signbit(vals) & (vals == 0)).any() and (~np.signbit(vals) & (vals == 0)).any()
+    kept = torch.empty(cap, dtype=torch.int32, device="cuda")
+    cu = torch.empty(R + 1, dtype=torch.int32, device="cuda")
+    F.focus_topk_select(dims, torch.from_numpy(vals).cuda(), dec_g, bud_g, kept, cu, ws)
+    okept, ocu, _ = orc.select(vals.astype(np.float64), dec, budget)
+    np.testing.assert_array_equal(cu.cpu().numpy(), ocu)
+    np.testing.assert_array_equal(kept.cpu().numpy(), okept)
+    # through the delta step: I1 - I0 of equal values is +0.0, of (-0.0) - (+0.0) is -0.0
+    i0 = rng.choice(np.array([0.0, -0.0, 0.25], np.float32), size=(R, B))
+    i1 = rng.choice(np.array([0.0, -0.0, 0.25], np.float32), size=(R, B))
+    delta = torch.empty(R, B, device="cuda")
+    F.focus_importance_delta(dims, torch.from_numpy(i0).cuda(), torch.from_numpy(i1).cuda(),
+                             dec_g, delta)
+    _, pooled = orc.delta_pool_mask(i0.astype(np.float64), i1.astype(np.float64), dec)
+    np.testing.assert_array_equal(delta.cpu().numpy(), pooled.astype(np.float32))  # -0 == +0
+    F.focus_topk_select(dims, delta, dec_g, bud_g, kept, cu, ws)
+    okept, ocu, _ = orc.select(pooled, dec, budget)
+    np.testing.assert_array_equal(cu.cpu().numpy(), ocu)
+    np.testing.assert_array_equal(kept.cpu().numpy(), okept)
+    assert F.focus_read_device_status(ws) == 0
+
+
 def test_zero_budget_and_all_decoded(orc):
     p = synth.make_problem(1, overrides=dict(R=4, prefix=("uniform", 0, 300)))
     p.budget = torch.tensor([0, -5, 3, 40], dtype=torch.int32)

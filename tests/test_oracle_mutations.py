@@ -1,8 +1,9 @@
 """Each plausible mistake planted in a copy of the oracle (on the CPU) must fail at
-least one pin.  A mistake is planted at every place the same expression occurs.  This shows the pins constrain every step the oracle takes:
-scale, softmax denominator, column index, head mapping, query indexing, the
-delta's sign, the pooling window, the mask, the tie-break, the budget clamp,
-the output order and the compaction source row."""
+least one pin.  A mistake is planted at every place the same expression occurs.  This
+shows the pins constrain every step the oracle takes: scale, softmax denominator,
+column index, head mapping, query indexing, the delta's sign, the pooling window, the
+mask, the tie-break (signed zeros included), the budget clamp, the output order and the
+compaction source row."""
 import os
 
 import pytest
@@ -27,6 +28,9 @@ MUTATIONS = {
     "pool_window_asymmetric": ("t <= j + half", "t < j + half"),
     "mask_dropped": ("decoded[(size_t)r * B + j] ? -INFINITY : best", "best"),
     "tie_break_reversed": ("    return a < b;", "    return a > b;"),
+    "signed_zeros_ordered": ("    if (va < vb)\n        return 0;\n    return a < b;",
+                             "    if (va < vb)\n        return 0;\n    if (signbit(va) != signbit(vb))\n"
+                             "        return signbit(vb) != 0;\n    return a < b;"),
     "negative_budget_not_clamped": ("int k = budget[r] < 0 ? 0 : budget[r];", "int k = budget[r];"),
     "output_not_ascending": ("while (t > 0 && chosen[t - 1] > x)", "while (0)"),
     "compact_wrong_source": ("hidden + ((size_t)r * B + j) * H",
