@@ -24,7 +24,9 @@
 //               registers (no second pass over the keys), and their column sums
 //               over the 128 rows (warp butterfly, then the four lane quadrants in
 //               fixed order) go to `partial`.  No float atomics: the result is
-//               deterministic and equal keys give bit-equal columns.
+//               deterministic, and equal keys weighted by the same warpgroup (the
+//               whole block when B <= 64, else each 64-column half) give
+//               bit-equal columns.
 // Split prefixes (small batches only): when the items would fill at most half of
 // the grid, each item's prefix is split into chunks of at least four key tiles,
 // one work item per chunk.  The chunks of an item come consecutively in the list,

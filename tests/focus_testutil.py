@@ -102,17 +102,21 @@ def selection_margin(raw_row, pooled_row, decoded_row, k) -> float:
 
     The k-th largest masked pooled value v_k is the cut.  Pooled values are window
     maxima of the raw delta, so equal values at neighbouring positions are copies of
-    one raw value (and duplicated keys give equal raw values); such exact ties are
-    broken by position identically on both sides.  What can move the cut is another
-    raw value close to v_k, pooled or hidden inside a window, so the margin is the
-    distance from v_k to the nearest raw delta of the block that differs from it;
-    infinite when k is 0 or every masked position is kept.
+    one raw value; such exact ties are broken by position identically on both sides.
+    Two raw positions that both hold exactly v_k (duplicated keys) are a tie of two
+    separately computed values: the rule lets their order differ, so the margin is 0.
+    Otherwise what can move the cut is another raw value close to v_k, pooled or hidden
+    inside a window, so the margin is the distance from v_k to the nearest raw delta of
+    the block that differs from it; infinite when k is 0 or every masked position is
+    kept.
     """
     masked = np.flatnonzero(np.asarray(decoded_row) == 0)
     if k == 0 or k >= masked.size:
         return float("inf")
     vk = np.sort(np.asarray(pooled_row, np.float64)[masked])[::-1][k - 1]
     raw = np.asarray(raw_row, np.float64)
+    if np.count_nonzero(raw == vk) >= 2:
+        return 0.0
     other = raw[raw != vk]
     return float(np.min(np.abs(other - vk))) if other.size else float("inf")
 

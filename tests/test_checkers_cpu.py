@@ -23,6 +23,10 @@ def test_selection_margin_hand_case():
     raw2 = raw.copy()
     raw2[2] = 0.499
     assert selection_margin(raw2, pooled, dec, 3) == pytest.approx(0.001)
+    # two raw positions holding exactly the value at the cut (duplicated keys): a tie
+    raw3 = np.array([0.10, 0.50, 0.20, 0.30, 0.50, 0.00])
+    pooled3 = np.array([0.50, 0.50, 0.50, 0.50, 0.50, 0.50])
+    assert selection_margin(raw3, pooled3, dec, 3) == 0.0
     # nothing to decide: k = 0 or every masked position kept
     assert selection_margin(raw, pooled, dec, 0) == np.inf
     dec2 = np.array([1, 1, 1, 0, 0, 1], np.uint8)
