@@ -159,6 +159,32 @@ __device__ __forceinline__ int item_of_round(int k) {
     return k * g + ((k & 1) ? g - 1 - c : c);
 }
 
+// With at least kDynamicItemsPerCta items per CTA (unsplit kernel) items are claimed
+// dynamically: each CTA starts with item blockIdx.x, and its producer claims item
+// gridDim.x + atomicAdd(counter) two key tiles before the end of its current item, so
+// CTAs take the longest-first list about in the order they become free (a greedy
+// longest-first schedule).  The producer passes each index to the MMA and softmax
+// warps through a ring of kItemSlots shared-memory slots (full: published; empty: read
+// by all nine warps).  With fewer items per CTA the static snake order pairs long and
+// short items as well and costs nothing at the end.
+constexpr int kItemSlots = 4;
+constexpr long long kDynamicItemsPerCta = 4;
+
+// The item a consumer role (the MMA thread, or a softmax warp) takes in its k-th
+// round: from the producer's ring when items are claimed dynamically, else the
+// static snake order.  A wait that gives up returns an index past every item.
+__device__ __forceinline__ int next_item(bool dyn, int k, uint64_t *full, uint64_t *empty,
+                                         volatile int *ring, uint32_t *status,
+                                         volatile int *abort_flag) {
+    if (!dyn) return item_of_round(k);
+    const int slot = k & (kItemSlots - 1);
+    if (!mbar_wait(&full[slot], (k / kItemSlots) & 1, status, abort_flag)) return 0x7fffffff;
+    const int it = ring[slot];
+    __syncwarp(__activemask());  // every participating lane has read the slot
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[slot]);
+    return it;
+}
+
 // One thread waits until the counter reaches `target` (the group's other chunks
 // have published their row statistics).  Bounded: on timeout it sets
 // FOCUS_DEV_TIMEOUT and the abort flag; it also returns when another role aborted.
@@ -227,6 +253,9 @@ template <int HEAD_DIM, bool SPLIT>
 __global__ void __launch_bounds__(kAttnThreads, 2)
 attn_stats_kernel(const __grid_constant__ AttnParams p) {
     using S = AttnSmem<HEAD_DIM>;
+    // Items claimed dynamically (see next_item) when the launch has several per CTA;
+    // split chunks keep the static order their waits rely on.
+    const bool dyn = !SPLIT && p.dynamic;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -241,8 +270,11 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
     uint64_t *s_empty = s_full + 2;        // [2] S buffer read out by the 8 softmax warps
     uint64_t *stat_bar = s_empty + 2;      // both halves' (m, l) of the item are in smem
     uint64_t *red_bar = stat_bar + 1;      // column partial sums of the item are in smem
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(red_bar + 1);
+    uint64_t *item_full = red_bar + 1;     // [kItemSlots] next item index published
+    uint64_t *item_empty = item_full + kItemSlots;  // [kItemSlots] read by MMA + softmax warps
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(item_empty + kItemSlots);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *item_ring = abort_flag + 1;  // [kItemSlots] item indices, in claim order
     float *red = reinterpret_cast<float *>(smem + S::kRedOff);     // [4 quadrants][128 columns]
     float2 *stat = reinterpret_cast<float2 *>(smem + S::kStatOff); // [2 halves][128 rows]
 
@@ -263,6 +295,10 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
         }
         mbar_init(stat_bar, kSoftmaxWarps);
         mbar_init(red_bar, kSoftmaxWarps);
+        for (int q = 0; q < kItemSlots; ++q) {
+            mbar_init(&item_full[q], 1);
+            mbar_init(&item_empty[q], kSoftmaxWarps + 1);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -294,8 +330,23 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
             const uint64_t pol = p.MT == 1 ? l2_policy_evict_first() : l2_policy_evict_normal();
             uint32_t kt = 0;   // key tiles issued by this CTA
             int last_q = -1;   // item count of the last Q load issued
-            int k = 0;
-            for (int it = item_of_round(0); it < n_items; it = item_of_round(++k)) {
+            int next = dyn ? static_cast<int>(blockIdx.x) : item_of_round(0);
+            for (int k = 0;; ++k) {
+                const int it = next;
+                if (dyn) {
+                    // Publish this CTA's k-th item (or the end) to the MMA and softmax warps.
+                    // The next one is claimed two key tiles before this item's last (below).
+                    const int slot = k & (kItemSlots - 1);
+                    if (!mbar_wait(&item_empty[slot], ((k / kItemSlots) & 1) ^ 1, p.status,
+                                   abort_flag))
+                        break;
+                    item_ring[slot] = it;
+                    mbar_arrive(&item_full[slot]);
+                    if (it >= n_items) break;
+                } else {
+                    if (it >= n_items) break;
+                    next = item_of_round(k + 1);
+                }
                 const Item w = decode_item<SPLIT>(p, it);
                 if (w.bad) atomicOr(p.status, FOCUS_DEV_BAD_INPUT);
                 if (!mbar_wait(q_empty, (k & 1) ^ 1, p.status, abort_flag)) break;
@@ -307,6 +358,11 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
                 last_q = k;
                 bool ok = true;
                 for (int i = 0; i < w.n_tiles; ++i, ++kt) {
+                    // Claim late, so CTAs take the longest-first list close to when they
+                    // become free, yet early enough that the atomic's latency stays hidden.
+                    if (dyn && i == (w.n_tiles > 2 ? w.n_tiles - 2 : 0))
+                        next = static_cast<int>(gridDim.x) +
+                               static_cast<int>(atomicAdd(p.item_counter, 1u));
                     const int t = w.t0 + i;                              // prefix tile index
                     const bool blk = w.final && i == w.n_tiles - 1;      // the block tile
                     const int s = kt % kStages;
@@ -365,9 +421,10 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
             const uint32_t a_base = smem_u32(sQ);
             uint32_t kt = 0;  // key tiles consumed
             uint32_t st = 0;  // S tiles produced
-            int k = 0;
             bool ok = true;
-            for (int it = item_of_round(0); ok && it < n_items; it = item_of_round(++k)) {
+            for (int k = 0; ok; ++k) {
+                const int it = next_item(dyn, k, item_full, item_empty, item_ring, p.status, abort_flag);
+                if (it >= n_items) break;
                 const Item w = decode_item<SPLIT>(p, it);
                 if (!mbar_wait(q_full, k & 1, p.status, abort_flag)) break;
                 for (int i = 0; i < w.n_tiles; ++i, ++kt, ++st) {
@@ -409,10 +466,11 @@ attn_stats_kernel(const __grid_constant__ AttnParams p) {
         const float c = p.scale_log2;
         const float2 c2 = make_float2(c, c);
         uint32_t st = 0;
-        int k = 0;
         int kf = 0;  // final chunks done (the reduction barrier completes once per final chunk)
         bool ok = true;
-        for (int it = item_of_round(0); ok && it < n_items; it = item_of_round(++k)) {
+        for (int k = 0; ok; ++k) {
+            const int it = next_item(dyn, k, item_full, item_empty, item_ring, p.status, abort_flag);
+            if (it >= n_items) break;
             const Item w = decode_item<SPLIT>(p, it);
             const int rows_valid = min(kTileRows, p.G * p.B - w.mt * kTileRows);
             float m = -INFINITY;  // running max of the scaled logits (log2 domain), this half
@@ -642,13 +700,15 @@ cudaError_t launch_attn_stats(const AttnParams &p, int head_dim, cudaStream_t st
                             (split ? p.chunk_max : 1);
     if (items <= 0) return cudaSuccess;
     const long long grid = items < 2ll * sm_count() ? items : 2ll * sm_count();
+    AttnParams q = p;
+    q.dynamic = !split && items >= kDynamicItemsPerCta * grid;
     cudaError_t e;
     if (head_dim == 64)
-        e = split ? launch_attn_variant<64, true>(p, grid, stream, pdl)
-                  : launch_attn_variant<64, false>(p, grid, stream, pdl);
+        e = split ? launch_attn_variant<64, true>(q, grid, stream, pdl)
+                  : launch_attn_variant<64, false>(q, grid, stream, pdl);
     else
-        e = split ? launch_attn_variant<128, true>(p, grid, stream, pdl)
-                  : launch_attn_variant<128, false>(p, grid, stream, pdl);
+        e = split ? launch_attn_variant<128, true>(q, grid, stream, pdl)
+                  : launch_attn_variant<128, false>(q, grid, stream, pdl);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

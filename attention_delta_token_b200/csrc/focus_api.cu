@@ -62,7 +62,8 @@ int chunk_max_for(const focus_dims_t &d) {
     return static_cast<int>(c < kMaxChunks ? c : kMaxChunks);
 }
 
-// Workspace: [status 256 B][order: R int32][partial: 2 x R x Hkv x MT x B fp32]
+// Workspace: [status 256 B: the status word; at +64 the exchange counter, at +128 the
+//            attention kernel's item counter][order: R int32][partial: 2 x R x Hkv x MT x B fp32]
 //            [lists: R x B int32][counts: R int32]   (retained positions under constraints)
 //            and with split prefixes (chunk_max_for > 1): [item_base: R+1 int32]
 //            [chunk_cnt: 2 x R x Hkv x MT uint32][chunk_stat: groups x (chunk_max-1) x 256 float2]
@@ -208,6 +209,7 @@ void fill_common(AttnParams &p, const focus_dims_t &d, const int32_t *cu_prefix,
     p.order = reinterpret_cast<const int32_t *>(ws + w.order);
     p.partial = reinterpret_cast<float *>(ws + w.partial);
     p.status = reinterpret_cast<uint32_t *>(ws + w.status);
+    p.item_counter = reinterpret_cast<unsigned int *>(ws + w.status + 128);
     p.total_prefix = total_prefix;
     p.R = d.R;
     p.B = d.B;
@@ -259,9 +261,10 @@ focus_status_t setup_attention(AttnParams &p, const focus_dims_t &d, int layers,
     return FOCUS_OK;
 }
 
-// The planner's share of a split-prefix launch: per-rank item offsets and zeroed
-// chunk counters.
-void plan_split(focus::PlanParams &pp, const AttnParams &p) {
+// The planner's share of an attention launch: the kernel's item counter zeroed and,
+// with split prefixes, per-rank item offsets and zeroed chunk counters.
+void plan_attention(focus::PlanParams &pp, const AttnParams &p) {
+    pp.item_counter = p.item_counter;
     if (p.chunk_max <= 1) return;
     pp.chunk_max = p.chunk_max;
     // With layer 0's log-sum-exps given, its groups have no prefix: one item each.
@@ -382,7 +385,7 @@ focus_status_t focus_attn_stats(const focus_dims_t *dims, const void *q, const v
     pp.status = p.status;
     pp.R = d.R;
     pp.B = d.B;
-    plan_split(pp, p);
+    plan_attention(pp, p);
     FOCUS_CUDA(focus::launch_plan(pp, s));
     FOCUS_CUDA(launch_attn_traced(p, d.head_dim, s));
     focus::ReduceParams rp{p.partial, importance, d.R, d.B, d.Hkv, p.MT, 1};
@@ -689,7 +692,7 @@ focus_status_t evict_impl(const focus_dims_t *dims, const focus_evict_args_t &x)
     pp.capacity = x.capacity;
     pp.R = d.R;
     pp.B = d.B;
-    plan_split(pp, p);
+    plan_attention(pp, p);
     FOCUS_CUDA(focus::launch_plan(pp, s));
     FOCUS_CUDA(launch_attn_traced(p, d.head_dim, s, /*pdl=*/true));
 
@@ -731,7 +734,7 @@ focus_status_t partial_importance_impl(const focus_dims_t *dims, const void *q0,
     pp.status = p.status;
     pp.R = d.R;
     pp.B = d.B;
-    plan_split(pp, p);
+    plan_attention(pp, p);
     FOCUS_CUDA(focus::launch_plan(pp, s));
     FOCUS_CUDA(launch_attn_traced(p, d.head_dim, s, /*pdl=*/true));
     focus::ReduceParams rp;

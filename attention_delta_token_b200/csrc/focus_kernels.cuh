@@ -50,6 +50,8 @@ struct AttnParams {
     const int32_t *order;      // [R] request processing order (longest prefix first)
     float *partial;            // [n_layers][R][Hkv][MT][B] column sums per kv head / row tile
     uint32_t *status;          // device status word
+    unsigned int *item_counter;  // items claimed after the first round (zeroed by the planner)
+    int dynamic;               // claim items dynamically (set at launch from the item count)
     long long total_prefix;
     int R, B, Hq, Hkv, G, MT, n_layers;
     int tok_per_tile;          // 128 / G block tokens per row tile
@@ -106,6 +108,7 @@ struct PlanParams {
     int chunk_max, per_req, single_groups, n_groups;
     int32_t *item_base;        // [R+1]
     unsigned int *chunk_cnt;   // [n_groups]
+    unsigned int *item_counter;  // the attention kernel's item counter, zeroed (or null)
 };
 cudaError_t launch_plan(const PlanParams &p, cudaStream_t stream);
 

@@ -111,6 +111,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
     __shared__ int warp_tot[33];
     const int R = p.R;
     pdl_launch_dependents();  // the attention kernel may set up while this runs
+    if (threadIdx.x == 0 && p.item_counter) *p.item_counter = 0u;
 
     if (p.order && R <= kRankSortR) {
         // Rank of each request under (L desc, r asc): a plain count, no sort passes.
