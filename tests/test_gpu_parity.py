@@ -204,6 +204,25 @@ def test_deterministic_full_ragged_workload():
         np.testing.assert_array_equal(a[k], b[k], err_msg=k)
 
 
+def test_results_do_not_depend_on_the_schedule():
+    """A request's outputs are the same bits whichever schedule processed it: the metric
+    workload (4,096 attention items, claimed dynamically by the CTAs) against 32 and 48 of its
+    requests run alone (512 and 768 items: the static order), which also changes which CTA
+    takes which item and when."""
+    p = synth.make_problem(2, wide_logits=True)
+    full = run_evict(p.to("cuda"))
+    for req in (list(range(0, 256, 8)), list(range(3, 256, 5))[:48]):
+        sub = run_evict(p.subset(req).to("cuda"))
+        for key in ("i0", "i1", "delta"):
+            np.testing.assert_array_equal(full[key][req], sub[key], err_msg=key)
+        cu_f, cu_s = full["cu_seqlens"], sub["cu_seqlens"]
+        for t, r in enumerate(req):
+            np.testing.assert_array_equal(full["kept"][cu_f[r]:cu_f[r + 1]],
+                                          sub["kept"][cu_s[t]:cu_s[t + 1]], err_msg=str(r))
+            np.testing.assert_array_equal(full["packed"][cu_f[r]:cu_f[r + 1]],
+                                          sub["packed"][cu_s[t]:cu_s[t + 1]], err_msg=str(r))
+
+
 def test_consecutive_denoising_steps_vs_oracle(orc):
     """One workspace and one set of output buffers across five denoising steps, as an
     engine would use them: after each step a few of the kept (still-masked) tokens become
