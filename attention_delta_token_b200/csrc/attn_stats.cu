@@ -8,8 +8,9 @@
 // keys followed by its B block keys; I_j also sums over the query heads.
 //
 // Work item = one (layer, request, kv head, 128-row query tile).  The kernel is
-// persistent: two CTAs per SM, each taking one item per round from the list
-// (longest prefix first), in snake order across the grid.  Per CTA (10 warps):
+// persistent: two CTAs per SM take items from the list (longest prefix first),
+// claimed dynamically from a counter when there are at least four per CTA, else
+// one per round in snake order across the grid.  Per CTA (10 warps):
 //   warp 0      TMA producer: the item's Q tile (once per item, as soon as the
 //               previous item's MMAs have released it), then 128-key tiles of the
 //               prefix and finally the block keys, through a 2-stage ring;
