@@ -206,12 +206,14 @@ def test_deterministic_full_ragged_workload():
 
 def test_results_do_not_depend_on_the_schedule():
     """A request's outputs are the same bits whichever schedule processed it: the metric
-    workload (4,096 attention items, claimed dynamically by the CTAs) against 32 and 48 of its
-    requests run alone (512 and 768 items: the static order), which also changes which CTA
-    takes which item and when."""
+    workload (4,096 attention items, claimed dynamically by the CTAs) against 32, 48 and 73 of
+    its requests run alone (512, 768 and 1,168 items: the static order) and 74 of them (1,184
+    items, exactly four per CTA: dynamic again), which also changes which CTA takes which item
+    and when."""
     p = synth.make_problem(2, wide_logits=True)
     full = run_evict(p.to("cuda"))
-    for req in (list(range(0, 256, 8)), list(range(3, 256, 5))[:48]):
+    for req in (list(range(0, 256, 8)), list(range(3, 256, 5))[:48], list(range(73)),
+                list(range(100, 174))):
         sub = run_evict(p.subset(req).to("cuda"))
         for key in ("i0", "i1", "delta"):
             np.testing.assert_array_equal(full[key][req], sub[key], err_msg=key)
