@@ -144,8 +144,9 @@ FOCUS_API focus_status_t focus_plan_capacity(const focus_dims_t *dims, const uin
                                              int64_t *capacity_out);
 
 /* Zero the workspace's status region (enqueued on `stream`): the device status
- * word and the peer exchange's block counter.  Call once before the first use of
- * a workspace and whenever the status should restart. */
+ * word, the peer exchange's block counter and the attention kernel's item counter
+ * (which every call that runs the attention kernel also resets first).  Call once
+ * before the first use of a workspace and whenever the status should restart. */
 FOCUS_API focus_status_t focus_clear_device_status(void *workspace, size_t workspace_bytes, void *stream);
 
 /*
